@@ -1,0 +1,445 @@
+#!/usr/bin/env python3
+"""Benchmark of libkda's KDA hot path on B200; prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload prefill_8k|varlen_prologue|long_256k|decode_256x32] [--no-rows]
+
+Headline (default workload prefill_8k: B=1, H=32, T=8192, dk=dv=128, bf16 I/O, fp32
+gates/beta/state, chunk 64): prefill tokens/s of kda_chunk_fwd with inputs resident in
+HBM, timed per step with CUDA events on the launching stream, L2 flushed between steps.
+`e2e` is the same metric through the C ABI with pinned HOST buffers (host->device copy of
+the step's inputs and device->host copy of o and the final state inside the timed region).
+`rows` adds the other steps of the path measured in the same run: the conv prologue on
+the packed 64-sequence workload and the decode step on 256 x 32 states.
+Under torchrun (N > 1) every rank runs its own replica (weak scaling, no collective on
+the data path); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (H=32,d=128) & decode GB/s; % of roofline on 1×B200"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# Algorithmic bytes per token*head of the prefill (d = 128, bf16 q/k/v/o, fp32 g, beta):
+# q, k, v in (3 * 256) + o out (256) + g (512) + beta (4) = 1540; plus h0/ht once per state.
+def prefill_bytes(T_tot, H, dk, dv, N, io_bytes=2, h0=False, ht=True):
+    per_tok = H * ((2 * dk + 2 * dv) * io_bytes + 4 * dk + 4)
+    state = N * H * dk * dv * 4
+    return T_tot * per_tok + state * (int(h0) + int(ht))
+
+
+def prefill_flops(T_tot, H, dk, dv, C=64):
+    # 6 dk dv (Qhat S, W S, Ktilde^T Ut) + C (3 dk + 2 dv) (A, P, W, U, intra-chunk O) + C^2/3
+    return T_tot * H * (6 * dk * dv + C * (3 * dk + 2 * dv) + C * C / 3)
+
+
+def decode_bytes(N, H, dk, dv, io_bytes=2):
+    return N * H * (2 * dk * dv * 4 + (2 * dk + 2 * dv) * io_bytes + 4 * dk + 4)
+
+
+def conv_bytes(T_tot, H, dk, dv, io_bytes=2):
+    return T_tot * H * (2 * dk + dv) * io_bytes * 2
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons of this process's GPU during a region."""
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9 or (self.uuid and self.uuid not in parts[0]):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+# CPU oracle arm                                                               #
+# --------------------------------------------------------------------------- #
+
+def oracle_prefill_rate(min_seconds=10.0, max_reps=50):
+    """Times the fp64 oracle on the prefill_8k workload (all 32 heads x 8192 tokens) on the
+    host cores; repeats whole passes until min_seconds. Returns (tokens/s, cores, sample)."""
+    import oracle
+    from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_prefill
+    d = make_prefill(WORKLOADS["prefill_8k"], "cpu")
+    f64 = lambda t: t.double().numpy()       # noqa: E731
+    args = [f64(d[n]) for n in ("q", "k", "v", "g", "beta")]
+    cores = os.cpu_count() or 1
+    oracle.load()
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.kda_fwd(*args, 1.0, None, d["cu_host"], nthreads=cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            break
+    tokens = reps * d["T_tot"]
+    sample = (f"{reps} full pass(es) of prefill_8k (B=1,H=32,T=8192,dk=dv=128) through the "
+              f"fp64 token-by-token oracle, parallel over heads on {cores} threads, {el:.1f} s")
+    return tokens / el, cores, sample, el / reps
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rate, cores, sample, sec_per_pass = None, None, None, None
+    import oracle
+    from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_prefill
+    d = make_prefill(WORKLOADS["prefill_8k"], "cpu")
+    f64 = lambda t: t.double().numpy()       # noqa: E731
+    a = [f64(d[n]) for n in ("q", "k", "v", "g", "beta")]
+    cores = os.cpu_count() or 1
+    oracle.load()
+    for _ in range(args.warmup):
+        oracle.kda_fwd(*a, 1.0, None, d["cu_host"], nthreads=cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.kda_fwd(*a, 1.0, None, d["cu_host"], nthreads=cores)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    rate = args.steps * d["T_tot"] / total
+    sample = (f"each step: one full pass of prefill_8k (B=1,H=32,T=8192,dk=dv=128) through the "
+              f"fp64 token-by-token oracle on {cores} host threads")
+    line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prefill_8k: B=1,H=32,T=8192,dk=dv=128,chunk 64"},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- #
+# GPU arm                                                                      #
+# --------------------------------------------------------------------------- #
+
+def _events_time(torch, fn, steps, warmup, flush=None, stream=None):
+    """Per-step device time (ms) with CUDA events on `stream`; `flush` runs between steps,
+    outside the timed events."""
+    stream = stream or torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from kimi_delta_attention_32_b200 import kda
+    from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_decode, make_prefill
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (libkda has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    kda.load_library()
+    peaks, peaks_src = load_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+
+    l2_flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def flush():
+        l2_flush.fill_(1)
+
+    wl = WORKLOADS[args.workload]
+    stream = torch.cuda.current_stream()
+    launches_per_step = 1
+    rows = {}
+
+    if args.workload == "decode_256x32":
+        d = make_decode(wl, dev, steps=max(1, args.steps + args.warmup))
+        state = d["h0"].clone()
+        N, H, dk, dv = d["N"], d["H"], d["dk"], d["dv"]
+        qn = torch.nn.functional.normalize(d["q_raw"].float(), dim=-1).to(d["q_raw"].dtype)
+        kn = torch.nn.functional.normalize(d["k_raw"].float(), dim=-1).to(d["k_raw"].dtype)
+        it = iter(range(10 ** 9))
+
+        def step():
+            s = next(it) % d["steps"]
+            kda.recurrent_step(qn[s], kn[s], d["v_raw"][s], d["g"][s], d["beta"][s], state,
+                               stream=stream)
+        units = N        # tokens per step (one per sequence), over H heads
+        algo_bytes = decode_bytes(N, H, dk, dv)
+        wl_desc = (f"decode_256x32: N={N} sequences x H={H}, fp32 state {dk}x{dv}, bf16 q/k/v/o, "
+                   "one token per sequence per step")
+        flops = N * H * 7 * dk * dv
+        dtype = "f32"
+    else:
+        d = make_prefill(wl, dev)
+        T_tot, N, H, dk, dv = d["T_tot"], d["N"], d["H"], d["dk"], d["dv"]
+        if wl.prologue:
+            q, k, v = kda.conv_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["w_q"], d["w_k"],
+                                   d["w_v"], cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"])
+        else:
+            q, k, v = d["q"], d["k"], d["v"]
+        o = torch.empty_like(v)
+        ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+
+        def step():
+            kda.chunk_fwd(q, k, v, d["g"], d["beta"], 1.0, h0=d["h0"], ht=ht, o=o,
+                          cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], stream=stream)
+        units = T_tot
+        algo_bytes = prefill_bytes(T_tot, H, dk, dv, N, h0=d["h0"] is not None)
+        wl_desc = {"prefill_8k": "prefill_8k: B=1,H=32,T=8192,dk=dv=128,bf16 q/k/v/o,fp32 g/beta/"
+                                 "state,chunk 64,zero h0,final state returned",
+                   "varlen_prologue": f"varlen_prologue: 64 packed sequences U[128,16384] "
+                                      f"(T_tot={T_tot}),H=32,dk=dv=128,bf16,h0~N(0,0.02) "
+                                      "(timed: chunked prefill on the prologue's outputs)",
+                   "long_256k": "long_256k: B=1,H=32,T=262144,dk=dv=128,bf16,skewed gates"
+                   }.get(args.workload, args.workload)
+        flops = prefill_flops(T_tot, H, dk, dv)
+        dtype = "f32" if wl.io == "f32" else "bf16-io/f32"
+
+    uuid = ""
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(uuid) as clk:
+        times = _events_time(torch, step, args.steps, 0, flush=flush, stream=stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = sum(times)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    value = units * world * args.steps / (ms_total / 1e3)
+    achieved = algo_bytes / (statistics.mean(times) / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None,
+                "algorithmic_bytes_per_launch": algo_bytes,
+                "peak_source": f"{peaks_src} hbm_gbs",
+                "flop_term_frac": (flops / (statistics.mean(times) / 1e3) / 1e12)
+                / float(peaks["bf16_tflops"])}
+
+    # ---------------- e2e through the C ABI with pinned host buffers ----------------
+    e2e = None
+    if args.workload != "decode_256x32" and not args.no_e2e:
+        names = ["q", "k", "v", "g", "beta"]
+        host = {}
+        srcs = {"q": q, "k": k, "v": v, "g": d["g"], "beta": d["beta"]}
+        for nm in names:
+            host[nm] = torch.empty(srcs[nm].shape, dtype=srcs[nm].dtype, pin_memory=True)
+            host[nm].copy_(srcs[nm])
+        dbuf = {nm: torch.empty_like(srcs[nm]) for nm in names}
+        o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        ht_host = torch.empty(ht.shape, dtype=ht.dtype, pin_memory=True)
+        h2d = sum(host[nm].numel() * host[nm].element_size() for nm in names)
+        d2h = o_host.numel() * o_host.element_size() + ht_host.numel() * ht_host.element_size()
+
+        def e2e_step():
+            for nm in names:
+                dbuf[nm].copy_(host[nm], non_blocking=True)
+            kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], 1.0,
+                          h0=d["h0"], ht=ht, o=o, cu_seqlens=d["cu_seqlens"],
+                          cu_host=d["cu_host"], stream=stream)
+            o_host.copy_(o, non_blocking=True)
+            ht_host.copy_(ht, non_blocking=True)
+        et = _events_time(torch, e2e_step, max(2, args.steps // 2), 2, stream=stream)
+        ems = sum(et)
+        if world > 1:
+            tt = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": units * world * len(et) / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ems / len(et)}
+
+    # ---------------- other rows of the path, same run ----------------
+    if not args.no_rows and args.workload == "prefill_8k":
+        rows = measure_rows(torch, kda, dev, flush, hbm_peak, stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, cores, sample, _ = oracle_prefill_rate() if args.workload == "prefill_8k" else \
+            (None, None, None, None)
+        if rate is not None:
+            cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": sample}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+            "data": "synthetic (seeded, device-generated)",
+            "config": {"workload": wl_desc, "parallelism": f"replicas x{world}" if world > 1
+                       else "1 GPU", "l2": "flushed (256 MiB write) between timed steps"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(), "rows": rows}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure_rows(torch, kda, dev, flush, hbm_peak, stream):
+    """Conv prologue (packed 64-sequence workload) and decode step (256 x 32 states)."""
+    from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_decode, make_prefill
+    out = {}
+    wl = WORKLOADS["varlen_prologue"]
+    d = make_prefill(wl, dev)
+    qo, ko, vo = (torch.empty_like(d[n]) for n in ("q_raw", "k_raw", "v_raw"))
+
+    def conv():
+        kda.conv_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["w_q"], d["w_k"], d["w_v"], qo, ko, vo,
+                     cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], stream=stream)
+    t = _events_time(torch, conv, 5, 2, flush=flush, stream=stream)
+    b = conv_bytes(d["T_tot"], d["H"], d["dk"], d["dv"])
+    ms = statistics.mean(t)
+    out["a1_conv_prologue"] = {"workload": f"varlen_prologue raw q/k/v (T_tot={d['T_tot']},H=32,"
+                                           "d=128,bf16)", "ms": ms, "GB/s": b / ms / 1e6,
+                               "frac_hbm": b / ms / 1e6 / hbm_peak,
+                               "tokens/s": d["T_tot"] / ms * 1e3}
+    del d, qo, ko, vo
+    torch.cuda.empty_cache()
+
+    wl = WORKLOADS["decode_256x32"]
+    steps = 16
+    dd = make_decode(wl, dev, steps=steps)
+    qn = torch.nn.functional.normalize(dd["q_raw"].float(), dim=-1).to(dd["q_raw"].dtype)
+    kn = torch.nn.functional.normalize(dd["k_raw"].float(), dim=-1).to(dd["k_raw"].dtype)
+    state = dd["h0"].clone()
+    cache = dd["conv_state"].clone()
+    it = iter(range(10 ** 9))
+
+    def dec():
+        s = next(it) % steps
+        kda.recurrent_step(qn[s], kn[s], dd["v_raw"][s], dd["g"][s], dd["beta"][s], state,
+                           stream=stream)
+    t = _events_time(torch, dec, 20, 3, flush=flush, stream=stream)
+    b = decode_bytes(wl.N, wl.H, wl.dk, wl.dv)
+    ms = statistics.mean(t)
+    it2 = iter(range(10 ** 9))
+
+    def pair():
+        s = next(it2) % steps
+        x = [dd[n][s].unsqueeze(1) for n in ("q_raw", "k_raw", "v_raw")]
+        qq, kk, vv = kda.conv_fwd(*x, dd["w_q"], dd["w_k"], dd["w_v"], conv_state=cache,
+                                  stream=stream)
+        kda.recurrent_step(qq[:, 0], kk[:, 0], vv[:, 0], dd["g"][s], dd["beta"][s], state,
+                           stream=stream)
+    tp = _events_time(torch, pair, 20, 3, flush=flush, stream=stream)
+    out["a5_decode_step"] = {"workload": "decode_256x32: 256 seq x 32 heads, fp32 128x128 state",
+                             "ms": ms, "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm_peak,
+                             "tokens/s": wl.N / ms * 1e3,
+                             "conv_plus_step_ms": statistics.mean(tp)}
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill_8k",
+                    choices=["prefill_8k", "varlen_prologue", "long_256k", "decode_256x32"])
+    ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,166 @@
+/*
+ * kda.h -- C ABI of libkda, a B200 (sm_100a) implementation of the Kimi Delta
+ * Attention (KDA) linear-attention core.
+ *
+ * What the operations compute comes from pages about the AliceAI-Foundation-
+ * 80B-A3B-Base model:
+ *  - sarnas.ru, "Яндекс открыл веса AliceAI-Foundation-80B-A3B-Base: MoE-модель,
+ *    обученная с нуля", section "Что именно изменилось": KDA keeps a fixed-size
+ *    state; for each token it reads the value the state holds for the token's
+ *    key, compares it with the new value and writes back only the difference;
+ *    it forgets with one coefficient per state row (Gated DeltaNet has one
+ *    coefficient for the whole state).
+ *  - m.lqnn.cn/news/205170, section "KDA 与 Gated Attention：每 4 层只留 1 层
+ *    全注意力": q/k/v first pass a kernel-4 causal convolution with a cache that
+ *    is advanced per step; the recurrence is state = state * exp(gate) + delta
+ *    with delta = prediction residual x sigmoid(beta); beta in (0, 1).
+ *  - m.lqnn.cn/news/255115, section "二、第一关：配置文件": the conv kernel is at
+ *    least 2 and the chunk size positive.
+ *
+ * Per (sequence, head), with state S (dk x dv, row i = key channel i) and token t:
+ *     S   <- diag(exp(g_t)) S                       per-row forgetting
+ *     u_t  = v_t - S^T k_t                          read-out and residual
+ *     S   <- S + beta_t k_t u_t^T                   write only the correction
+ *     o_t  = scale * S^T q_t                        output from the updated state
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are caller-owned DEVICE memory, 16-byte aligned,
+ *    row-major and dense. Host pointers are marked "host".
+ *  - Token-major layouts: q, k, g : [T_tot, H, dk];  v, o : [T_tot, H, dv];
+ *    beta : [T_tot, H];  state : [N, H, dk, dv] fp32.
+ *  - io selects the element type of q, k, v, o (and of the conv tensors):
+ *    KDA_IO_F32 (float) or KDA_IO_BF16 (__nv_bfloat16). g, beta, state and conv
+ *    weights are always fp32.
+ *  - Batches: padded (cu_seqlens == NULL): B sequences of T tokens each, so
+ *    N = B and T_tot = B*T; packed (cu_seqlens != NULL): N sequences, sequence n
+ *    is tokens [cu[n], cu[n+1]), T_tot = cu[N]; cu_seqlens (device, int32 [N+1])
+ *    and cu_seqlens_host (host copy) must both be given and hold the same values.
+ *  - stream is a cudaStream_t (NULL = the legacy default stream). Every call is
+ *    asynchronous on it; results are valid once the stream has been synchronised.
+ *    The library allocates nothing, frees nothing and never synchronises (except
+ *    kda_last_device_error, which says so).
+ *  - Errors: arguments are checked on the host before anything is launched; a
+ *    failing check launches nothing and returns KDA_ERR_INVALID_ARG or
+ *    KDA_ERR_UNSUPPORTED. A launch failure returns KDA_ERR_CUDA. No call aborts
+ *    or throws. Preconditions that are NOT checked: g <= 0, beta in (0, 1),
+ *    finite inputs, and that cu_seqlens matches cu_seqlens_host.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* a null, misaligned, negative or inconsistent argument */
+    KDA_ERR_UNSUPPORTED = 2,   /* a valid size this build has no kernel for */
+    KDA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the query says */
+    KDA_ERR_CUDA = 4,          /* a CUDA runtime error while launching */
+    KDA_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (see kda_last_device_error) */
+} kda_status;
+
+typedef enum { KDA_IO_F32 = 0, KDA_IO_BF16 = 1 } kda_io_dtype;
+
+/* Static English text for a status; never NULL. */
+const char* kda_status_string(kda_status status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int kda_version(void);
+
+/*
+ * kda_conv_fwd -- fused short causal depthwise convolution + SiLU (+ L2 norm of q, k).
+ * (m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...": kernel-4 causal
+ *  conv of q, k and v with a cache advanced per step; m.lqnn.cn/news/255115,
+ *  section "二、第一关：配置文件": kernel >= 2.)
+ *
+ * For each channel c of x in {q_raw, k_raw, v_raw} (channel c = h*d + i):
+ *     y[t, c] = silu( sum_{j=0}^{K-1} w[c, j] * x[t-(K-1)+j, c] ),  silu(z) = z / (1 + e^-z)
+ * where positions before a sequence's first token read the conv history of
+ * that sequence (conv_state, oldest first) or zero when conv_state is NULL.
+ * Then each dk-vector of the q and k outputs is divided by sqrt(sum y^2 + l2_eps).
+ * No bias. The conv never crosses a sequence boundary.
+ *
+ *  q_raw, k_raw : [T_tot, H, dk] io dtype      v_raw : [T_tot, H, dv] io dtype
+ *  w_q, w_k     : [H*dk, K] fp32               w_v   : [H*dv, K] fp32 (tap K-1 = current token)
+ *  q_out, k_out, v_out : same shapes as the inputs; must not overlap any input.
+ *  conv_state   : [N, H*(2*dk+dv), K-1] io dtype, channels ordered q, then k, then v,
+ *                 or NULL. In: the K-1 raw inputs preceding each sequence (oldest
+ *                 first). Out (overwritten in place): the last K-1 raw inputs of the
+ *                 history followed by this call's tokens. Decode is the padded
+ *                 case with T == 1.
+ *  Supported: dk, dv in {64, 128}; K == 4; io F32 or BF16.
+ */
+kda_status kda_conv_fwd(const void* q_raw, const void* k_raw, const void* v_raw,
+                        const float* w_q, const float* w_k, const float* w_v,
+                        void* q_out, void* k_out, void* v_out, void* conv_state,
+                        const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                        int B, int T, int N, int H, int dk, int dv, int K, float l2_eps,
+                        kda_io_dtype io, void* stream);
+
+/*
+ * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd needs
+ * for these sizes (written to *bytes, host). Zero means none; the call then
+ * accepts workspace == NULL.
+ */
+kda_status kda_chunk_fwd_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, int chunk,
+                                        kda_io_dtype io, size_t* bytes);
+
+/*
+ * kda_chunk_fwd -- chunked prefill of the KDA recurrence over a padded or packed batch.
+ * (sarnas.ru, section "Что именно изменилось"; m.lqnn.cn/news/205170, section
+ *  "KDA 与 Gated Attention ..."; chunk > 0 from m.lqnn.cn/news/255115.)
+ *
+ * Computes, for every token, exactly the per-token recurrence above; the chunk
+ * length only changes the order of the arithmetic (the result is the same up to
+ * rounding). o[t] = scale * S_t^T q_t with S_t the state after token t.
+ *
+ *  q, k : [T_tot, H, dk] io dtype   v : [T_tot, H, dv] io dtype   o : [T_tot, H, dv] io dtype
+ *  g    : [T_tot, H, dk] fp32 per-channel log-decay (<= 0)
+ *  beta : [T_tot, H] fp32 write strength in (0, 1)
+ *  scale: multiplies the output (1.0 for no scaling)
+ *  h0   : [N, H, dk, dv] fp32 initial states, or NULL for zero states
+ *  ht   : [N, H, dk, dv] fp32 final states, or NULL to skip; may alias h0
+ *  chunk: tokens per chunk; this build supports 64.
+ *  Supported: dk == dv in {64, 128} for io F32; dk == dv == 128 or 64 for BF16.
+ *  Empty sequences are allowed (their final state is the initial state).
+ */
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, float scale, const float* h0, float* ht, void* o,
+                         const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                         int B, int T, int N, int H, int dk, int dv, int chunk,
+                         kda_io_dtype io, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * kda_recurrent_step -- one decode token per (sequence, head), state updated in place.
+ * (sarnas.ru, section "Что именно изменилось"; m.lqnn.cn/news/205170, section
+ *  "KDA 与 Gated Attention ...": the per-token loop state = state*exp(gate)+delta.)
+ *
+ *  q, k : [N, H, dk] io dtype   v, o : [N, H, dv] io dtype
+ *  g    : [N, H, dk] fp32   beta : [N, H] fp32
+ *  state: [N, H, dk, dv] fp32, read and overwritten with the state after the token.
+ *  o    : must not overlap any input.
+ *  Supported: dk, dv in {64, 128}.
+ */
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, float scale, float* state, void* o,
+                              int N, int H, int dk, int dv, kda_io_dtype io, void* stream);
+
+/*
+ * kda_last_device_error -- synchronises `stream`, then returns and clears the
+ * device-side error word that kernels set when a bounded wait gives up
+ * (KDA_ERR_TIMEOUT) -- KDA_OK if none. Returns KDA_ERR_CUDA if the stream
+ * reports a CUDA error.
+ */
+kda_status kda_last_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

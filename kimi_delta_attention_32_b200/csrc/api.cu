@@ -1,0 +1,163 @@
+// api.cu -- the C ABI of libkda: argument checks, then the kernel launches.
+// Checks mirror the model's hard configuration validation (m.lqnn.cn/news/255115,
+// section "二、第一关：配置文件": conv kernel >= 2, chunk size > 0, head counts
+// that divide) and the library's own layout rules; nothing is launched when a
+// check fails.
+#include "kda.h"
+
+#include <stdint.h>
+
+#define KDA_API extern "C" __attribute__((visibility("default")))
+
+#include "common.cuh"
+#include "launchers.h"
+
+namespace kda {
+__device__ unsigned int g_device_error = 0;
+}
+
+namespace {
+
+constexpr int kVersion = 100;   // 0.1.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+bool ok_req(const void* p) { return p != nullptr && aligned16(p); }
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+// Resolves padded/packed batch geometry; returns false on inconsistent input.
+bool batch_geometry(const int32_t* cu, const int32_t* cu_host, int B, int T, int N,
+                    int64_t* T_tot, int* N_out) {
+    if ((cu == nullptr) != (cu_host == nullptr)) return false;
+    if (cu == nullptr) {
+        if (B < 0 || T < 0) return false;
+        *T_tot = (int64_t)B * T;
+        *N_out = B;
+        return true;
+    }
+    if (N < 0 || cu_host[0] != 0) return false;
+    for (int n = 0; n < N; ++n)
+        if (cu_host[n + 1] < cu_host[n]) return false;
+    *T_tot = cu_host[N];
+    *N_out = N;
+    return true;
+}
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+}  // namespace
+
+KDA_API const char* kda_status_string(kda_status status) {
+    switch (status) {
+        case KDA_OK: return "ok";
+        case KDA_ERR_INVALID_ARG: return "invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "unsupported size or option";
+        case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+        case KDA_ERR_CUDA: return "CUDA error";
+        case KDA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+KDA_API int kda_version(void) { return kVersion; }
+
+KDA_API kda_status kda_conv_fwd(const void* q_raw, const void* k_raw, const void* v_raw,
+                        const float* w_q, const float* w_k, const float* w_v,
+                        void* q_out, void* k_out, void* v_out, void* conv_state,
+                        const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                        int B, int T, int N, int H, int dk, int dv, int K, float l2_eps,
+                        kda_io_dtype io, void* stream) {
+    if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
+    if (H <= 0 || dk <= 0 || dv <= 0 || K < 2 || !(l2_eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+    int64_t T_tot = 0;
+    int Nn = 0;
+    if (!batch_geometry(cu_seqlens, cu_seqlens_host, B, T, N, &T_tot, &Nn)) return KDA_ERR_INVALID_ARG;
+    const void* req[] = {q_raw, k_raw, v_raw, w_q, w_k, w_v, q_out, k_out, v_out};
+    for (const void* p : req)
+        if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
+    if (!ok_opt(conv_state) || !ok_opt(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    if (K != 4 || !head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    kda::ConvArgs a;
+    a.x[0] = q_raw; a.x[1] = k_raw; a.x[2] = v_raw;
+    a.w[0] = w_q; a.w[1] = w_k; a.w[2] = w_v;
+    a.y[0] = q_out; a.y[1] = k_out; a.y[2] = v_out;
+    a.conv_state = conv_state;
+    a.cu = cu_seqlens;
+    a.T_tot = T_tot;
+    a.T_pad = cu_seqlens ? 0 : T;
+    a.N = Nn; a.H = H; a.dk = dk; a.dv = dv;
+    a.eps = l2_eps;
+    a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
+    return from_cuda(kda::launch_conv(a, static_cast<cudaStream_t>(stream)));
+}
+
+KDA_API kda_status kda_chunk_fwd_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, int chunk,
+                                        kda_io_dtype io, size_t* bytes) {
+    if (bytes == nullptr || N < 0 || T_tot < 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0)
+        return KDA_ERR_INVALID_ARG;
+    if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
+    *bytes = 0;
+    return KDA_OK;
+}
+
+KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, float scale, const float* h0, float* ht, void* o,
+                         const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                         int B, int T, int N, int H, int dk, int dv, int chunk,
+                         kda_io_dtype io, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
+    if (H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0) return KDA_ERR_INVALID_ARG;
+    int64_t T_tot = 0;
+    int Nn = 0;
+    if (!batch_geometry(cu_seqlens, cu_seqlens_host, B, T, N, &T_tot, &Nn)) return KDA_ERR_INVALID_ARG;
+    const void* req[] = {q, k, v, g, beta, o};
+    for (const void* p : req)
+        if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
+    if (!ok_opt(h0) || !ok_opt(ht) || !ok_opt(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    if (chunk != 64 || dk != dv || !head_dim_ok(dk)) return KDA_ERR_UNSUPPORTED;
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.scale = scale;
+    a.h0 = h0; a.ht = ht; a.o = o;
+    a.cu = cu_seqlens; a.cu_host = cu_seqlens_host;
+    a.T_tot = T_tot;
+    a.T_pad = cu_seqlens ? 0 : T;
+    a.N = Nn; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk;
+    a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
+    return from_cuda(kda::launch_chunk_simt(a, static_cast<cudaStream_t>(stream)));
+}
+
+KDA_API kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, float scale, float* state, void* o,
+                              int N, int H, int dk, int dv, kda_io_dtype io, void* stream) {
+    if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    const void* req[] = {q, k, v, g, beta, state, o};
+    for (const void* p : req)
+        if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    kda::StepArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.scale = scale;
+    a.state = state; a.o = o;
+    a.N = N; a.H = H; a.dk = dk; a.dv = dv;
+    a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
+    return from_cuda(kda::launch_recurrent_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+KDA_API kda_status kda_last_device_error(void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, kda::g_device_error, sizeof(word)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(kda::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        return KDA_ERR_TIMEOUT;
+    }
+    return KDA_OK;
+}
+

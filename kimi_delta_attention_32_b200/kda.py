@@ -1,0 +1,182 @@
+"""Thin ctypes binding of libkda (the C ABI in include/kda.h).
+
+Argument marshalling only: every step of the computation runs in libkda's CUDA
+kernels. Tensors are torch CUDA tensors (torch provides device memory and
+streams); the current torch stream is passed unless one is given. If libkda.so
+is missing this module raises on first use -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, \
+    KDA_ERR_TIMEOUT = range(6)
+KDA_IO_F32, KDA_IO_BF16 = 0, 1
+
+EXPORTED = ("kda_status_string", "kda_version", "kda_conv_fwd", "kda_chunk_fwd_workspace_size",
+            "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: status {status} ({msg})")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libkda.so and declare its signatures. Raises if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is not None and path == LIB_PATH:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"libkda.so not found at {path}; build it with "
+                               "`python -m kimi_delta_attention_32_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, i32p, fp = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+        ci, cf, cs = ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.kda_status_string.argtypes = [ci]
+        lib.kda_status_string.restype = ctypes.c_char_p
+        lib.kda_version.argtypes = []
+        lib.kda_version.restype = ci
+        lib.kda_conv_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, vp, vp, i32p,
+                                     ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci, ci,
+                                     cf, ci, vp]
+        lib.kda_conv_fwd.restype = ci
+        lib.kda_chunk_fwd_workspace_size.argtypes = [ci, ctypes.c_int64, ci, ci, ci, ci, ci,
+                                                     ctypes.POINTER(cs)]
+        lib.kda_chunk_fwd_workspace_size.restype = ci
+        lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, cf, fp, fp, vp, i32p,
+                                      ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci, ci,
+                                      ci, vp, cs, vp]
+        lib.kda_chunk_fwd.restype = ci
+        lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, cf, fp, vp, ci, ci, ci, ci, ci, vp]
+        lib.kda_recurrent_step.restype = ci
+        lib.kda_last_device_error.argtypes = [vp]
+        lib.kda_last_device_error.restype = ci
+        if path == LIB_PATH:
+            _lib = lib
+        return lib
+
+
+def _check(fn: str, status: int):
+    if status != KDA_OK:
+        raise KdaError(fn, status, load_library().kda_status_string(status).decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _io(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_IO_BF16
+    if t.dtype == torch.float32:
+        return KDA_IO_F32
+    raise TypeError(f"unsupported I/O dtype {t.dtype}")
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _host_cu(cu_host):
+    if cu_host is None:
+        return None, None
+    arr = (ctypes.c_int32 * len(cu_host))(*[int(x) for x in cu_host])
+    return arr, ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
+
+
+def conv_fwd(q_raw, k_raw, v_raw, w_q, w_k, w_v, q_out=None, k_out=None, v_out=None,
+             conv_state=None, cu_seqlens=None, cu_host=None, l2_eps=1e-6, K=4, stream=None):
+    """Fused causal conv (kernel K) + SiLU + L2 norm of q, k. Shapes: x [T_tot,H,d] for the
+    packed form (cu_seqlens given) or [B,T,H,d] for the padded form. Returns (q, k, v)."""
+    lib = load_library()
+    q_out = torch.empty_like(q_raw) if q_out is None else q_out
+    k_out = torch.empty_like(k_raw) if k_out is None else k_out
+    v_out = torch.empty_like(v_raw) if v_out is None else v_out
+    if cu_seqlens is None:
+        B, T, H, dk = q_raw.shape if q_raw.dim() == 4 else (1, *q_raw.shape)
+        N = B
+    else:
+        B, T = 1, 0
+        _, H, dk = q_raw.shape
+        N = len(cu_host) - 1
+    dv = v_raw.shape[-1]
+    keep, cuh = _host_cu(cu_host)
+    st = lib.kda_conv_fwd(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(w_q), _ptr(w_k), _ptr(w_v),
+                          _ptr(q_out), _ptr(k_out), _ptr(v_out), _ptr(conv_state),
+                          _ptr(cu_seqlens), cuh, B, T, N, H, dk, dv, K, float(l2_eps),
+                          _io(q_raw), _stream(stream))
+    del keep
+    _check("kda_conv_fwd", st)
+    return q_out, k_out, v_out
+
+
+def chunk_fwd_workspace_size(N, T_tot, H, dk, dv, chunk=64, io=KDA_IO_BF16) -> int:
+    lib = load_library()
+    out = ctypes.c_size_t(0)
+    _check("kda_chunk_fwd_workspace_size",
+           lib.kda_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, chunk, io, ctypes.byref(out)))
+    return out.value
+
+
+def chunk_fwd(q, k, v, g, beta, scale=1.0, h0=None, ht=None, o=None, cu_seqlens=None,
+              cu_host=None, chunk=64, output_final_state=True, workspace=None, stream=None):
+    """Chunked prefill. Packed: q [T_tot,H,dk] with cu_seqlens (device int32) and cu_host
+    (list); padded: q [B,T,H,dk]. Returns (o, ht) (ht None if not requested)."""
+    lib = load_library()
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape if q.dim() == 4 else (1, *q.shape)
+        N = B
+        T_tot = B * T
+    else:
+        B, T = 1, 0
+        T_tot, H, dk = q.shape
+        N = len(cu_host) - 1
+    dv = v.shape[-1]
+    o = torch.empty_like(v) if o is None else o
+    if ht is None and output_final_state:
+        ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    io = _io(q)
+    need = chunk_fwd_workspace_size(N, T_tot, H, dk, dv, chunk, io)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    keep, cuh = _host_cu(cu_host)
+    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(h0),
+                           _ptr(ht), _ptr(o), _ptr(cu_seqlens), cuh, B, T, N, H, dk, dv, chunk,
+                           io, _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                           _stream(stream))
+    del keep
+    _check("kda_chunk_fwd", st)
+    return o, ht
+
+
+def recurrent_step(q, k, v, g, beta, state, scale=1.0, o=None, stream=None):
+    """One decode token per (sequence, head); q,k,g [N,H,dk], v [N,H,dv], beta [N,H],
+    state [N,H,dk,dv] fp32 updated in place. Returns o [N,H,dv]."""
+    lib = load_library()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty_like(v) if o is None else o
+    st = lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                _ptr(state), _ptr(o), N, H, dk, dv, _io(q), _stream(stream))
+    _check("kda_recurrent_step", st)
+    return o
+
+
+def last_device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device-side error status."""
+    return load_library().kda_last_device_error(_stream(stream))

@@ -1,0 +1,141 @@
+"""CPU tests of the C ABI: the library loads, exports every function kda.h declares,
+and rejects bad arguments on the host before anything is launched."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from kimi_delta_attention_32_b200 import build as kbuild
+from kimi_delta_attention_32_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "kda.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted(kda.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libkda.so does not export {name}"
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.kda_status_string(s)
+    assert lib.kda_status_string(99) == b"unknown status"
+    assert lib.kda_version() >= 100
+
+
+FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: checks fail first
+MIS = ctypes.c_void_p(0x10004)           # misaligned
+
+
+def _chunk(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, scale=1.0, h0=None, ht=None, o=FAKE,
+             cu=None, cuh=None, B=1, T=64, N=1, H=2, dk=128, dv=128, chunk=64, io=1, ws=None,
+             wsb=0, stream=None)
+    a.update(kw)
+    return lib.kda_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["scale"], a["h0"],
+                             a["ht"], a["o"], a["cu"], a["cuh"], a["B"], a["T"], a["N"], a["H"],
+                             a["dk"], a["dv"], a["chunk"], a["io"], a["ws"], a["wsb"],
+                             a["stream"])
+
+
+def _cu_host(vals):
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return arr, ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(o=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(k=MIS), kda.KDA_ERR_INVALID_ARG),
+    (dict(h0=MIS), kda.KDA_ERR_INVALID_ARG),
+    (dict(chunk=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(chunk=-64), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(io=7), kda.KDA_ERR_INVALID_ARG),
+    (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dk=96, dv=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dk=128, dv=64), kda.KDA_ERR_UNSUPPORTED),
+])
+def test_chunk_fwd_rejects(lib, kw, status):
+    assert _chunk(lib, **kw) == status
+
+
+def test_chunk_fwd_rejects_bad_cu_seqlens(lib):
+    keep, cuh = _cu_host([0, 5, 3])                      # not monotone
+    assert _chunk(lib, cu=FAKE, cuh=cuh, N=2) == kda.KDA_ERR_INVALID_ARG
+    keep, cuh = _cu_host([1, 5, 9])                      # does not start at 0
+    assert _chunk(lib, cu=FAKE, cuh=cuh, N=2) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, cu=FAKE, cuh=None, N=2) == kda.KDA_ERR_INVALID_ARG   # host copy missing
+    keep, cuh = _cu_host([0, 5, 9])
+    assert _chunk(lib, cu=None, cuh=cuh, N=2) == kda.KDA_ERR_INVALID_ARG    # device copy missing
+    del keep
+
+
+def _conv(lib, **kw):
+    a = dict(x=FAKE, w=FAKE, y=FAKE, cs=None, cu=None, cuh=None, B=2, T=16, N=2, H=2, dk=128,
+             dv=128, K=4, eps=1e-6, io=1)
+    a.update(kw)
+    return lib.kda_conv_fwd(a["x"], a["x"], a["x"], a["w"], a["w"], a["w"], a["y"], a["y"],
+                            a["y"], a["cs"], a["cu"], a["cuh"], a["B"], a["T"], a["N"], a["H"],
+                            a["dk"], a["dv"], a["K"], a["eps"], a["io"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=1), kda.KDA_ERR_INVALID_ARG),           # conv kernel must be >= 2
+    (dict(K=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(x=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(w=MIS), kda.KDA_ERR_INVALID_ARG),
+    (dict(cs=MIS), kda.KDA_ERR_INVALID_ARG),
+    (dict(eps=-1.0), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=-2), kda.KDA_ERR_INVALID_ARG),
+    (dict(K=3), kda.KDA_ERR_UNSUPPORTED),
+    (dict(K=2), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dk=32), kda.KDA_ERR_UNSUPPORTED),
+])
+def test_conv_fwd_rejects(lib, kw, status):
+    assert _conv(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(state=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(q=MIS), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dv=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=256), kda.KDA_ERR_UNSUPPORTED),
+])
+def test_recurrent_step_rejects(lib, kw, status):
+    a = dict(q=FAKE, state=FAKE, N=4, H=2, dk=128, dv=128)
+    a.update(kw)
+    st = lib.kda_recurrent_step(a["q"], FAKE, FAKE, FAKE, FAKE, 1.0, a["state"], FAKE, a["N"],
+                                a["H"], a["dk"], a["dv"], 1, None)
+    assert st == status
+
+
+def test_workspace_query(lib):
+    out = ctypes.c_size_t(123)
+    assert lib.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 128, 64, 1, ctypes.byref(out)) == 0
+    assert lib.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 128, 0, 1, ctypes.byref(out)) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 128, 64, 1, None) == \
+        kda.KDA_ERR_INVALID_ARG
