@@ -24,8 +24,9 @@
  *     o_t  = scale * S^T q_t                        output from the updated state
  *
  * Conventions shared by every call
- *  - All tensor pointers are caller-owned DEVICE memory, 16-byte aligned,
- *    row-major and dense. Host pointers are marked "host".
+ *  - All tensor pointers are caller-owned DEVICE memory, row-major and dense,
+ *    16-byte aligned except beta (4-byte aligned is enough). Host pointers are
+ *    marked "host".
  *  - Token-major layouts: q, k, g : [T_tot, H, dk];  v, o : [T_tot, H, dv];
  *    beta : [T_tot, H];  state : [N, H, dk, dv] fp32.
  *  - io selects the element type of q, k, v, o (and of the conv tensors):

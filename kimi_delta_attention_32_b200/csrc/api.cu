@@ -21,6 +21,7 @@ namespace {
 constexpr int kVersion = 100;   // 0.1.0
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 bool ok_req(const void* p) { return p != nullptr && aligned16(p); }
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
@@ -113,9 +114,10 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
     int64_t T_tot = 0;
     int Nn = 0;
     if (!batch_geometry(cu_seqlens, cu_seqlens_host, B, T, N, &T_tot, &Nn)) return KDA_ERR_INVALID_ARG;
-    const void* req[] = {q, k, v, g, beta, o};
+    const void* req[] = {q, k, v, g, o};
     for (const void* p : req)
         if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
+    if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
     if (!ok_opt(h0) || !ok_opt(ht) || !ok_opt(cu_seqlens)) return KDA_ERR_INVALID_ARG;
     if (chunk != 64 || dk != dv || !head_dim_ok(dk)) return KDA_ERR_UNSUPPORTED;
     kda::ChunkArgs a;
@@ -134,9 +136,10 @@ KDA_API kda_status kda_recurrent_step(const void* q, const void* k, const void* 
                               int N, int H, int dk, int dv, kda_io_dtype io, void* stream) {
     if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
-    const void* req[] = {q, k, v, g, beta, state, o};
+    const void* req[] = {q, k, v, g, state, o};
     for (const void* p : req)
         if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
+    if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
     kda::StepArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.scale = scale;
