@@ -46,6 +46,13 @@ bool batch_geometry(const int32_t* cu, const int32_t* cu_host, int B, int T, int
 
 kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
+// Device address of the error word on the current device.
+unsigned int* device_error_word() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, kda::g_device_error) != cudaSuccess) return nullptr;
+    return static_cast<unsigned int*>(p);
+}
+
 }  // namespace
 
 KDA_API const char* kda_status_string(kda_status status) {
@@ -128,6 +135,11 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
     a.T_pad = cu_seqlens ? 0 : T;
     a.N = Nn; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk;
     a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
+    if (kda::chunk_tc_supported(a)) {
+        unsigned int* err = device_error_word();
+        if (err == nullptr) return KDA_ERR_CUDA;
+        return from_cuda(kda::launch_chunk_tc(a, err, static_cast<cudaStream_t>(stream)));
+    }
     return from_cuda(kda::launch_chunk_simt(a, static_cast<cudaStream_t>(stream)));
 }
 
