@@ -224,12 +224,28 @@ def run_ours(args):
     def flush():
         l2_flush.fill_(1)
 
-    wl = WORKLOADS[args.workload]
+    wl = WORKLOADS.get(args.workload, WORKLOADS["prefill_8k"])
     stream = torch.cuda.current_stream()
     launches_per_step = 1
     rows = {}
 
-    if args.workload == "decode_256x32":
+    if args.workload == "conv_8k":
+        # conv prologue alone on prefill_8k-shaped raw inputs (B=1, H=32, T=8192, d=128, bf16)
+        import dataclasses
+        cw = dataclasses.replace(WORKLOADS["varlen_prologue"], N=1, varlen=(), T=8192, h0_std=0.0)
+        d = make_prefill(cw, dev)
+        qo, ko, vo = (torch.empty_like(d[n]) for n in ("q_raw", "k_raw", "v_raw"))
+
+        def step():
+            kda.conv_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["w_q"], d["w_k"], d["w_v"], qo, ko,
+                         vo, cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], stream=stream)
+        units = d["T_tot"]
+        algo_bytes = conv_bytes(d["T_tot"], d["H"], d["dk"], d["dv"])
+        wl_desc = "conv_8k: conv+SiLU+L2 prologue on B=1,H=32,T=8192,dk=dv=128 raw bf16 q/k/v"
+        flops = 0
+        dtype = "bf16-io/f32"
+        args.no_e2e = True
+    elif args.workload == "decode_256x32":
         d = make_decode(wl, dev, steps=max(1, args.steps + args.warmup))
         state = d["h0"].clone()
         N, H, dk, dv = d["N"], d["H"], d["dk"], d["dv"]
@@ -429,7 +445,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill_8k",
-                    choices=["prefill_8k", "varlen_prologue", "long_256k", "decode_256x32"])
+                    choices=["prefill_8k", "varlen_prologue", "long_256k", "decode_256x32",
+                             "conv_8k"])
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -6,6 +6,8 @@
 #include "kda.h"
 
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #define KDA_API extern "C" __attribute__((visibility("default")))
 
@@ -45,6 +47,13 @@ bool batch_geometry(const int32_t* cu, const int32_t* cu_host, int B, int T, int
 }
 
 kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// Tensor-core prefill variant: the 4-CTA cluster pipeline unless KDA_CHUNK_KERNEL=single
+// selects the one-CTA-per-(sequence, head) kernel.
+bool use_cluster_prefill() {
+    const char* e = getenv("KDA_CHUNK_KERNEL");
+    return !(e != nullptr && strcmp(e, "single") == 0);
+}
 
 // Device address of the error word on the current device.
 unsigned int* device_error_word() {
@@ -138,7 +147,9 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
     if (kda::chunk_tc_supported(a)) {
         unsigned int* err = device_error_word();
         if (err == nullptr) return KDA_ERR_CUDA;
-        return from_cuda(kda::launch_chunk_tc(a, err, static_cast<cudaStream_t>(stream)));
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        return from_cuda(use_cluster_prefill() ? kda::launch_chunk_tcx(a, err, st)
+                                               : kda::launch_chunk_tc(a, err, st));
     }
     return from_cuda(kda::launch_chunk_simt(a, static_cast<cudaStream_t>(stream)));
 }
@@ -175,4 +186,3 @@ KDA_API kda_status kda_last_device_error(void* stream) {
     }
     return KDA_OK;
 }
-

@@ -92,4 +92,20 @@ __device__ __forceinline__ int find_seq(const int32_t* cu, int N, int64_t t) {
     return lo;
 }
 
+// Phase timestamps for performance work: a no-op unless the library is built with
+// -DKDA_TRACE, which records %globaltimer (ns) for the first cluster's CTAs into
+// g_trace[cta][chunk][mark] of the including translation unit.
+#ifdef KDA_TRACE
+static __device__ unsigned long long g_trace[4][512][16];
+__device__ __forceinline__ void trace_mark(int cta, int chunk, int mark) {
+    if (threadIdx.x == 0 && blockIdx.x < 4 && chunk < 512) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        g_trace[cta][chunk][mark] = t;
+    }
+}
+#else
+__device__ __forceinline__ void trace_mark(int, int, int) {}
+#endif
+
 }  // namespace kda

@@ -40,21 +40,69 @@ struct ConvParams {
     int step_mode;       // one token per sequence: read and write the cache here
 };
 
+// Register image of CPL consecutive elements of type T (8 or 16 bytes), and its unpacking.
+template <typename T, int CPL>
+struct RawVec;
+template <>
+struct RawVec<__nv_bfloat16, 4> {
+    using Word = uint2;
+    static __device__ __forceinline__ void unpack(const Word& w, float* o) {
+        o[0] = __uint_as_float(w.x << 16); o[1] = __uint_as_float(w.x & 0xffff0000u);
+        o[2] = __uint_as_float(w.y << 16); o[3] = __uint_as_float(w.y & 0xffff0000u);
+    }
+};
+template <>
+struct RawVec<__nv_bfloat16, 2> {
+    using Word = uint32_t;
+    static __device__ __forceinline__ void unpack(const Word& w, float* o) {
+        o[0] = __uint_as_float(w << 16); o[1] = __uint_as_float(w & 0xffff0000u);
+    }
+};
+template <>
+struct RawVec<float, 4> {
+    using Word = uint4;
+    static __device__ __forceinline__ void unpack(const Word& w, float* o) {
+        o[0] = __uint_as_float(w.x); o[1] = __uint_as_float(w.y);
+        o[2] = __uint_as_float(w.z); o[3] = __uint_as_float(w.w);
+    }
+};
+template <>
+struct RawVec<float, 2> {
+    using Word = uint2;
+    static __device__ __forceinline__ void unpack(const Word& w, float* o) {
+        o[0] = __uint_as_float(w.x); o[1] = __uint_as_float(w.y);
+    }
+};
+
 template <typename T, int D>
 __device__ __forceinline__ void conv_unit(const ConvParams& p, int z, int h, int64_t t0) {
     constexpr int CPL = D / 32;
+    using Word = typename RawVec<T, CPL>::Word;
     const int lane = threadIdx.x & 31;
-    const T* __restrict__ x = static_cast<const T*>(p.x[z]);
-    T* __restrict__ y = static_cast<T*>(p.y[z]);
+    // selects rather than p.x[z]: indexing the parameter arrays at run time would copy them
+    // to local memory
+    const T* __restrict__ x = static_cast<const T*>(z == 0 ? p.x[0] : z == 1 ? p.x[1] : p.x[2]);
+    T* __restrict__ y = static_cast<T*>(z == 0 ? p.y[0] : z == 1 ? p.y[1] : p.y[2]);
+    const float* wz = z == 0 ? p.w[0] : z == 1 ? p.w[1] : p.w[2];
     T* cache = static_cast<T*>(p.conv_state);
     const int H = p.H;
     const int cl = lane * CPL;                                    // channel within the head
     const int cstate = (z == 0 ? 0 : z == 1 ? H * p.dk : 2 * H * p.dk) + h * D + cl;
+    const int64_t t1 = t0 + kTile < p.T_tot ? t0 + kTile : p.T_tot;
+    const int ntok = (int)(t1 - t0);
 
+    // Issue every load of the tile first: the three tokens before it and its kTile tokens.
+    Word raw[kHist + kTile];
+#pragma unroll
+    for (int m = 0; m < kHist + kTile; ++m) {
+        const int64_t t = t0 - kHist + m;
+        raw[m] = Word{};
+        if (t >= 0 && t < t1) raw[m] = *reinterpret_cast<const Word*>(x + (t * H + h) * D + cl);
+    }
     float w[CPL][kTaps];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
-        const float4 wv = *reinterpret_cast<const float4*>(p.w[z] + (int64_t)(h * D + cl + c) * kTaps);
+        const float4 wv = *reinterpret_cast<const float4*>(wz + (int64_t)(h * D + cl + c) * kTaps);
         w[c][0] = wv.x; w[c][1] = wv.y; w[c][2] = wv.z; w[c][3] = wv.w;
     }
 
@@ -70,44 +118,43 @@ __device__ __forceinline__ void conv_unit(const ConvParams& p, int z, int h, int
         eos = bos + p.T_pad;
     }
 
-    // hist[m] = input at position t-3+m (m = 0 oldest).
+    // hist[m] = input at position t-3+m (m = 0 oldest) of the current sequence.
     float hist[kHist][CPL];
-    auto load_hist = [&](int64_t t) {
-#pragma unroll
-        for (int m = 0; m < kHist; ++m) {
-            const int64_t tp = t - kHist + m;
-            if (tp >= bos) {
-                Vec<T, CPL>::load(x + (tp * H + h) * D + cl, hist[m]);
-            } else if (cache) {
-                const int slot = kHist - (int)(bos - tp);           // oldest first
-#pragma unroll
-                for (int c = 0; c < CPL; ++c)
-                    hist[m][c] = to_f32(cache[((int64_t)n * p.Ctot + cstate + c) * kHist + slot]);
-            } else {
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) hist[m][c] = 0.f;
-            }
-        }
-    };
-    load_hist(t0);
-
     const bool norm = (z < 2);
-    const int64_t t1 = t0 + kTile < p.T_tot ? t0 + kTile : p.T_tot;
-    for (int64_t t = t0; t < t1; ++t) {
-        if (t >= eos) {                       // crossed into the next non-empty sequence
-            if (p.cu) {
-                do { ++n; } while (p.cu[n + 1] <= t);
-                bos = p.cu[n];
-                eos = p.cu[n + 1];
-            } else {
-                ++n;
-                bos = eos;
-                eos = bos + p.T_pad;
+#pragma unroll
+    for (int tt = 0; tt < kTile; ++tt) {
+        if (tt >= ntok) break;
+        const int64_t t = t0 + tt;
+        if (tt == 0 || t >= eos) {
+            if (t >= eos) {                       // crossed into the next non-empty sequence
+                if (p.cu) {
+                    do { ++n; } while (p.cu[n + 1] <= t);
+                    bos = p.cu[n];
+                    eos = p.cu[n + 1];
+                } else {
+                    ++n;
+                    bos = eos;
+                    eos = bos + p.T_pad;
+                }
             }
-            load_hist(t);
+#pragma unroll
+            for (int m = 0; m < kHist; ++m) {
+                const int64_t tp = t - kHist + m;
+                if (tp >= bos) {
+                    RawVec<T, CPL>::unpack(raw[tt + m], hist[m]);
+                } else if (cache) {
+                    const int slot = kHist - (int)(bos - tp);           // oldest first
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c)
+                        hist[m][c] = to_f32(cache[((int64_t)n * p.Ctot + cstate + c) * kHist + slot]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) hist[m][c] = 0.f;
+                }
+            }
         }
         float xt[CPL], out[CPL];
-        Vec<T, CPL>::load(x + (t * H + h) * D + cl, xt);
+        RawVec<T, CPL>::unpack(raw[kHist + tt], xt);
         float ss = 0.f;
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
@@ -115,9 +162,9 @@ __device__ __forceinline__ void conv_unit(const ConvParams& p, int z, int h, int
             zc = fmaf(w[c][1], hist[1][c], zc);
             zc = fmaf(w[c][2], hist[2][c], zc);
             zc = fmaf(w[c][3], xt[c], zc);
-            const float s = zc / (1.f + expf(-zc));
-            out[c] = s;
-            ss = fmaf(s, s, ss);
+            const float sv = zc / (1.f + __expf(-zc));
+            out[c] = sv;
+            ss = fmaf(sv, sv, ss);
         }
         if (norm) {
             ss = warp_sum(ss);
@@ -170,7 +217,7 @@ __global__ void conv_cache_kernel(const ConvParams p) {
     else if (c < 2 * p.H * p.dk) { z = 1; ch = c - p.H * p.dk; D = p.dk; }
     else { z = 2; ch = c - 2 * p.H * p.dk; D = p.dv; }
     (void)D;
-    const T* x = static_cast<const T*>(p.x[z]);
+    const T* x = static_cast<const T*>(z == 0 ? p.x[0] : z == 1 ? p.x[1] : p.x[2]);
     T* cs = static_cast<T*>(p.conv_state) + idx * kHist;
     const int rowlen = (z < 2 ? p.dk : p.dv) * p.H;           // channels per token of x[z]
     T old[kHist], nw[kHist];

@@ -154,3 +154,168 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 }  // namespace tc
 }  // namespace kda
+
+namespace kda {
+namespace tc {
+
+// ---- thread-block clusters and distributed shared memory ----
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster16(uint32_t addr, uint4 v) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                 ::"r"(cluster_addr) : "memory");
+}
+// Wait with cluster-scope acquire (pairs with mbar_arrive_remote), bounded.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity,
+                                                          long long limit_cycles) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (clock64() - t0 > limit_cycles) return false;
+    }
+    return true;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+__device__ __forceinline__ void fence_async_cluster() {
+    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+
+// ---- 16-byte asynchronous global -> shared copy (zero-fills when src_bytes == 0) ----
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* gptr, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 ::"r"(saddr), "l"(gptr), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+}  // namespace tc
+}  // namespace kda
+
+namespace kda {
+namespace tc {
+
+// One lane of a converged warp returns true (tcgen05.mma / commit issue).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(pred));
+    return pred != 0;
+}
+// Issued by every lane of one converged warp: one lane issues the MMA.
+__device__ __forceinline__ void warp_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    if (elect_one()) mma_bf16(d_tmem, adesc, bdesc, idesc, accumulate);
+    __syncwarp();
+}
+__device__ __forceinline__ void warp_commit(uint64_t* bar) {
+    if (elect_one()) mma_commit(bar);
+    __syncwarp();
+}
+// Descriptor advanced by a byte offset (the start address field is in 16-byte units).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// Remote arrive that also announces `bytes` of incoming transactions on a peer's mbarrier.
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_addr, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
+                 ::"r"(cluster_addr), "r"(bytes) : "memory");
+}
+// Bulk copy from this CTA's shared memory into a peer's, completing on the peer's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                                  uint32_t mbar_cluster) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst_cluster), "r"(src_cta), "r"(bytes), "r"(mbar_cluster) : "memory");
+}
+
+}  // namespace tc
+}  // namespace kda
+
+namespace kda {
+namespace tc {
+
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// ---- warp-level 16x16 fp32 block products on the tensor cores (TF32 inputs, fp32 sums) ----
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// acc (two 16x8 accumulator fragments) += A (16x16, row stride lda) * B (16x16, row stride ldb).
+// Every lane of the warp takes part.
+__device__ __forceinline__ void warp_block_mma16(float (*acc)[4], const float* A, int lda,
+                                                 const float* B, int ldb) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < 16; kk += 8) {
+        uint32_t a[4];
+        a[0] = to_tf32(A[g * lda + kk + t]);
+        a[1] = to_tf32(A[(g + 8) * lda + kk + t]);
+        a[2] = to_tf32(A[g * lda + kk + t + 4]);
+        a[3] = to_tf32(A[(g + 8) * lda + kk + t + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t b[2];
+            b[0] = to_tf32(B[(kk + t) * ldb + 8 * nt + g]);
+            b[1] = to_tf32(B[(kk + t + 4) * ldb + 8 * nt + g]);
+            mma_tf32_16x8x8(acc[nt], a, b);
+        }
+    }
+}
+// Writes scale * acc (two 16x8 fragments) to a 16x16 fp32 block with row stride ld.
+__device__ __forceinline__ void warp_block_store16(float* C, int ld, const float (*acc)[4], float scale) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        C[g * ld + 8 * nt + 2 * t] = scale * acc[nt][0];
+        C[g * ld + 8 * nt + 2 * t + 1] = scale * acc[nt][1];
+        C[(g + 8) * ld + 8 * nt + 2 * t] = scale * acc[nt][2];
+        C[(g + 8) * ld + 8 * nt + 2 * t + 1] = scale * acc[nt][3];
+    }
+}
+
+}  // namespace tc
+}  // namespace kda

@@ -132,6 +132,35 @@ def test_chunk_varlen_ragged(io, d_head):
     check_prefill(d, d["q"], d["k"], d["v"], o, ht)
 
 
+@pytest.mark.parametrize("variant", ["cluster", "single"])
+@pytest.mark.parametrize("lens", [[300, 1, 64], [129, 700]])
+def test_chunk_extreme_decay_takes_exact_path(variant, lens, monkeypatch):
+    """Channels decaying by ~e^-4 per token push the half-chunk decay far past e^-80, so
+    those chunks form A and P exactly on CUDA cores; the result must still match."""
+    monkeypatch.setenv("KDA_CHUNK_KERNEL", variant)
+    wl = small("prefill_8k", N=len(lens), H=2, io="bf16", h0_std=0.02, seed=36)
+    d = make_prefill(wl, DEV, lengths=lens)
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(37)
+    u = torch.randn(d["g"].shape, generator=gen, device=DEV) - 4.0
+    strong = torch.nn.functional.logsigmoid(u)
+    d["g"][:, :, :16] = strong[:, :, :16]          # 16 of 128 channels per head
+    o, ht = run_chunk(d)
+    torch.cuda.synchronize()
+    check_prefill(d, d["q"], d["k"], d["v"], o, ht)
+
+
+@pytest.mark.parametrize("variant", ["cluster", "single"])
+def test_chunk_variants_match_oracle(variant, monkeypatch):
+    monkeypatch.setenv("KDA_CHUNK_KERNEL", variant)
+    lens = [1, 63, 64, 65, 0, 130, 7, 200, 1000]
+    wl = small("prefill_8k", N=len(lens), H=3, io="bf16", h0_std=0.02, seed=38)
+    d = make_prefill(wl, DEV, lengths=lens)
+    o, ht = run_chunk(d)
+    torch.cuda.synchronize()
+    check_prefill(d, d["q"], d["k"], d["v"], o, ht)
+
+
 def test_chunk_padded_equals_packed():
     wl = small("prefill_8k", N=3, H=2, T=100, io="bf16", h0_std=0.02, seed=32)
     d = make_prefill(wl, DEV)
