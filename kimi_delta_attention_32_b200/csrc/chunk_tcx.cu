@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "launchers.h"
 #include "tc.cuh"
+#include "tma_host.h"
 
 namespace kda {
 namespace {
@@ -52,29 +53,34 @@ __device__ __forceinline__ SlotMap slot_map(int slot) {
 }
 constexpr uint32_t S_TP = 57344;      // T'   : B, K-major rows token r, K = token i
 constexpr uint32_t S_VT = 65536;      // V^T  : A, MN-major, K = token, M = value ch (2 blocks)
-constexpr uint32_t S_FAC = 81920;     // eRef[128], eC[128], eCR[128] (fp32)
+constexpr uint32_t kFacBytes = 1536;  // per chunk: eRef[128], eC[128], eCR[128] (fp32)
 constexpr uint32_t C_SLOT0 = 0;
 constexpr uint32_t C_ST = 2 * kSlotBytes;       // Sm  : A, K-major rows value ch, K = key ch (2 atom cols)
 constexpr uint32_t C_UT = C_ST + 32768;         // Ut^T: A, K-major rows value ch, K = token
-constexpr uint32_t C_MISC = C_UT + 16384;
+constexpr uint32_t C_FAC = C_UT + 16384;        // factor ring: chunk n in entry n % 3, so a
+                                                // ring slot can be released before they are read
+constexpr uint32_t C_MISC = C_FAC + 3 * kFacBytes;
 // ---- producer shared memory ----
 constexpr uint32_t P_XQ = 0;          // raw q [64][128] bf16
 constexpr uint32_t P_XK = 16384;      // raw k [64][128] bf16
-constexpr uint32_t P_XG = 32768;      // raw g / gamma [64][128] f32
-constexpr uint32_t P_LK = 65536;      // Lk: first M block of the A|P A operand; K-major A of Z
-constexpr uint32_t P_HS = 81920;      // two hand-off sets (alternate tasks), each:
+constexpr uint32_t P_LK = 32768;      // Lk: first M block of the A|P A operand; K-major A of Z
+constexpr uint32_t P_HS = 49152;      // two hand-off sets (alternate tasks), each:
 constexpr uint32_t H_LQ = 0;          //   Lq (second M block of the A|P A operand)
 constexpr uint32_t H_RT = 16384;      //   R
-constexpr uint32_t H_TP = 32768;      //   T'
-constexpr uint32_t H_PO = 40960;      //   P
-constexpr uint32_t H_FAC = 49152;     //   eRef, eC, eCR
-constexpr uint32_t kHsBytes = 51200;
-constexpr uint32_t kHandoffTx = 16384 + 16384 + 8192 + 8192 + 1536;   // bytes bulk-copied per chunk
-constexpr uint32_t P_SCR = P_HS + 2 * kHsBytes;   // Nm [64][68], Tm [64][68], Y [3][16][24] (fp32)
+constexpr uint32_t H_ZO = 32768;      //   Z (exact path: A in fp32 until the inverse starts)
+constexpr uint32_t H_TP = 49152;      //   T'
+constexpr uint32_t H_PO = 57344;      //   P
+constexpr uint32_t H_FAC = 65536;     //   eRef, eC, eCR
+constexpr uint32_t kHsBytes = 67584;
+constexpr uint32_t kHandoffTx = 16384 * 3 + 8192 * 2 + 1536;   // bytes bulk-copied per chunk
+constexpr uint32_t P_SCR = P_HS + 2 * kHsBytes;   // raw g / gamma [64][128] f32, then
+                                                  // Nm [64][68], Tm [64][68], Y [3][16][24] (fp32)
+constexpr uint32_t P_XG = P_SCR;
 constexpr uint32_t P_MISC = P_SCR + 40960;
-constexpr uint32_t kMiscBytes = 1536;
+constexpr uint32_t kMiscBytes = 2560;   // barriers, beta[64], decay sums [4][128]
 constexpr uint32_t kSmemBytes = (P_MISC > C_MISC ? P_MISC : C_MISC) + kMiscBytes + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(320 + 4 * 128 * 4 <= kMiscBytes, "misc area");
 
 // misc area (relative to the role's misc base)
 constexpr uint32_t M_BAR_MMA = 0;     // own MMA completions
@@ -82,14 +88,18 @@ constexpr uint32_t M_BAR_A = 8;       // consumer: full[0]; producer: free
 constexpr uint32_t M_BAR_B = 16;      // consumer: full[1]
 constexpr uint32_t M_TMEM = 24;
 constexpr uint32_t M_TMP = 32;
+constexpr uint32_t M_BAR_C = 40;      // producer: q, k tiles landed; consumer: V tile of slot 0
+constexpr uint32_t M_BAR_D = 48;      // producer: g tile landed;    consumer: V tile of slot 1
 constexpr uint32_t M_BETA = 64;       // producer: beta[64]
-constexpr uint32_t M_GSUM = 320;      // producer: [2][128]
+constexpr uint32_t M_GSUM = 320;      // producer: [4][128] token-quarter decay sums
 
 // consumer TMEM columns: [X0 | O0 | S(128) | .. | O1 | X1]; producer: [A|P | Z]
 constexpr uint32_t TC_X0 = 0, TC_O0 = 64, TC_S = 128, TC_O1 = 256, TC_X1 = 320, kTmemC = 512;
 constexpr uint32_t TP_AP = 0, TP_Z = 64, kTmemP = 128;
 
 struct Params {
+    CUtensorMap tq, tk, tg, tv, to;   // TMA maps: q, k, o [T,H,128] bf16 and g [T,H,128] f32 in
+                                      // (128, 1, 64) boxes; v in (64, 1, 64) boxes, 128B swizzle
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
     const __nv_bfloat16* v;
@@ -162,6 +172,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
 
     const uint32_t c_misc = map_to_rank(sb + C_MISC, 0);
     const uint32_t c_slot0 = map_to_rank(sb + C_SLOT0, 0);
+    const uint32_t c_fac = map_to_rank(sb + C_FAC, 0);
 
     auto wait_mma = [&]() -> bool {
         const bool ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitCycles);
@@ -169,27 +180,37 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         if (!ok) atomicOr(p.err, kErrTimeout);
         return __syncthreads_or(!ok) == 0;
     };
-    auto issue_loads = [&](int64_t c0, int L) {
-        for (int e = tid; e < kC * 16; e += kThreads) {
-            const int r = e >> 4, jj = e & 15;
-            const bool ok = r < L;
-            const int64_t off = ok ? ((c0 + r) * H + h) * kD + jj * 8 : 0;
-            cp_async16(sb + P_XQ + r * 256 + jj * 16, p.q + off, ok ? 16u : 0u);
-            cp_async16(sb + P_XK + r * 256 + jj * 16, p.k + off, ok ? 16u : 0u);
+    // Raw q, k tiles (staging, free after the folds) and g tile (in the inverse's scratch,
+    // free once T' is written) of a chunk, by TMA from one thread. Rows past the sequence are
+    // masked where they are read; rows past the whole batch arrive as zeros.
+    uint64_t* bar_qk = reinterpret_cast<uint64_t*>(misc + M_BAR_C);
+    uint64_t* bar_g = reinterpret_cast<uint64_t*>(misc + M_BAR_D);
+    uint32_t ph_qk = 0, ph_g = 0;
+    auto issue_loads = [&](int64_t c0, int) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar_qk, 32768u);
+            tma_load_3d(sb + P_XQ, &p.tq, 0, h, (int)c0, bar_qk);
+            tma_load_3d(sb + P_XK, &p.tk, 0, h, (int)c0, bar_qk);
         }
-        for (int e = tid; e < kC * 32; e += kThreads) {
-            const int r = e >> 5, jj = e & 31;
-            const bool ok = r < L;
-            const int64_t off = ok ? ((c0 + r) * H + h) * kD + jj * 4 : 0;
-            cp_async16(sb + P_XG + r * 512 + jj * 16, p.g + off, ok ? 16u : 0u);
+    };
+    auto issue_g = [&](int64_t c0) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar_g, 32768u);
+            tma_load_3d(sb + P_XG, &p.tg, 0, h, (int)c0, bar_g);
         }
-        cp_async_commit();
+    };
+    auto wait_load = [&](uint64_t* bar, uint32_t& ph) -> bool {
+        const bool ok = mbar_wait_bounded(bar, ph, kWaitCycles);
+        ph ^= 1u;
+        if (!ok) atomicOr(p.err, kErrTimeout);
+        return __syncthreads_or(!ok) == 0;
     };
 
     int n = prank - 1;
     if (n < nchunks) {
         const int64_t c0 = bos + (int64_t)n * kC;
-        issue_loads(c0, (int)(eos - c0 < kC ? eos - c0 : kC));
+        issue_loads(c0, 0);
+        issue_g(c0);
     }
     for (int task = 0; n < nchunks && !aborted; n += kProducers, ++task) {
         const int64_t c0 = bos + (int64_t)n * kC;
@@ -198,63 +219,89 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         const uint32_t hs = P_HS + (uint32_t)(task & 1) * kHsBytes;     // this task's hand-off set
         float* fac = reinterpret_cast<float*>(sm + hs + H_FAC);
         if (tid < kC) s_beta[tid] = tid < L ? p.beta[(c0 + tid) * H + h] : 0.f;
-        cp_async_wait<0>();
-        __syncthreads();
+        if (!wait_load(bar_qk, ph_qk) || !wait_load(bar_g, ph_g)) { aborted = true; break; }
         trace_mark(prank, n, 0);
 
-        // ---- cumulative decay per channel (thread: channel c, tokens [32*wg, +32)) ----
-        const int c = row;
+        // ---- cumulative decay (thread: channels 2*cp, 2*cp+1; tokens [16*tq, 16*tq+16)) ----
+        // kept in log2 units so that every decay factor is one ex2.approx
+        const int cp = tid & 63, tq = tid >> 6;
+        const int c = row;                      // channel owned for the factors below
         float* Xg = reinterpret_cast<float*>(sm + P_XG);
+        const uint32_t* Xq2 = reinterpret_cast<const uint32_t*>(sm + P_XQ);
+        const uint32_t* Xk2 = reinterpret_cast<const uint32_t*>(sm + P_XK);
         const __nv_bfloat16* Xq = reinterpret_cast<const __nv_bfloat16*>(sm + P_XQ);
         const __nv_bfloat16* Xk = reinterpret_cast<const __nv_bfloat16*>(sm + P_XK);
-        float gam[32];
+        constexpr float kLog2e = 1.4426950408889634f;
+        float gam0[16], gam1[16];
         {
-            float acc = 0.f;
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                acc += Xg[(32 * wg + t) * kD + c];
-                gam[t] = acc;
+            for (int t = 0; t < 16; ++t) {
+                const int r = 16 * tq + t;
+                const float2 gv = r < L ? *reinterpret_cast<const float2*>(Xg + r * kD + 2 * cp)
+                                        : make_float2(0.f, 0.f);
+                a0 = fmaf(gv.x, kLog2e, a0);
+                a1 = fmaf(gv.y, kLog2e, a1);
+                gam0[t] = a0;
+                gam1[t] = a1;
             }
-            s_gsum[wg * 128 + c] = acc;
+            s_gsum[tq * 128 + 2 * cp] = a0;
+            s_gsum[tq * 128 + 2 * cp + 1] = a1;
         }
         __syncthreads();
-        const float gA = s_gsum[c], gB = s_gsum[128 + c];
-        if (wg) {
+        float off0 = 0.f, off1 = 0.f;           // decay of the earlier token quarters
+        for (int k2 = 0; k2 < tq; ++k2) { off0 += s_gsum[k2 * 128 + 2 * cp]; off1 += s_gsum[k2 * 128 + 2 * cp + 1]; }
 #pragma unroll
-            for (int t = 0; t < 32; ++t) gam[t] += gA;
+        for (int t = 0; t < 16; ++t) { gam0[t] += off0; gam1[t] += off1; }
+        // per channel c (thread row): half-chunk decays, in log2 units
+        const float gA2 = s_gsum[c] + s_gsum[128 + c];                 // tokens 0..31
+        const float gB2 = s_gsum[256 + c] + s_gsum[384 + c];           // tokens 32..63
+        const float kHalf2 = kHalfRange * kLog2e;
+        const int bad = __syncthreads_or((gA2 < -kHalf2) || (gB2 < -kHalf2));
+        // references per channel pair (this thread's channels), log2 units
+        const float gm0 = s_gsum[2 * cp] + s_gsum[128 + 2 * cp], gm1 = s_gsum[2 * cp + 1] + s_gsum[128 + 2 * cp + 1];
+        const float gC0 = gm0 + s_gsum[256 + 2 * cp] + s_gsum[384 + 2 * cp];
+        const float gC1 = gm1 + s_gsum[256 + 2 * cp + 1] + s_gsum[384 + 2 * cp + 1];
+        const float gr0 = bad ? 0.f : gm0, gr1 = bad ? 0.f : gm1;      // reference for Lk / Lq
+        const float gs0 = bad ? gC0 : gm0, gs1 = bad ? gC1 : gm1;      // reference for R
+        if (tq == 0) {
+            fac[2 * cp] = ex2_approx(gr0);
+            fac[2 * cp + 1] = ex2_approx(gr1);
+            fac[128 + 2 * cp] = ex2_approx(gC0);
+            fac[128 + 2 * cp + 1] = ex2_approx(gC1);
+            fac[256 + 2 * cp] = ex2_approx(gC0 - gs0);
+            fac[256 + 2 * cp + 1] = ex2_approx(gC1 - gs1);
         }
-        const float gC = gA + gB;
-        const int bad = __syncthreads_or((gA < -kHalfRange) || (gB < -kHalfRange));
-        trace_mark(prank, n, 8);
-        const float gref = bad ? 0.f : gA;          // reference for Lk / Lq
-        const float gref2 = bad ? gC : gA;          // reference for R
-        if (wg) {
-            fac[c] = __expf(gref);
-            fac[128 + c] = __expf(gC);
-            fac[256 + c] = __expf(gC - gref2);
-        }
-        if (bad) {
+        if (bad) {                              // natural-log gamma for the exact path
 #pragma unroll
-            for (int t = 0; t < 32; ++t) Xg[(32 * wg + t) * kD + c] = gam[t];
+            for (int t = 0; t < 16; ++t)
+                *reinterpret_cast<float2*>(Xg + (16 * tq + t) * kD + 2 * cp) =
+                    make_float2(gam0[t] * (1.f / kLog2e), gam1[t] * (1.f / kLog2e));
         }
         // ---- folded operands Lk, Lq (A of A|P), R (B of A|P) ----
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-            float lk[8], lq[8], rr[8];
+        for (int qq = 0; qq < 2; ++qq) {
+            float lk0[8], lq0[8], rr0[8], lk1[8], lq1[8], rr1[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int t = 8 * qq + u;
-                const int r = 32 * wg + t;
-                const float kx = bf(Xk + r * kD + c), qx = bf(Xq + r * kD + c);
-                const float a = __expf(gam[t] - gref), b = __expf(gref2 - gam[t]);
-                lk[u] = kx * a;
-                lq[u] = qx * a;
-                rr[u] = kx * b;
+                const int r = 16 * tq + t;
+                const bool ok = r < L;
+                const uint32_t kw = ok ? Xk2[r * 64 + cp] : 0u, qw = ok ? Xq2[r * 64 + cp] : 0u;
+                const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xffff0000u);
+                const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xffff0000u);
+                const float a0 = ex2_approx(gam0[t] - gr0), b0 = ex2_approx(gs0 - gam0[t]);
+                const float a1 = ex2_approx(gam1[t] - gr1), b1 = ex2_approx(gs1 - gam1[t]);
+                lk0[u] = k0 * a0; lq0[u] = q0 * a0; rr0[u] = k0 * b0;
+                lk1[u] = k1 * a1; lq1[u] = q1 * a1; rr1[u] = k1 * b1;
             }
-            const int ch = 4 * wg + qq;
-            st16(sm, P_LK + mnmaj_chunk(c, ch, 0, 16), pack8(lk));
-            st16(sm, hs + H_LQ + mnmaj_chunk(c, ch, 0, 16), pack8(lq));
-            st16(sm, hs + H_RT + mnmaj_chunk(c, ch, 0, 16), pack8(rr));
+            const int ch = 2 * tq + qq;         // 8-token chunk index within the 64 tokens
+            st16(sm, P_LK + mnmaj_chunk(2 * cp, ch, 0, 16), pack8(lk0));
+            st16(sm, P_LK + mnmaj_chunk(2 * cp + 1, ch, 0, 16), pack8(lk1));
+            st16(sm, hs + H_LQ + mnmaj_chunk(2 * cp, ch, 0, 16), pack8(lq0));
+            st16(sm, hs + H_LQ + mnmaj_chunk(2 * cp + 1, ch, 0, 16), pack8(lq1));
+            st16(sm, hs + H_RT + mnmaj_chunk(2 * cp, ch, 0, 16), pack8(rr0));
+            st16(sm, hs + H_RT + mnmaj_chunk(2 * cp + 1, ch, 0, 16), pack8(rr1));
         }
         fence_async_smem();
         __syncthreads();
@@ -310,7 +357,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                 while (r * (r + 1) / 2 > pidx) --r;
                 const int i = pidx - r * (r + 1) / 2;
                 float a = 0.f, pp = 0.f;
-                for (int cc = lane; cc < kD; cc += 32) {
+                for (int cc = lane; cc < kD && r < L; cc += 32) {
                     const float ki = bf(Xk + i * kD + cc) * expf(Xg[r * kD + cc] - Xg[i * kD + cc]);
                     a = fmaf(bf(Xk + r * kD + cc), ki, a);
                     pp = fmaf(bf(Xq + r * kD + cc), ki, pp);
@@ -318,8 +365,9 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                 a = warp_sum(a);
                 pp = warp_sum(pp);
                 if (lane == 0) {
-                    Nm[r * kLd + i] = (i < r) ? s_beta[r] * a : 0.f;
-                    Nm[i * kLd + r] = 0.f;
+                    float* Aex = reinterpret_cast<float*>(sm + hs + H_ZO);     // [64][64]
+                    Aex[r * 64 + i] = (i < r) ? s_beta[r] * a : 0.f;
+                    Aex[i * 64 + r] = (i < r) ? 0.f : Aex[i * 64 + r];
                     Pop[(kmaj_chunk(r, i >> 3, 0, 64) + (i & 7) * 2) / 2] = __float2bfloat16_rn(pp);
                     if (i < r) Pop[(kmaj_chunk(i, r >> 3, 0, 64) + (r & 7) * 2) / 2] = __float2bfloat16_rn(0.f);
                 }
@@ -329,6 +377,9 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                 const int64_t c1 = c0 + (int64_t)kProducers * kC;
                 issue_loads(c1, (int)(eos - c1 < kC ? eos - c1 : kC));
             }
+            // gamma (in the scratch) is dead: move diag(beta) A into place
+            const float* Aex = reinterpret_cast<const float*>(sm + hs + H_ZO);
+            for (int e = tid; e < kC * kC; e += kThreads) Nm[(e >> 6) * kLd + (e & 63)] = Aex[e];
         }
         __syncthreads();
         trace_mark(prank, n, 3);
@@ -373,18 +424,29 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                     warp_block_store16(Tm + (16 * B) * kLd + 16 * b, kLd, acc2, -1.f);
                 }
                 __syncthreads();
+                if (d == 1) trace_mark(prank, n, 14);
+                if (d == 3) trace_mark(prank, n, 15);
             }
+            // T' = T diag(beta): 8 consecutive columns per item from two 16-byte reads
             for (int e = tid; e < kC * 8; e += kThreads) {
                 const int r = e >> 3, q8 = e & 7;
+                const float4 t0 = *reinterpret_cast<const float4*>(Tm + r * kLd + 8 * q8);
+                const float4 t1 = *reinterpret_cast<const float4*>(Tm + r * kLd + 8 * q8 + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(s_beta + 8 * q8);
+                const float4 b1 = *reinterpret_cast<const float4*>(s_beta + 8 * q8 + 4);
+                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
                 float w8[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int i = 8 * q8 + u;
-                    w8[u] = (i < r) ? Tm[r * kLd + i] * s_beta[i] : (i == r ? s_beta[r] : 0.f);
+                    w8[u] = (i < r) ? tv[u] * bv[u] : (i == r ? bv[u] : 0.f);
                 }
                 st16(sm, hs + H_TP + kmaj_chunk(r, q8, 0, 64), pack8(w8));
             }
         }
+        __syncthreads();
+        if (n + kProducers < nchunks) issue_g(c0 + (int64_t)kProducers * kC);
         trace_mark(prank, n, 4);
         fence_async_smem();
         tc_fence_before();
@@ -404,44 +466,44 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         trace_mark(prank, n, 5);
         tc_fence_after();
 
-        // ---- hand the chunk to the consumer (ring slot n % 2) ----
-        if (n >= 2) {
-            const bool ok = mbar_wait_cluster_bounded(bar_free, ph_free, kWaitCycles);
-            ph_free ^= 1u;
-            if (!ok) atomicOr(p.err, kErrTimeout);
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
-        const uint32_t dst = c_slot0 + (uint32_t)slot * kSlotBytes;
-        trace_mark(prank, n, 6);
-        const SlotMap mp = slot_map(slot);
+        // ---- Z -> bf16 into the hand-off set (local), then hand the chunk over ----
         {
             float val[32];
             tmem_ld32(tm + lane_sel + TP_Z + 32 * wg, val);
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq)
-                st_cluster16(dst + mp.zo + mnmaj_chunk(row, 4 * wg + qq, 0, 16), pack8(val + 8 * qq));
+                st16(sm, hs + H_ZO + mnmaj_chunk(row, 4 * wg + qq, 0, 16), pack8(val + 8 * qq));
         }
-        trace_mark(prank, n, 12);
-        // each thread publishes its own Z stores with a release arrival on the slot's barrier
-        fence_async_cluster();
-        const uint32_t full = c_misc + (slot ? M_BAR_B : M_BAR_A);
-        mbar_arrive_remote(full);
-        trace_mark(prank, n, 13);
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
-            // one more arrival announcing the bulk bytes, then the copies; all of it completes
-            // the slot's "full" barrier in the consumer
-            mbar_arrive_expect_tx_remote(full, kHandoffTx);
-            bulk_copy_to_peer(dst + mp.lq, sb + hs + H_LQ, 16384, full);
-            bulk_copy_to_peer(dst + mp.rt, sb + hs + H_RT, 16384, full);
-            bulk_copy_to_peer(dst + S_TP, sb + hs + H_TP, 8192, full);
-            bulk_copy_to_peer(dst + mp.po, sb + hs + H_PO, 8192, full);
-            bulk_copy_to_peer(dst + S_FAC, sb + hs + H_FAC, 1536, full);
+        trace_mark(prank, n, 12);
+        if (n >= 2) {                           // ring slot n % 2 must have been released
+            const bool ok = mbar_wait_cluster_bounded(bar_free, ph_free, kWaitCycles);
+            ph_free ^= 1u;
+            if (!ok) atomicOr(p.err, kErrTimeout);
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        trace_mark(prank, n, 6);
+        if (warp == 0) {
+            // one arrival announcing the bytes, then the bulk copies into the consumer's slot
+            // (one per lane); together they complete that slot's "full" barrier
+            const int lane = tid & 31;
+            const uint32_t dst = c_slot0 + (uint32_t)slot * kSlotBytes;
+            const SlotMap mp = slot_map(slot);
+            const uint32_t full = c_misc + (slot ? M_BAR_B : M_BAR_A);
+            // relaxed: the bytes travel in the bulk copies, which complete the barrier themselves
+            if (lane == 0) mbar_arrive_expect_tx_remote_relaxed(full, kHandoffTx);
+            __syncwarp();
+            if (lane == 0) bulk_copy_to_peer(dst + mp.lq, sb + hs + H_LQ, 16384, full);
+            if (lane == 1) bulk_copy_to_peer(dst + mp.zo, sb + hs + H_ZO, 16384, full);
+            if (lane == 2) bulk_copy_to_peer(dst + mp.rt, sb + hs + H_RT, 16384, full);
+            if (lane == 3) bulk_copy_to_peer(dst + S_TP, sb + hs + H_TP, 8192, full);
+            if (lane == 4) bulk_copy_to_peer(dst + mp.po, sb + hs + H_PO, 8192, full);
+            if (lane == 5) bulk_copy_to_peer(c_fac + (uint32_t)(n % 3) * kFacBytes, sb + hs + H_FAC, kFacBytes, full);
         }
         trace_mark(prank, n, 7);
     }
-    cp_async_wait<0>();
 }
 
 // ============================== consumer ==============================
@@ -464,32 +526,51 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
     for (int cc = 0; cc < 64; ++cc)
         sreg[cc] = p.h0 ? p.h0[sbase + (int64_t)(64 * wg + cc) * kD + j] : 0.f;
 
+    // V tile of chunk nn into its slot by TMA: two (64 channels x 64 tokens) boxes whose
+    // 128B-swizzled image is exactly the MN-major operand layout. Rows past the sequence do
+    // not matter (the matching columns of T' are zero).
+    uint64_t* bar_v0 = reinterpret_cast<uint64_t*>(misc + M_BAR_C);
+    uint64_t* bar_v1 = reinterpret_cast<uint64_t*>(misc + M_BAR_D);
+    uint32_t ph_v0 = 0, ph_v1 = 0;
     auto issue_v = [&](int nn) {
-        const int64_t c0 = bos + (int64_t)nn * kC;
-        const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
-        const uint32_t base = sb + C_SLOT0 + (nn & 1) * kSlotBytes + S_VT;
-        for (int e = tid; e < kC * 16; e += kThreads) {
-            const int r = e >> 4, jj = e & 15;
-            const bool ok = r < L;
-            const int64_t off = ok ? ((c0 + r) * H + h) * kD + jj * 8 : 0;
-            cp_async16(base + mnmaj_chunk(r, jj & 7, jj >> 3, 8), p.v + off, ok ? 16u : 0u);
+        if (tid == 0) {
+            uint64_t* bv = (nn & 1) ? bar_v1 : bar_v0;
+            const uint32_t base = sb + C_SLOT0 + (nn & 1) * kSlotBytes + S_VT;
+            const int c0 = (int)(bos + (int64_t)nn * kC);
+            mbar_arrive_expect_tx(bv, 16384u);
+            tma_load_3d(base, &p.tv, 0, h, c0, bv);
+            tma_load_3d(base + 8192, &p.tv, 64, h, c0, bv);
         }
-        cp_async_commit();
     };
-    // Output epilogue: O of chunk nn is read from TMEM right after its last MMA completed
-    // (oval) and written to HBM while the next chunk's MMAs run.
+    auto wait_v = [&](int nn) -> bool {
+        const int sl = nn & 1;
+        const bool ok = mbar_wait_bounded(sl ? bar_v1 : bar_v0, sl ? ph_v1 : ph_v0, kWaitCycles);
+        if (sl) ph_v1 ^= 1u; else ph_v0 ^= 1u;
+        if (!ok) atomicOr(p.err, kErrTimeout);
+        return __syncthreads_or(!ok) == 0;
+    };
+    // Output epilogue: O of chunk nn goes from TMEM to a row-major [token][channel] bf16
+    // staging tile (the Ut^T buffer, free once the chunk's last MMAs completed), then to HBM
+    // as one TMA tile store (a ragged last chunk: one bulk copy per valid token, so rows of the
+    // next sequence are never touched), overlapping the next chunk.
     float oval[32];
-    auto load_o = [&](int nn) {
-        tmem_ld32(tm + lane_sel + ((nn & 1) ? TC_O1 : TC_O0) + 32 * wg, oval);
+    auto load_o = [&](int nn) { tmem_ld32(tm + lane_sel + ((nn & 1) ? TC_O1 : TC_O0) + 32 * wg, oval); };
+    auto stage_o = [&]() {
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + C_UT);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) st[(32 * wg + t) * kD + j] = __float2bfloat16_rn(p.scale * oval[t]);
     };
-    auto store_o = [&](int nn) {
+    auto store_o = [&](int nn) {               // warp 1, after the staging writes are fenced
         const int64_t c0 = bos + (int64_t)nn * kC;
         const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int r = 32 * wg + t;
-            if (r < L) p.o[((c0 + r) * H + h) * kD + j] = __float2bfloat16_rn(p.scale * oval[t]);
+        const int lane = tid & 31;
+        if (L == kC) {
+            if (lane == 0) tma_store_3d(&p.to, 0, h, (int)c0, sb + C_UT);
+        } else {
+            for (int r = lane; r < L; r += 32)
+                bulk_store(p.o + ((c0 + r) * H + h) * kD, sb + C_UT + r * 256, 256);
         }
+        bulk_commit();
     };
     auto wait_mma = [&]() -> bool {
         const bool ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitCycles);
@@ -497,50 +578,62 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         if (!ok) atomicOr(p.err, kErrTimeout);
         return __syncthreads_or(!ok) == 0;
     };
-    if (nchunks > 0) issue_v(0);
+    auto wait_full = [&](int nn) -> bool {
+        const int sl = nn & 1;
+        const bool ok = mbar_wait_cluster_bounded(sl ? bar_full1 : bar_full0,
+                                                  sl ? ph_full1 : ph_full0, kWaitCycles);
+        if (sl) ph_full1 ^= 1u; else ph_full0 ^= 1u;
+        if (!ok) atomicOr(p.err, kErrTimeout);
+        return __syncthreads_or(!ok) == 0;
+    };
+    // -U^T = -(V^T T'^T) of chunk nn into its X accumulator (one converged warp).
+    auto issue_u = [&](int nn) {
+        const uint32_t so = C_SLOT0 + (nn & 1) * kSlotBytes;
+        tc_fence_after();
+        const uint32_t id_u = idesc_bf16(128, 64, true, false, true);
+        const uint64_t a0 = make_desc(sb + so + S_VT, 8192, 1024);
+        const uint64_t b0 = make_desc(sb + so + S_TP, 16, 1024);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            warp_mma(tm + ((nn & 1) ? TC_X1 : TC_X0), desc_add(a0, s * 2048), desc_add(b0, s * 32), id_u, s > 0);
+    };
+    // Sm(nn) = (diag(e^{gamma_ref(nn)}) S)^T as the bf16 A operand (S already updated).
+    auto write_sm = [&](int nn) {
+        const float* fac = reinterpret_cast<const float*>(sm + C_FAC + (nn % 3) * kFacBytes);
+        const float4* fac4 = reinterpret_cast<const float4*>(fac + 64 * wg);
+#pragma unroll
+        for (int qq = 0; qq < 8; ++qq) {
+            const float4 e0 = fac4[2 * qq], e1 = fac4[2 * qq + 1];
+            const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+            float w8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) w8[u] = sreg[8 * qq + u] * ev[u];
+            st16(sm, C_ST + kmaj_chunk(j, qq, wg, 128), pack8(w8));
+        }
+    };
+
+    // prologue: operands of chunk 0 (and the V tile of chunk 1)
+    if (nchunks > 0) {
+        issue_v(0);
+        if (nchunks > 1) issue_v(1);
+        if (!wait_v(0)) aborted = true;
+        if (!aborted && !wait_full(0)) aborted = true;
+        if (!aborted) {
+            write_sm(0);
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (warp == 0) issue_u(0);
+        }
+    }
 
     for (int n = 0; n < nchunks && !aborted; ++n) {
         const int slot = n & 1;
         const uint32_t so = C_SLOT0 + slot * kSlotBytes;
         const SlotMap mp = slot_map(slot);
-        const float* fac = reinterpret_cast<const float*>(sm + so + S_FAC);
+        const float* fac = reinterpret_cast<const float*>(sm + C_FAC + (n % 3) * kFacBytes);
         const uint32_t tX = slot ? TC_X1 : TC_X0;
         trace_mark(0, n, 0);
-
-        if (n + 1 < nchunks) { issue_v(n + 1); cp_async_wait<1>(); }
-        else cp_async_wait<0>();
-        fence_async_smem();
-        trace_mark(0, n, 8);
-        {
-            const bool ok = mbar_wait_cluster_bounded(slot ? bar_full1 : bar_full0,
-                                                      slot ? ph_full1 : ph_full0, kWaitCycles);
-            if (slot) ph_full1 ^= 1u; else ph_full0 ^= 1u;
-            trace_mark(0, n, 9);
-            if (!ok) atomicOr(p.err, kErrTimeout);
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
-        trace_mark(0, n, 1);
-        // -U^T = -(V^T T'^T) needs only the chunk's operands: start it before the state operand.
-        if (warp == 0) {
-            tc_fence_after();
-            const uint32_t id_u = idesc_bf16(128, 64, true, false, true);
-            const uint64_t a0 = make_desc(sb + so + S_VT, 8192, 1024);
-            const uint64_t b0 = make_desc(sb + so + S_TP, 16, 1024);
-#pragma unroll
-            for (int s = 0; s < 4; ++s) warp_mma(tm + tX, desc_add(a0, s * 2048), desc_add(b0, s * 32), id_u, s > 0);
-        }
-        // ---- Sm = (diag(e^{gamma_ref}) S)^T as a bf16 A operand ----
-#pragma unroll
-        for (int qq = 0; qq < 8; ++qq) {
-            float w8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) w8[u] = sreg[8 * qq + u] * fac[64 * wg + 8 * qq + u];
-            st16(sm, C_ST + kmaj_chunk(j, qq, wg, 128), pack8(w8));
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        trace_mark(0, n, 2);
 
         // ---- [X | O] (+)= Sm [Z | Lq]: X = -Ut^T, O = Sm Lq^T ----
         if (warp == 0) {
@@ -559,11 +652,13 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             for (int s = 1; s < 8; ++s)
                 warp_mma(tm + dW, desc_add(aS, (s >> 2) * 16384 + (s & 3) * 32), desc_add(bW, s * 2048), id128, 1);
             warp_commit(bar_mma);
-            trace_mark(0, n, 10);
         }
-        if (n > 0) store_o(n - 1);
-        trace_mark(0, n, 3);
+        trace_mark(0, n, 1);
+        // the staging tile of O(n - 1) is rewritten below: its TMA store must have read it
+        if (warp == 1) bulk_wait_read0();
+        trace_mark(0, n, 2);
         if (!wait_mma()) { aborted = true; break; }
+        trace_mark(0, n, 10);
         tc_fence_after();
         {
             float val[32];
@@ -576,7 +671,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        trace_mark(0, n, 4);
+        trace_mark(0, n, 3);
 
         // ---- [O | dS^T] (+)= Ut^T [P | R] ----
         if (warp == 0) {
@@ -595,41 +690,60 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             for (int s = 1; s < 4; ++s) warp_mma(tm + dW, desc_add(aU, s * 32), desc_add(bW, s * 32), id192, 1);
             warp_commit(bar_mma);
         }
+        // the V tile of this slot was consumed by -U^T (complete): fetch the one of chunk n + 2
+        if (n + 2 < nchunks) issue_v(n + 2);
+        trace_mark(0, n, 4);
         if (!wait_mma()) { aborted = true; break; }
-        trace_mark(0, n, 11);
+        // every MMA that reads ring slot n % 2 has completed (the chunk's factors live in the
+        // factor ring): tell the producer of chunk n + 2 it may write the slot
+        if (tid == 0 && n + 2 < nchunks)
+            mbar_arrive_remote_relaxed(map_to_rank(sb + P_MISC + M_BAR_A, 1 + (n + 2) % kProducers));
+        trace_mark(0, n, 5);
+        const bool more = n + 1 < nchunks;
+        if (more) {
+            // operands of chunk n + 1 (its V tile was requested one chunk earlier)
+            if (!wait_v(n + 1)) { aborted = true; break; }
+            if (!wait_full(n + 1)) { aborted = true; break; }
+        }
+        trace_mark(0, n, 6);
         tc_fence_after();
         {
             float val[32];
+            const float4* eC4 = reinterpret_cast<const float4*>(fac + 128 + 64 * wg);
+            const float4* eR4 = reinterpret_cast<const float4*>(fac + 256 + 64 * wg);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 tmem_ld32(tm + lane_sel + TC_S + 64 * wg + 32 * half, val);
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const int cc = 32 * half + t;
-                    const int c = 64 * wg + cc;
-                    sreg[cc] = fmaf(fac[128 + c], sreg[cc], fac[256 + c] * val[t]);
+                for (int t4 = 0; t4 < 8; ++t4) {
+                    const float4 ec = eC4[8 * half + t4], er = eR4[8 * half + t4];
+                    const float ecv[4] = {ec.x, ec.y, ec.z, ec.w}, erv[4] = {er.x, er.y, er.z, er.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int cc = 32 * half + 4 * t4 + u;
+                        sreg[cc] = fmaf(ecv[u], sreg[cc], erv[u] * val[4 * t4 + u]);
+                    }
                 }
             }
         }
         load_o(n);
-        trace_mark(0, n, 5);
+        stage_o();
+        if (more) write_sm(n + 1);
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        trace_mark(0, n, 12);
-        // slot n % 2 is free again: tell the producer of chunk n + 2
-        if (tid == 0 && n + 2 < nchunks)
-            mbar_arrive_remote_relaxed(map_to_rank(sb + P_MISC + M_BAR_A, 1 + (n + 2) % kProducers));
-        trace_mark(0, n, 6);
+        trace_mark(0, n, 7);
+        if (more && warp == 0) issue_u(n + 1);
+        if (warp == 1) store_o(n);
     }
-    if (nchunks > 0 && !aborted) store_o(nchunks - 1);     // loaded at the end of the last chunk
-    cp_async_wait<0>();
+    if (warp == 1) bulk_wait0();
     if (p.ht && !aborted) {
 #pragma unroll
         for (int cc = 0; cc < 64; ++cc) p.ht[sbase + (int64_t)(64 * wg + cc) * kD + j] = sreg[cc];
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(sm);
@@ -649,11 +763,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const Params p) 
     }
     if (threadIdx.x == 0) {
         mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_MMA), 1);
-        // consumer "full" barriers: every producer thread arrives once (its Z stores) plus the
-        // arrival that announces the bulk copy; producer "free" barrier: one consumer arrival
-        const uint32_t cnt = is_consumer ? (uint32_t)kThreads + 1u : 1u;
-        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_A), cnt);
-        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_B), cnt);
+        // consumer "full" barriers: one producer arrival + the bulk bytes; producer "free"
+        // barrier: one consumer arrival
+        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_A), 1);
+        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_B), 1);
+        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_C), 1);
+        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_D), 1);
     }
     tc_fence_before();
     cluster_sync();                     // barriers of every CTA exist before any remote arrive
@@ -681,6 +796,13 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, unsigned int* err, cudaStream_t
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     Params p;
+    const bool maps_ok =
+        make_tmap_thd(&p.tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false) &&
+        make_tmap_thd(&p.tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false) &&
+        make_tmap_thd(&p.tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.T_tot, a.H, kD, kD, kC, false) &&
+        make_tmap_thd(&p.tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, 64, kC, true) &&
+        make_tmap_thd(&p.to, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false);
+    if (!maps_ok) return cudaErrorInvalidValue;
     p.q = static_cast<const __nv_bfloat16*>(a.q);
     p.k = static_cast<const __nv_bfloat16*>(a.k);
     p.v = static_cast<const __nv_bfloat16*>(a.v);

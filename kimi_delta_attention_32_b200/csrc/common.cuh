@@ -97,15 +97,15 @@ __device__ __forceinline__ int find_seq(const int32_t* cu, int N, int64_t t) {
 // g_trace[cta][chunk][mark] of the including translation unit.
 #ifdef KDA_TRACE
 static __device__ unsigned long long g_trace[4][512][16];
-__device__ __forceinline__ void trace_mark(int cta, int chunk, int mark) {
-    if (threadIdx.x == 0 && blockIdx.x < 4 && chunk < 512) {
+__device__ __forceinline__ void trace_mark(int cta, int chunk, int mark, int who = 0) {
+    if (threadIdx.x == who && blockIdx.x < 4 && chunk < 512) {
         unsigned long long t;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
         g_trace[cta][chunk][mark] = t;
     }
 }
 #else
-__device__ __forceinline__ void trace_mark(int, int, int) {}
+__device__ __forceinline__ void trace_mark(int, int, int, int = 0) {}
 #endif
 
 }  // namespace kda

@@ -120,6 +120,7 @@ __device__ __forceinline__ void conv_unit(const ConvParams& p, int z, int h, int
 
     // hist[m] = input at position t-3+m (m = 0 oldest) of the current sequence.
     float hist[kHist][CPL];
+    T* yrow = y + (t0 * H + h) * D + cl;
     const bool norm = (z < 2);
 #pragma unroll
     for (int tt = 0; tt < kTile; ++tt) {
@@ -162,7 +163,7 @@ __device__ __forceinline__ void conv_unit(const ConvParams& p, int z, int h, int
             zc = fmaf(w[c][1], hist[1][c], zc);
             zc = fmaf(w[c][2], hist[2][c], zc);
             zc = fmaf(w[c][3], xt[c], zc);
-            const float sv = zc / (1.f + __expf(-zc));
+            const float sv = __fdividef(zc, 1.f + __expf(-zc));
             out[c] = sv;
             ss = fmaf(sv, sv, ss);
         }
@@ -172,7 +173,8 @@ __device__ __forceinline__ void conv_unit(const ConvParams& p, int z, int h, int
 #pragma unroll
             for (int c = 0; c < CPL; ++c) out[c] *= inv;
         }
-        Vec<T, CPL>::store(y + (t * H + h) * D + cl, out);
+        Vec<T, CPL>::store(yrow, out);
+        yrow += (int64_t)H * D;
         if (p.step_mode && cache) {
             // decode: new cache = the two newest history entries, then this token
 #pragma unroll
