@@ -273,10 +273,14 @@ def run_ours(args):
             q, k, v = d["q"], d["k"], d["v"]
         o = torch.empty_like(v)
         ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+        ws_bytes = kda.chunk_fwd_workspace_size(N, T_tot, H, dk, dv,
+                                                io=kda.KDA_IO_F32 if wl.io == "f32" else kda.KDA_IO_BF16)
+        ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev) if ws_bytes else None
 
         def step():
             kda.chunk_fwd(q, k, v, d["g"], d["beta"], 1.0, h0=d["h0"], ht=ht, o=o,
-                          cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], stream=stream)
+                          cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], workspace=ws,
+                          stream=stream)
         units = T_tot
         algo_bytes = prefill_bytes(T_tot, H, dk, dv, N, h0=d["h0"] is not None)
         wl_desc = {"prefill_8k": "prefill_8k: B=1,H=32,T=8192,dk=dv=128,bf16 q/k/v/o,fp32 g/beta/"
@@ -341,7 +345,7 @@ def run_ours(args):
                 dbuf[nm].copy_(host[nm], non_blocking=True)
             kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], 1.0,
                           h0=d["h0"], ht=ht, o=o, cu_seqlens=d["cu_seqlens"],
-                          cu_host=d["cu_host"], stream=stream)
+                          cu_host=d["cu_host"], workspace=ws, stream=stream)
             o_host.copy_(o, non_blocking=True)
             ht_host.copy_(ht, non_blocking=True)
         et = _events_time(torch, e2e_step, max(2, args.steps // 2), 2, stream=stream)

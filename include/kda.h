@@ -106,7 +106,11 @@ kda_status kda_conv_fwd(const void* q_raw, const void* k_raw, const void* v_raw,
 /*
  * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd needs
  * for these sizes (written to *bytes, host). Zero means none; the call then
- * accepts workspace == NULL.
+ * accepts workspace == NULL. The bf16, dk = dv = 128, chunk-64 prefill needs a
+ * fixed ~47.8 MB whatever the batch: per-SM hand-off rings through which the
+ * kernel's producer CTAs pass each chunk's operands to its consumer CTA via L2.
+ * The contents need no initialisation and are dead after the call; one
+ * workspace may serve consecutive calls on one stream, not concurrent ones.
  */
 kda_status kda_chunk_fwd_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, int chunk,
                                         kda_io_dtype io, size_t* bytes);
@@ -127,6 +131,9 @@ kda_status kda_chunk_fwd_workspace_size(int N, int64_t T_tot, int H, int dk, int
  *  h0   : [N, H, dk, dv] fp32 initial states, or NULL for zero states
  *  ht   : [N, H, dk, dv] fp32 final states, or NULL to skip; may alias h0
  *  chunk: tokens per chunk; this build supports 64.
+ *  workspace: device memory of at least kda_chunk_fwd_workspace_size() bytes,
+ *         16-byte aligned, owned by the caller (KDA_ERR_WORKSPACE otherwise);
+ *         may be NULL when that size is 0.
  *  Supported: dk == dv in {64, 128} for io F32; dk == dv == 128 or 64 for BF16.
  *  Empty sequences are allowed (their final state is the initial state).
  */

@@ -55,6 +55,11 @@ bool use_cluster_prefill() {
     return !(e != nullptr && strcmp(e, "single") == 0);
 }
 
+// The bf16, dk = dv = 128, chunk-64 prefill runs on the cluster pipeline, which needs a workspace.
+bool cluster_prefill_path(kda_io_dtype io, int dk, int dv, int chunk) {
+    return io == KDA_IO_BF16 && dk == 128 && dv == 128 && chunk == 64;
+}
+
 // Device address of the error word on the current device.
 unsigned int* device_error_word() {
     void* p = nullptr;
@@ -113,7 +118,7 @@ KDA_API kda_status kda_chunk_fwd_workspace_size(int N, int64_t T_tot, int H, int
     if (bytes == nullptr || N < 0 || T_tot < 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0)
         return KDA_ERR_INVALID_ARG;
     if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
-    *bytes = 0;
+    *bytes = cluster_prefill_path(io, dk, dv, chunk) ? kda::chunk_tcx_workspace_bytes() : 0;
     return KDA_OK;
 }
 
@@ -123,8 +128,6 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
                          int B, int T, int N, int H, int dk, int dv, int chunk,
                          kda_io_dtype io, void* workspace, size_t workspace_bytes,
                          void* stream) {
-    (void)workspace;
-    (void)workspace_bytes;
     if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
     if (H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0) return KDA_ERR_INVALID_ARG;
     int64_t T_tot = 0;
@@ -145,11 +148,15 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
     a.N = Nn; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk;
     a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
     if (kda::chunk_tc_supported(a)) {
+        const bool cluster = use_cluster_prefill();
+        if (cluster && (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0 ||
+                        workspace_bytes < kda::chunk_tcx_workspace_bytes()))
+            return KDA_ERR_WORKSPACE;
         unsigned int* err = device_error_word();
         if (err == nullptr) return KDA_ERR_CUDA;
         cudaStream_t st = static_cast<cudaStream_t>(stream);
-        return from_cuda(use_cluster_prefill() ? kda::launch_chunk_tcx(a, err, st)
-                                               : kda::launch_chunk_tc(a, err, st));
+        if (!cluster) return from_cuda(kda::launch_chunk_tc(a, err, st));
+        return from_cuda(kda::launch_chunk_tcx(a, workspace, workspace_bytes, err, st));
     }
     return from_cuda(kda::launch_chunk_simt(a, static_cast<cudaStream_t>(stream)));
 }

@@ -1,26 +1,34 @@
 // chunk_tcx.cu -- chunked KDA prefill, bf16 I/O, dk = dv = 128, chunk 64, as a producer /
 // consumer pipeline inside one thread-block cluster per (sequence, head).
 //
-// Same per-chunk algebra as the sequential kernel (sarnas.ru, "Яндекс открыл веса
-// AliceAI-Foundation-80B-A3B-Base ...", section "Что именно изменилось"; m.lqnn.cn/news/205170,
-// section "KDA 与 Gated Attention ..."), with the decay folded around a per-chunk reference
-// gamma_ref (the chunk middle, or the chunk start when the range test fails):
-//   Lk = k e^{gamma - gamma_ref},  Lq = q e^{gamma - gamma_ref},  R = k e^{gamma_ref2 - gamma}
-//   [A ; P] = [Lk ; Lq] R^T                                   (gamma_ref2 = gamma_ref)
-//   T' = (I + diag(beta) A)^-1 diag(beta),   Z = Lk^T T'^T      (= e^{-gamma_ref} W^T)
-//   Sm = (diag(e^{gamma_ref}) S)^T
-//   Ut^T = V^T T'^T - Sm Z,   O^T = Sm Lq^T + Ut^T P^T,   dS^T = Ut^T R
-//   S' = diag(e^{gamma_C}) S + diag(e^{gamma_C - gamma_ref2}) dS
-// A chunk whose half-chunk decay exceeds 80 in some channel takes gamma_ref = 0 and
-// gamma_ref2 = gamma_C, and forms A and P exactly on CUDA cores; every factor is then <= 1.
+// The recurrence (sarnas.ru, "Яндекс открыл веса AliceAI-Foundation-80B-A3B-Base ...", section
+// "Что именно изменилось"; m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...") is
+// linear in the state, so one chunk maps the state at its start, S, to the state at its end by
+// S' = M S + N with M, N built from the chunk's inputs alone. This kernel splits exactly along
+// that line: producers build everything that does not depend on S; the consumer applies it.
+// With gamma the within-chunk cumulative log-decay, gamma_C its last row and gamma_ref a
+// per-chunk reference (the chunk middle, or 0 when a half chunk decays by more than 80 in some
+// channel), per chunk:
+//   Lk = k e^{gamma - gamma_ref},  Lq = q e^{gamma - gamma_ref}
+//   R = k e^{gamma_ref - gamma},   Rh = k e^{gamma_C - gamma}              (every Rh <= |k|)
+//   [A ; P] = [Lk ; Lq] R^T   (strictly / inclusively lower triangular parts)
+//   T' = (I + diag(beta) A)^-1 diag(beta)
+//   Yh^T = Rh^T T',  Wh^T = P T',  Gm = -Lk^T Yh,  Qh = Lq^T - Lk^T Wh
+// and with Sm = S^T diag(e^{gamma_ref}) (bf16), on the consumer:
+//   S'^T = S^T diag(e^{gamma_C}) + V^T Yh + Sm Gm        (fp32 state, fp32 decay term)
+//   O^T  = scale (V^T Wh + Sm Qh)
+// A chunk that fails the range test forms A and P' exactly on CUDA cores (gamma_ref = 0, so
+// every factor is <= 1).
 //
-// Cluster of 4 CTAs: rank 0 is the consumer -- it owns the fp32 state and runs only the
-// sequential chain (U^T, Ut^T, O^T, dS^T on tcgen05, state update); ranks 1..3 are producers,
-// each preparing every third chunk (loads, cumulative decay, folded operands, A|P on
-// tcgen05, fp32 triangular inverse, Z on tcgen05) and writing the chunk's operands straight
-// into a two-slot ring in the consumer's shared memory over DSMEM. Flow control is by
-// cluster-scope mbarriers: "full" in the consumer (one producer arrival per chunk) and
-// "free" in each producer (one consumer arrival per chunk it may write). All waits are bounded.
+// Cluster of 4 CTAs: rank 0 is the consumer. Per chunk it issues V^T [Yh | Wh] as soon as the
+// operands are in, then the chain Sm [Gm | Qh] (A operand Sm in tensor memory), updates the fp32
+// state in registers and writes the next Sm back to tensor memory; O leaves through a TMA
+// store. Ranks 1..3 are producers, each preparing every third chunk. A chunk's operands travel
+// through L2, not DSMEM (bulk copies between SMs of a cluster move ~30-60 GB/s, TMA loads from
+// L2 150-220 GB/s): the producer bulk-stores them into a four-slot ring in global memory owned
+// by the consumer's SM, the consumer TMA-loads them two chunks ahead into a two-slot ring in its
+// shared memory. Only the flags use cluster barriers: "gfull" (ring slot written) in the
+// consumer, "gfree" (ring slot read) in each producer. Every wait is bounded.
 #include "common.cuh"
 #include "launchers.h"
 #include "tc.cuh"
@@ -33,7 +41,7 @@ using namespace tc;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;          // 16 warps: latency hiding for the CUDA-core phases
 constexpr int kProducers = 3;
 constexpr int kCluster = 1 + kProducers;
 constexpr float kHalfRange = 80.f;
@@ -41,75 +49,75 @@ constexpr long long kWaitCycles = 4000000000LL;
 constexpr int kLd = 68;                // fp32 row stride of the 64x64 scratch (16-byte rows)
 constexpr int kLdY = 24;               // row stride of the per-warp 16x16 merge scratch
 
-// ---- consumer shared memory: two ring slots, then the state operands ----
-// A slot holds one chunk's operands. The order inside a slot alternates so that the wide
-// MMAs see adjacent B operands matching adjacent TMEM accumulators:
-//   slot 0: [Z | Lq] (MN-major, N = 128) -> [X0 | O0];  [P | R] (K-major rows, N = 192) -> [O0 | S]
-//   slot 1: [Lq | Z]                      -> [O1 | X1];  [R | P]                      -> [S | O1]
-constexpr uint32_t kSlotBytes = 83968;
-struct SlotMap { uint32_t zo, lq, po, rt; };
-__device__ __forceinline__ SlotMap slot_map(int slot) {
-    return slot == 0 ? SlotMap{0u, 16384u, 32768u, 40960u} : SlotMap{16384u, 0u, 49152u, 32768u};
-}
-constexpr uint32_t S_TP = 57344;      // T'   : B, K-major rows token r, K = token i
-constexpr uint32_t S_VT = 65536;      // V^T  : A, MN-major, K = token, M = value ch (2 blocks)
-constexpr uint32_t kFacBytes = 1536;  // per chunk: eRef[128], eC[128], eCR[128] (fp32)
-constexpr uint32_t C_SLOT0 = 0;
-constexpr uint32_t C_ST = 2 * kSlotBytes;       // Sm  : A, K-major rows value ch, K = key ch (2 atom cols)
-constexpr uint32_t C_UT = C_ST + 32768;         // Ut^T: A, K-major rows value ch, K = token
-constexpr uint32_t C_FAC = C_UT + 16384;        // factor ring: chunk n in entry n % 3, so a
-                                                // ring slot can be released before they are read
-constexpr uint32_t C_MISC = C_FAC + 3 * kFacBytes;
+// ---- one chunk's hand-off (identical image in the producer's staging and a consumer slot) ----
+constexpr uint32_t S_YW = 0;          // [Yh^T (rows key ch 0..127) | Wh^T (rows token 0..63)]:
+                                      //   K-major (K = token), one 128B-swizzled atom column
+constexpr uint32_t S_GQ = 24576;      // [Gm | Qh]: MN-major (K = key ch), three 64-wide N atoms
+constexpr uint32_t S_FAC = 73728;     // e^{gamma_ref}[128], e^{gamma_C}[128] (fp32)
+constexpr uint32_t kSlotBytes = 74752;
+constexpr int kRing = 4;                                // global ring slots per consumer SM
+
+// ---- consumer shared memory ----
+constexpr uint32_t C_SLOT0 = 0;                       // two slots
+constexpr uint32_t C_V = 2 * kSlotBytes;              // V ring, 3 x (two 64-ch SW128 boxes)
+constexpr uint32_t C_OST = C_V + 3 * 16384;           // O staging [64 tokens][128 ch] bf16
+constexpr uint32_t C_MISC = C_OST + 16384;
 // ---- producer shared memory ----
-constexpr uint32_t P_XQ = 0;          // raw q [64][128] bf16
-constexpr uint32_t P_XK = 16384;      // raw k [64][128] bf16
-constexpr uint32_t P_LK = 32768;      // Lk: first M block of the A|P A operand; K-major A of Z
-constexpr uint32_t P_HS = 49152;      // two hand-off sets (alternate tasks), each:
-constexpr uint32_t H_LQ = 0;          //   Lq (second M block of the A|P A operand)
-constexpr uint32_t H_RT = 16384;      //   R
-constexpr uint32_t H_ZO = 32768;      //   Z (exact path: A in fp32 until the inverse starts)
-constexpr uint32_t H_TP = 49152;      //   T'
-constexpr uint32_t H_PO = 57344;      //   P
-constexpr uint32_t H_FAC = 65536;     //   eRef, eC, eCR
-constexpr uint32_t kHsBytes = 67584;
-constexpr uint32_t kHandoffTx = 16384 * 3 + 8192 * 2 + 1536;   // bytes bulk-copied per chunk
-constexpr uint32_t P_SCR = P_HS + 2 * kHsBytes;   // raw g / gamma [64][128] f32, then
-                                                  // Nm [64][68], Tm [64][68], Y [3][16][24] (fp32)
-constexpr uint32_t P_XG = P_SCR;
-constexpr uint32_t P_MISC = P_SCR + 40960;
-constexpr uint32_t kMiscBytes = 2560;   // barriers, beta[64], decay sums [4][128]
+constexpr uint32_t P_X = 0;           // raw q, k [64][128] bf16 (folds), then the inverse's
+                                      // scratch Nm, Tm [64][68], Y [3][16][24] (fp32)
+constexpr uint32_t P_LK = 40960;      // Lk : rows key ch, K = token (A|P A block 0; K-major A)
+constexpr uint32_t P_LQ = 57344;      // Lq: same layout (A|P A block 1; K-major A)
+constexpr uint32_t P_RT = 73728;      // R  : B of A|P. Raw g (fp32, 32 KB) spans P_RT..P_RH
+constexpr uint32_t P_RH = 90112;      // Rh : K-major A of Yh^T
+constexpr uint32_t P_PO = 106496;     // P' : rows token, K = token (K-major A of Wh^T; the
+                                      //      M = 128 padding rows read T' below)
+constexpr uint32_t P_TP = 114688;     // T' : rows token, columns token (MN-major B)
+constexpr uint32_t P_ID = 122880;     // identity 64x64 (K-major B of the Lq term)
+constexpr uint32_t P_ST = 131072;     // hand-off staging (S_YW, S_GQ); exact path: Aex, gamma
+constexpr uint32_t P_MISC = P_ST + kSlotBytes;
+constexpr uint32_t kMiscBytes = 2560;
 constexpr uint32_t kSmemBytes = (P_MISC > C_MISC ? P_MISC : C_MISC) + kMiscBytes + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(320 + 4 * 128 * 4 <= kMiscBytes, "misc area");
+static_assert(2 * kC * kLd * 4 + 4 * 16 * kLdY * 4 <= P_LK, "inverse scratch");
 
-// misc area (relative to the role's misc base)
-constexpr uint32_t M_BAR_MMA = 0;     // own MMA completions
-constexpr uint32_t M_BAR_A = 8;       // consumer: full[0]; producer: free
-constexpr uint32_t M_BAR_B = 16;      // consumer: full[1]
-constexpr uint32_t M_TMEM = 24;
-constexpr uint32_t M_TMP = 32;
-constexpr uint32_t M_BAR_C = 40;      // producer: q, k tiles landed; consumer: V tile of slot 0
-constexpr uint32_t M_BAR_D = 48;      // producer: g tile landed;    consumer: V tile of slot 1
-constexpr uint32_t M_BETA = 64;       // producer: beta[64]
-constexpr uint32_t M_GSUM = 320;      // producer: [4][128] token-quarter decay sums
+// misc areas: 12 mbarriers at 8-byte steps, then scalars
+constexpr uint32_t kBars = 12;
+constexpr uint32_t M_TMEM = 96;
+constexpr uint32_t M_TMP = 100;       // unit_of scratch
+constexpr uint32_t M_SMID = 104;      // consumer: its SM id (selects the global ring)
+// consumer
+constexpr uint32_t M_BAR_S = 0;       // chain MMAs up to the state part
+constexpr uint32_t M_BAR_O = 8;       // chain MMAs up to the output part
+constexpr uint32_t M_LFULL = 16;      // shared slot [2] loaded from the ring
+constexpr uint32_t M_BAR_V = 32;      // V ring [3]
+constexpr uint32_t M_GFULL = 56;      // global ring slot [4] written (producer arrival)
+// producer
+constexpr uint32_t M_BAR_MMA = 0;
+constexpr uint32_t M_BAR_QK = 8;
+constexpr uint32_t M_BAR_G = 16;
+constexpr uint32_t M_GFREE = 24;      // [4] per ring slot: its previous chunk was read (one barrier
+                                      // per slot, so arrivals for later chunks never overrun)
+constexpr uint32_t M_BETA = 128;      // beta[64]
+constexpr uint32_t M_GSUM = 384;      // [4][128] token-quarter decay sums
+static_assert(M_GSUM + 4 * 128 * 4 <= kMiscBytes && M_GFULL + 8 * kRing <= 8 * kBars &&
+              M_GFREE + 8 * kRing <= M_GFULL, "misc area");
 
-// consumer TMEM columns: [X0 | O0 | S(128) | .. | O1 | X1]; producer: [A|P | Z]
-constexpr uint32_t TC_X0 = 0, TC_O0 = 64, TC_S = 128, TC_O1 = 256, TC_X1 = 320, kTmemC = 512;
-constexpr uint32_t TP_AP = 0, TP_Z = 64, kTmemP = 128;
+// consumer TMEM columns: D0 = [S part (128) | O part (64)], D1 likewise, Sm (64 cols of bf16 pairs)
+constexpr uint32_t TD0 = 0, TD1 = 256, TC_SM = 448, kTmemC = 512;
+// producer TMEM columns
+constexpr uint32_t TP_AP = 0, TP_Y = 64, TP_W = 128, TP_GQ = 256, kTmemP = 512;
 
 struct Params {
     CUtensorMap tq, tk, tg, tv, to;   // TMA maps: q, k, o [T,H,128] bf16 and g [T,H,128] f32 in
                                       // (128, 1, 64) boxes; v in (64, 1, 64) boxes, 128B swizzle
-    const __nv_bfloat16* q;
-    const __nv_bfloat16* k;
-    const __nv_bfloat16* v;
-    const float* g;
     const float* beta;
     float scale;
     const float* h0;
     float* ht;
     __nv_bfloat16* o;
     const int32_t* cu;
+    uint8_t* ring;                    // workspace: ring_sms x kRing x kSlotBytes
+    int ring_sms;
     int T_pad;
     int N, H;
     unsigned int* err;
@@ -122,6 +130,24 @@ __device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162
 __device__ __forceinline__ uint4 pack8(const float* v) {
     return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
                       pack_bf16(v[6], v[7]));
+}
+
+// Block-wide bounded wait for the phase of `bar` with the given parity: one thread polls (the
+// other 15 warps sleep in the block barrier instead of taking issue slots from the warp that
+// issues MMAs); false for every thread if the wait gave up.
+constexpr int kPoller = kThreads - 32;
+__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, bool cluster_scope,
+                                           unsigned int* err) {
+    int fail = 0;
+    if (threadIdx.x == kPoller) {
+        const bool ok = cluster_scope ? mbar_wait_cluster_bounded(bar, parity, kWaitCycles)
+                                      : mbar_wait_bounded(bar, parity, kWaitCycles);
+        if (!ok) {
+            atomicOr(err, kErrTimeout);
+            fail = 1;
+        }
+    }
+    return __syncthreads_or(fail) == 0;
 }
 
 // Sequence / head of this cluster. Packed batches with at most 256 sequences are processed
@@ -155,6 +181,41 @@ __device__ void unit_of(const Params& p, int unit, int* s_tmp, int& n, int& h, i
     }
 }
 
+// Exact A and P on CUDA cores for a chunk whose decay fails the range test (one warp per (r, i)
+// pair, lanes over channels): A (times beta) into an fp32 [64][64] scratch in the hand-off
+// staging, P into its bf16 operand. Rare, so kept out of line, away from the common path's
+// instruction stream. Every thread of the CTA calls it.
+__device__ __noinline__ void exact_ap(uint8_t* sm, const float* s_beta, int L) {
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const __nv_bfloat16* Xq = reinterpret_cast<const __nv_bfloat16*>(sm + P_X);
+    const __nv_bfloat16* Xk = reinterpret_cast<const __nv_bfloat16*>(sm + P_X + 16384);
+    __nv_bfloat16* Pop = reinterpret_cast<__nv_bfloat16*>(sm + P_PO);
+    const float* Gx = reinterpret_cast<const float*>(sm + P_ST + S_GQ);
+    float* Aex = reinterpret_cast<float*>(sm + P_ST + S_YW);        // [64][64]
+    const int lane = tid & 31;
+    for (int pidx = warp; pidx < kC * (kC + 1) / 2; pidx += kThreads / 32) {
+        int r = (int)((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
+        while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
+        while (r * (r + 1) / 2 > pidx) --r;
+        const int i = pidx - r * (r + 1) / 2;
+        float a = 0.f, pp = 0.f;
+        for (int cc = lane; cc < kD && r < L; cc += 32) {
+            const float ki = bf(Xk + i * kD + cc) * expf(Gx[r * kD + cc] - Gx[i * kD + cc]);
+            a = fmaf(bf(Xk + r * kD + cc), ki, a);
+            pp = fmaf(bf(Xq + r * kD + cc), ki, pp);
+        }
+        a = warp_sum(a);
+        pp = warp_sum(pp);
+        if (lane == 0) {
+            Aex[r * 64 + i] = (i < r) ? s_beta[r] * a : 0.f;
+            Aex[i * 64 + r] = (i < r) ? 0.f : Aex[i * 64 + r];
+            Pop[(kmaj_chunk(r, i >> 3, 0, 64) + (i & 7) * 2) / 2] = __float2bfloat16_rn(pp);
+            if (i < r) Pop[(kmaj_chunk(i, r >> 3, 0, 64) + (r & 7) * 2) / 2] = __float2bfloat16_rn(0.f);
+        }
+    }
+    __syncthreads();
+}
+
 // ============================== producer ==============================
 __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, int h,
                          int64_t bos, int64_t eos, bool& aborted) {
@@ -162,271 +223,277 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
     const uint32_t lane_sel = (uint32_t)(32 * (warp & 3)) << 16;
     uint8_t* misc = sm + P_MISC;
     uint64_t* bar_mma = reinterpret_cast<uint64_t*>(misc + M_BAR_MMA);
-    uint64_t* bar_free = reinterpret_cast<uint64_t*>(misc + M_BAR_A);
+    uint64_t* bar_qk = reinterpret_cast<uint64_t*>(misc + M_BAR_QK);
+    uint64_t* bar_g = reinterpret_cast<uint64_t*>(misc + M_BAR_G);
+    uint64_t* bar_gfree = reinterpret_cast<uint64_t*>(misc + M_GFREE);
     float* s_beta = reinterpret_cast<float*>(misc + M_BETA);
     float* s_gsum = reinterpret_cast<float*>(misc + M_GSUM);
     const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
     const int H = p.H;
     const int nchunks = (int)((eos - bos + kC - 1) / kC);
-    uint32_t ph_mma = 0, ph_free = 0;
+    uint32_t ph_mma = 0, ph_qk = 0, ph_g = 0, ph_gfree = 0;   // ph_gfree: bit per ring slot
 
     const uint32_t c_misc = map_to_rank(sb + C_MISC, 0);
-    const uint32_t c_slot0 = map_to_rank(sb + C_SLOT0, 0);
-    const uint32_t c_fac = map_to_rank(sb + C_FAC, 0);
-
-    auto wait_mma = [&]() -> bool {
-        const bool ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitCycles);
-        ph_mma ^= 1u;
-        if (!ok) atomicOr(p.err, kErrTimeout);
-        return __syncthreads_or(!ok) == 0;
+    uint8_t* ring = p.ring + (size_t)ld_cluster_u32(c_misc + M_SMID) * (kRing * kSlotBytes);
+    // Chunk whose ring store (one bulk copy by thread 0) was issued but not yet announced (-1:
+    // none). It is announced when the next chunk is handed off, a whole task later, so the wait
+    // for its completion is normally free: thread 0 waits for its bulk group, then arrives on
+    // the consumer's "gfull" barrier of that ring slot.
+    int pending = -1;
+    auto announce = [&]() {
+        if (tid == 0 && pending >= 0) {
+            bulk_wait0();
+            fence_proxy_async_global();
+            mbar_arrive_remote(c_misc + M_GFULL + 8u * (uint32_t)(pending % kRing));
+        }
+        pending = -1;
     };
-    // Raw q, k tiles (staging, free after the folds) and g tile (in the inverse's scratch,
-    // free once T' is written) of a chunk, by TMA from one thread. Rows past the sequence are
-    // masked where they are read; rows past the whole batch arrive as zeros.
-    uint64_t* bar_qk = reinterpret_cast<uint64_t*>(misc + M_BAR_C);
-    uint64_t* bar_g = reinterpret_cast<uint64_t*>(misc + M_BAR_D);
-    uint32_t ph_qk = 0, ph_g = 0;
-    auto issue_loads = [&](int64_t c0, int) {
+
+    auto wait_local = [&](uint64_t* bar, uint32_t& ph) -> bool {
+        const bool ok = block_wait(bar, ph, false, p.err);
+        ph ^= 1u;
+        return ok;
+    };
+    // raw q, k tiles of a chunk (into P_X) and its g tile (into P_RT..P_RH), by TMA from one
+    // thread. Rows past the sequence are masked where they are read; rows past the whole
+    // batch arrive as zeros.
+    auto issue_qk = [&](int64_t c0) {
         if (tid == 0) {
             mbar_arrive_expect_tx(bar_qk, 32768u);
-            tma_load_3d(sb + P_XQ, &p.tq, 0, h, (int)c0, bar_qk);
-            tma_load_3d(sb + P_XK, &p.tk, 0, h, (int)c0, bar_qk);
+            tma_load_3d(sb + P_X, &p.tq, 0, h, (int)c0, bar_qk);
+            tma_load_3d(sb + P_X + 16384, &p.tk, 0, h, (int)c0, bar_qk);
         }
     };
     auto issue_g = [&](int64_t c0) {
         if (tid == 0) {
             mbar_arrive_expect_tx(bar_g, 32768u);
-            tma_load_3d(sb + P_XG, &p.tg, 0, h, (int)c0, bar_g);
+            tma_load_3d(sb + P_RT, &p.tg, 0, h, (int)c0, bar_g);
         }
     };
-    auto wait_load = [&](uint64_t* bar, uint32_t& ph) -> bool {
-        const bool ok = mbar_wait_bounded(bar, ph, kWaitCycles);
-        ph ^= 1u;
-        if (!ok) atomicOr(p.err, kErrTimeout);
-        return __syncthreads_or(!ok) == 0;
-    };
+
+    // identity (B operand of the Lq term of Qh), written once
+    for (int e = tid; e < kC * 8; e += kThreads) {
+        const int r = e >> 3, q8 = e & 7;
+        float v8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v8[u] = (8 * q8 + u == r) ? 1.f : 0.f;
+        st16(sm, P_ID + kmaj_chunk(r, q8, 0, 64), pack8(v8));
+    }
 
     int n = prank - 1;
     if (n < nchunks) {
         const int64_t c0 = bos + (int64_t)n * kC;
-        issue_loads(c0, 0);
+        issue_qk(c0);
         issue_g(c0);
     }
     for (int task = 0; n < nchunks && !aborted; n += kProducers, ++task) {
         const int64_t c0 = bos + (int64_t)n * kC;
         const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
-        const int slot = n & 1;
-        const uint32_t hs = P_HS + (uint32_t)(task & 1) * kHsBytes;     // this task's hand-off set
-        float* fac = reinterpret_cast<float*>(sm + hs + H_FAC);
+        const bool has_next = n + kProducers < nchunks;
+        const int64_t c_next = c0 + (int64_t)kProducers * kC;
         if (tid < kC) s_beta[tid] = tid < L ? p.beta[(c0 + tid) * H + h] : 0.f;
-        if (!wait_load(bar_qk, ph_qk) || !wait_load(bar_g, ph_g)) { aborted = true; break; }
+        if (!wait_local(bar_qk, ph_qk) || !wait_local(bar_g, ph_g)) { aborted = true; break; }
         trace_mark(prank, n, 0);
 
-        // ---- cumulative decay (thread: channels 2*cp, 2*cp+1; tokens [16*tq, 16*tq+16)) ----
-        // kept in log2 units so that every decay factor is one ex2.approx
-        const int cp = tid & 63, tq = tid >> 6;
-        const int c = row;                      // channel owned for the factors below
-        float* Xg = reinterpret_cast<float*>(sm + P_XG);
-        const uint32_t* Xq2 = reinterpret_cast<const uint32_t*>(sm + P_XQ);
-        const uint32_t* Xk2 = reinterpret_cast<const uint32_t*>(sm + P_XK);
-        const __nv_bfloat16* Xq = reinterpret_cast<const __nv_bfloat16*>(sm + P_XQ);
-        const __nv_bfloat16* Xk = reinterpret_cast<const __nv_bfloat16*>(sm + P_XK);
+        // ---- cumulative decay (thread: channel c = row, tokens [16*qt, 16*qt + 16)) ----
+        // kept in log2 units so that every decay factor is one ex2.approx. Lanes run over
+        // consecutive channels, so every 16-byte store below hits 8 distinct swizzled bank groups.
+        const int c = row, qt = wg;
+        const float* Xg = reinterpret_cast<const float*>(sm + P_RT);
+        const __nv_bfloat16* Xq = reinterpret_cast<const __nv_bfloat16*>(sm + P_X);
+        const __nv_bfloat16* Xk = reinterpret_cast<const __nv_bfloat16*>(sm + P_X + 16384);
         constexpr float kLog2e = 1.4426950408889634f;
-        float gam0[16], gam1[16];
+        float gam[16];
         {
-            float a0 = 0.f, a1 = 0.f;
+            float a0 = 0.f;
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
-                const int r = 16 * tq + t;
-                const float2 gv = r < L ? *reinterpret_cast<const float2*>(Xg + r * kD + 2 * cp)
-                                        : make_float2(0.f, 0.f);
-                a0 = fmaf(gv.x, kLog2e, a0);
-                a1 = fmaf(gv.y, kLog2e, a1);
-                gam0[t] = a0;
-                gam1[t] = a1;
+                const int r = 16 * qt + t;
+                a0 = fmaf(r < L ? Xg[r * kD + c] : 0.f, kLog2e, a0);
+                gam[t] = a0;
             }
-            s_gsum[tq * 128 + 2 * cp] = a0;
-            s_gsum[tq * 128 + 2 * cp + 1] = a1;
+            s_gsum[qt * 128 + c] = a0;
         }
-        __syncthreads();
-        float off0 = 0.f, off1 = 0.f;           // decay of the earlier token quarters
-        for (int k2 = 0; k2 < tq; ++k2) { off0 += s_gsum[k2 * 128 + 2 * cp]; off1 += s_gsum[k2 * 128 + 2 * cp + 1]; }
+        __syncthreads();                        // the g tile is dead from here on
+        const float q0s = s_gsum[c], q1s = s_gsum[128 + c], q2s = s_gsum[256 + c], q3s = s_gsum[384 + c];
+        const float off = qt == 0 ? 0.f : (qt == 1 ? q0s : (qt == 2 ? q0s + q1s : q0s + q1s + q2s));
 #pragma unroll
-        for (int t = 0; t < 16; ++t) { gam0[t] += off0; gam1[t] += off1; }
-        // per channel c (thread row): half-chunk decays, in log2 units
-        const float gA2 = s_gsum[c] + s_gsum[128 + c];                 // tokens 0..31
-        const float gB2 = s_gsum[256 + c] + s_gsum[384 + c];           // tokens 32..63
+        for (int t = 0; t < 16; ++t) gam[t] += off;
+        const float gA = q0s + q1s, gB = q2s + q3s;           // half-chunk decays (log2)
         const float kHalf2 = kHalfRange * kLog2e;
-        const int bad = __syncthreads_or((gA2 < -kHalf2) || (gB2 < -kHalf2));
-        // references per channel pair (this thread's channels), log2 units
-        const float gm0 = s_gsum[2 * cp] + s_gsum[128 + 2 * cp], gm1 = s_gsum[2 * cp + 1] + s_gsum[128 + 2 * cp + 1];
-        const float gC0 = gm0 + s_gsum[256 + 2 * cp] + s_gsum[384 + 2 * cp];
-        const float gC1 = gm1 + s_gsum[256 + 2 * cp + 1] + s_gsum[384 + 2 * cp + 1];
-        const float gr0 = bad ? 0.f : gm0, gr1 = bad ? 0.f : gm1;      // reference for Lk / Lq
-        const float gs0 = bad ? gC0 : gm0, gs1 = bad ? gC1 : gm1;      // reference for R
-        if (tq == 0) {
-            fac[2 * cp] = ex2_approx(gr0);
-            fac[2 * cp + 1] = ex2_approx(gr1);
-            fac[128 + 2 * cp] = ex2_approx(gC0);
-            fac[128 + 2 * cp + 1] = ex2_approx(gC1);
-            fac[256 + 2 * cp] = ex2_approx(gC0 - gs0);
-            fac[256 + 2 * cp + 1] = ex2_approx(gC1 - gs1);
-        }
-        if (bad) {                              // natural-log gamma for the exact path
+        const int bad = __syncthreads_or((gA < -kHalf2) || (gB < -kHalf2));
+        const float gC = gA + gB;
+        const float gr = bad ? 0.f : gA;        // reference for Lk, Lq, R (token 31, or 0)
+        const float gs = bad ? gC : gA;         // R's reference (the exact path does not use R)
+        const float rhf = ex2_approx(gC - gs);  // Rh = R * rhf
+        // this chunk's factors, written into the staging once the previous ring store read it
+        const float fac_r = ex2_approx(gr), fac_c = ex2_approx(gC);
+        if (bad) {
+            // exact path: natural-log gamma goes to the hand-off staging, which the previous
+            // chunk's ring store must have read
+            if (tid == 0) bulk_wait_read0();
+            __syncthreads();
+            float* Gx = reinterpret_cast<float*>(sm + P_ST + S_GQ);
 #pragma unroll
-            for (int t = 0; t < 16; ++t)
-                *reinterpret_cast<float2*>(Xg + (16 * tq + t) * kD + 2 * cp) =
-                    make_float2(gam0[t] * (1.f / kLog2e), gam1[t] * (1.f / kLog2e));
+            for (int t = 0; t < 16; ++t) Gx[(16 * qt + t) * kD + c] = gam[t] * (1.f / kLog2e);
         }
-        // ---- folded operands Lk, Lq (A of A|P), R (B of A|P) ----
+        // ---- folded operands Lk, Lq (A of A|P), R (B of A|P), Rh: 8 tokens per 16-byte store ----
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-            float lk0[8], lq0[8], rr0[8], lk1[8], lq1[8], rr1[8];
+        for (int q8 = 0; q8 < 2; ++q8) {
+            float lk[8], lq[8], rr[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int t = 8 * qq + u;
-                const int r = 16 * tq + t;
+                const int t = 8 * q8 + u;
+                const int r = 16 * qt + t;
                 const bool ok = r < L;
-                const uint32_t kw = ok ? Xk2[r * 64 + cp] : 0u, qw = ok ? Xq2[r * 64 + cp] : 0u;
-                const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xffff0000u);
-                const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xffff0000u);
-                const float a0 = ex2_approx(gam0[t] - gr0), b0 = ex2_approx(gs0 - gam0[t]);
-                const float a1 = ex2_approx(gam1[t] - gr1), b1 = ex2_approx(gs1 - gam1[t]);
-                lk0[u] = k0 * a0; lq0[u] = q0 * a0; rr0[u] = k0 * b0;
-                lk1[u] = k1 * a1; lq1[u] = q1 * a1; rr1[u] = k1 * b1;
+                const float kv = ok ? __bfloat162float(Xk[r * kD + c]) : 0.f;
+                const float qv = ok ? __bfloat162float(Xq[r * kD + c]) : 0.f;
+                const float a = ex2_approx(gam[t] - gr), b = ex2_approx(gs - gam[t]);
+                lk[u] = kv * a; lq[u] = qv * a; rr[u] = kv * b;
             }
-            const int ch = 2 * tq + qq;         // 8-token chunk index within the 64 tokens
-            st16(sm, P_LK + mnmaj_chunk(2 * cp, ch, 0, 16), pack8(lk0));
-            st16(sm, P_LK + mnmaj_chunk(2 * cp + 1, ch, 0, 16), pack8(lk1));
-            st16(sm, hs + H_LQ + mnmaj_chunk(2 * cp, ch, 0, 16), pack8(lq0));
-            st16(sm, hs + H_LQ + mnmaj_chunk(2 * cp + 1, ch, 0, 16), pack8(lq1));
-            st16(sm, hs + H_RT + mnmaj_chunk(2 * cp, ch, 0, 16), pack8(rr0));
-            st16(sm, hs + H_RT + mnmaj_chunk(2 * cp + 1, ch, 0, 16), pack8(rr1));
+            const int ch = 2 * qt + q8;         // 8-token chunk index within the 64 tokens
+            st16(sm, P_LK + mnmaj_chunk(c, ch, 0, 16), pack8(lk));
+            st16(sm, P_LQ + mnmaj_chunk(c, ch, 0, 16), pack8(lq));
+            st16(sm, P_RT + mnmaj_chunk(c, ch, 0, 16), pack8(rr));
+#pragma unroll
+            for (int u = 0; u < 8; ++u) rr[u] *= rhf;
+            st16(sm, P_RH + mnmaj_chunk(c, ch, 0, 16), pack8(rr));
         }
         fence_async_smem();
         __syncthreads();
         trace_mark(prank, n, 1);
 
-        float* Nm = reinterpret_cast<float*>(sm + P_SCR);
-        __nv_bfloat16* Pop = reinterpret_cast<__nv_bfloat16*>(sm + hs + H_PO);
+        float* Nm = reinterpret_cast<float*>(sm + P_X);
+        __nv_bfloat16* Pop = reinterpret_cast<__nv_bfloat16*>(sm + P_PO);
         if (!bad) {
-            // raw inputs are no longer needed: prefetch this producer's next chunk
-            if (n + kProducers < nchunks) {
-                const int64_t c1 = c0 + (int64_t)kProducers * kC;
-                issue_loads(c1, (int)(eos - c1 < kC ? eos - c1 : kC));
-            }
-            trace_mark(prank, n, 9);
             if (warp == 0) {
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 64, true, true);
-                const uint64_t a0 = make_desc(sb + P_LK, hs + H_LQ - P_LK, 1024);
-                const uint64_t b0 = make_desc(sb + hs + H_RT, 16384, 1024);
+                const uint64_t a0 = make_desc(sb + P_LK, P_LQ - P_LK, 1024);
+                const uint64_t b0 = make_desc(sb + P_RT, 16384, 1024);
+                if (elect_one()) {
 #pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    warp_mma(tm + TP_AP, desc_add(a0, s * 2048), desc_add(b0, s * 2048), id, s > 0);
-                warp_commit(bar_mma);
-                trace_mark(prank, n, 10);
+                    for (int s = 0; s < 8; ++s)
+                        mma_bf16(tm + TP_AP, desc_add(a0, s * 2048), desc_add(b0, s * 2048), id, s > 0);
+                    mma_commit(bar_mma);
+                }
+                __syncwarp();
             }
-            if (!wait_mma()) { aborted = true; break; }
+            if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
             trace_mark(prank, n, 2);
             tc_fence_after();
-            float val[32];
-            tmem_ld32(tm + lane_sel + TP_AP + 32 * wg, val);
-            const int i0 = 32 * wg;
+            float val[16];
+            tmem_ld16(tm + lane_sel + TP_AP + 16 * wg, val);
+            const int i0 = 16 * wg;
             if (row < 64) {
                 const int r = row;
                 const float br = s_beta[r];
 #pragma unroll
-                for (int ii = 0; ii < 32; ++ii) Nm[r * kLd + i0 + ii] = (i0 + ii < r) ? br * val[ii] : 0.f;
+                for (int i4 = 0; i4 < 4; ++i4) {
+                    float4 w;
+                    w.x = (i0 + 4 * i4 + 0 < r) ? br * val[4 * i4 + 0] : 0.f;
+                    w.y = (i0 + 4 * i4 + 1 < r) ? br * val[4 * i4 + 1] : 0.f;
+                    w.z = (i0 + 4 * i4 + 2 < r) ? br * val[4 * i4 + 2] : 0.f;
+                    w.w = (i0 + 4 * i4 + 3 < r) ? br * val[4 * i4 + 3] : 0.f;
+                    *reinterpret_cast<float4*>(Nm + r * kLd + i0 + 4 * i4) = w;
+                }
             } else {
                 const int r = row - 64;
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
+                for (int qq = 0; qq < 2; ++qq) {
                     float pv[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) pv[u] = (i0 + 8 * qq + u <= r) ? val[8 * qq + u] : 0.f;
-                    st16(sm, hs + H_PO + kmaj_chunk(r, (i0 >> 3) + qq, 0, 64), pack8(pv));
+                    st16(sm, P_PO + kmaj_chunk(r, (i0 >> 3) + qq, 0, 64), pack8(pv));
                 }
             }
         } else {
-            // exact A and P on CUDA cores (one warp per (r, i) pair, lanes over channels)
-            const int lane = tid & 31;
-            for (int pidx = warp; pidx < kC * (kC + 1) / 2; pidx += kThreads / 32) {
-                int r = (int)((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
-                while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
-                while (r * (r + 1) / 2 > pidx) --r;
-                const int i = pidx - r * (r + 1) / 2;
-                float a = 0.f, pp = 0.f;
-                for (int cc = lane; cc < kD && r < L; cc += 32) {
-                    const float ki = bf(Xk + i * kD + cc) * expf(Xg[r * kD + cc] - Xg[i * kD + cc]);
-                    a = fmaf(bf(Xk + r * kD + cc), ki, a);
-                    pp = fmaf(bf(Xq + r * kD + cc), ki, pp);
-                }
-                a = warp_sum(a);
-                pp = warp_sum(pp);
-                if (lane == 0) {
-                    float* Aex = reinterpret_cast<float*>(sm + hs + H_ZO);     // [64][64]
-                    Aex[r * 64 + i] = (i < r) ? s_beta[r] * a : 0.f;
-                    Aex[i * 64 + r] = (i < r) ? 0.f : Aex[i * 64 + r];
-                    Pop[(kmaj_chunk(r, i >> 3, 0, 64) + (i & 7) * 2) / 2] = __float2bfloat16_rn(pp);
-                    if (i < r) Pop[(kmaj_chunk(i, r >> 3, 0, 64) + (r & 7) * 2) / 2] = __float2bfloat16_rn(0.f);
-                }
-            }
-            __syncthreads();
-            if (n + kProducers < nchunks) {
-                const int64_t c1 = c0 + (int64_t)kProducers * kC;
-                issue_loads(c1, (int)(eos - c1 < kC ? eos - c1 : kC));
-            }
-            // gamma (in the scratch) is dead: move diag(beta) A into place
-            const float* Aex = reinterpret_cast<const float*>(sm + hs + H_ZO);
+            exact_ap(sm, s_beta, L);
+            const float* Aex = reinterpret_cast<const float*>(sm + P_ST + S_YW);
+            // the raw tiles are dead: move diag(beta) A into the inverse's scratch
             for (int e = tid; e < kC * kC; e += kThreads) Nm[(e >> 6) * kLd + (e & 63)] = Aex[e];
         }
         __syncthreads();
         trace_mark(prank, n, 3);
 
-        // ---- T' = (I + N)^-1 diag(beta) in fp32 ----
-        // 16x16 diagonal blocks by column substitution (fp32), then the block merges
-        // T[b+d][b] = -T[b+d][b+d] * sum_{j=b}^{b+d-1} N[b+d][j] T[j][b] as warp-level
-        // tensor-core products (TF32 inputs, fp32 accumulation); T' is rounded to bf16 afterwards.
+        // ---- T' = (I + N)^-1 diag(beta) in fp32, N = diag(beta) A ----
+        // Block recursion on the unit lower triangular matrix: the inverse of [[A, 0], [B, C]]
+        // is [[A^-1, 0], [-C^-1 B A^-1, C^-1]]. 8x8 diagonal blocks by column substitution,
+        // then 8 -> 16 on CUDA cores (fp32), 16 -> 32 -> 64 as warp-level tensor-core products
+        // (TF32 inputs, fp32 sums). T' is rounded to bf16 afterwards.
         {
             float* Tm = Nm + kC * kLd;
-            float* Y = Tm + kC * kLd;                     // [3 warps][16][kLdY]
-            if (tid < 64) {
-                const int b = tid >> 4, i = tid & 15;
-                float x[16];
+            float* Y = Tm + kC * kLd;                     // [4][16][kLdY] products / [4][8][8]
+            if (tid < 64) {                               // level 0: block b, column i
+                const int b = tid >> 3, i = tid & 7;
+                const float* Nb = Nm + (8 * b) * kLd + 8 * b;
+                float x[8];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float s0 = 0.f, s1 = 0.f;
+                for (int r = 0; r < 8; ++r) {
+                    float s0 = 0.f;
 #pragma unroll
-                    for (int m = 0; m + 1 < r; m += 2) {
-                        s0 = fmaf(Nm[(16 * b + r) * kLd + 16 * b + m], x[m], s0);
-                        s1 = fmaf(Nm[(16 * b + r) * kLd + 16 * b + m + 1], x[m + 1], s1);
-                    }
-                    if (r & 1) s0 = fmaf(Nm[(16 * b + r) * kLd + 16 * b + r - 1], x[r - 1], s0);
-                    x[r] = (r < i) ? 0.f : (r == i ? 1.f : -(s0 + s1));
-                    Tm[(16 * b + r) * kLd + 16 * b + i] = x[r];
+                    for (int m = 0; m < r; ++m) s0 = fmaf(Nb[r * kLd + m], x[m], s0);
+                    x[r] = (r < i) ? 0.f : (r == i ? 1.f : -s0);
+                    Tm[(8 * b + r) * kLd + 8 * b + i] = x[r];
                 }
             }
             __syncthreads();
-            trace_mark(prank, n, 11);
-            // block merges on the tensor cores: warp w < 4 - d owns block (w + d, w)
-            for (int d = 1; d <= 3; ++d) {
-                if (warp < 4 - d) {
-                    const int b = warp, B = warp + d;
-                    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                    for (int jb = b; jb < B; ++jb)
-                        warp_block_mma16(acc, Nm + (16 * B) * kLd + 16 * jb, kLd, Tm + (16 * jb) * kLd + 16 * b, kLd);
-                    float* Yw = Y + warp * 16 * kLdY;
-                    warp_block_store16(Yw, kLdY, acc, 1.f);
-                    __syncwarp();
-                    float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                    warp_block_mma16(acc2, Tm + (16 * B) * kLd + 16 * B, kLd, Yw, kLdY);
-                    warp_block_store16(Tm + (16 * B) * kLd + 16 * b, kLd, acc2, -1.f);
-                }
-                __syncthreads();
-                if (d == 1) trace_mark(prank, n, 14);
-                if (d == 3) trace_mark(prank, n, 15);
+            trace_mark(prank, n, 4);
+            if (tid < 256) {                              // level 1: 16-block blk, element (r, j)
+                const int blk = tid >> 6, r = (tid >> 3) & 7, j = tid & 7, o = 16 * blk;
+                float y = 0.f;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) y = fmaf(Nm[(o + 8 + r) * kLd + o + m], Tm[(o + m) * kLd + o + j], y);
+                Y[blk * 64 + r * 8 + j] = y;
+                Tm[(o + r) * kLd + o + 8 + j] = 0.f;      // upper-right 8x8 of the 16-block
             }
+            __syncthreads();
+            if (tid < 256) {
+                const int blk = tid >> 6, r = (tid >> 3) & 7, j = tid & 7, o = 16 * blk;
+                float t = 0.f;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) t = fmaf(Tm[(o + 8 + r) * kLd + o + 8 + m], Y[blk * 64 + m * 8 + j], t);
+                Tm[(o + 8 + r) * kLd + o + j] = -t;
+            }
+            __syncthreads();
+            // level 2: 32-blocks g = 0, 1 on warps 0, 1; the other warps zero their upper-right 16x16
+            if (warp < 2) {
+                const int o = 32 * warp;
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                warp_block_mma16(acc, Nm + (o + 16) * kLd + o, kLd, Tm + o * kLd + o, kLd);
+                warp_block_store16(Y + warp * 16 * kLdY, kLdY, acc, 1.f);
+            } else {
+                for (int e = tid - 64; e < 512; e += kThreads - 64) {
+                    const int g2 = e >> 8, r = (e >> 4) & 15, j = e & 15;
+                    Tm[(32 * g2 + r) * kLd + 32 * g2 + 16 + j] = 0.f;
+                }
+            }
+            __syncthreads();
+            if (warp < 2) {
+                const int o = 32 * warp;
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                warp_block_mma16(acc, Tm + (o + 16) * kLd + o + 16, kLd, Y + warp * 16 * kLdY, kLdY);
+                warp_block_store16(Tm + (o + 16) * kLd + o, kLd, acc, -1.f);
+            }
+            __syncthreads();
+            // level 3: the lower-left 32x32 as 2x2 blocks of 16, warp w = (a, b)
+            if (warp < 4) {
+                const int a = warp >> 1, b = warp & 1;
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                for (int k2 = b; k2 < 2; ++k2)            // Y_ab = sum_k N21_ak T11_kb
+                    warp_block_mma16(acc, Nm + (32 + 16 * a) * kLd + 16 * k2, kLd, Tm + (16 * k2) * kLd + 16 * b, kLd);
+                warp_block_store16(Y + warp * 16 * kLdY, kLdY, acc, 1.f);
+            }
+            __syncthreads();
+            if (warp < 4) {
+                const int a = warp >> 1, b = warp & 1;
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                for (int k2 = 0; k2 <= a; ++k2)           // T21_ab = -sum_k T22_ak Y_kb
+                    warp_block_mma16(acc, Tm + (32 + 16 * a) * kLd + 32 + 16 * k2, kLd, Y + (2 * k2 + b) * 16 * kLdY, kLdY);
+                warp_block_store16(Tm + (32 + 16 * a) * kLd + 16 * b, kLd, acc, -1.f);
+            }
+            __syncthreads();
+            trace_mark(prank, n, 5);
             // T' = T diag(beta): 8 consecutive columns per item from two 16-byte reads
             for (int e = tid; e < kC * 8; e += kThreads) {
                 const int r = e >> 3, q8 = e & 7;
@@ -442,68 +509,119 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                     const int i = 8 * q8 + u;
                     w8[u] = (i < r) ? tv[u] * bv[u] : (i == r ? bv[u] : 0.f);
                 }
-                st16(sm, hs + H_TP + kmaj_chunk(r, q8, 0, 64), pack8(w8));
+                st16(sm, P_TP + kmaj_chunk(r, q8, 0, 64), pack8(w8));
             }
         }
-        __syncthreads();
-        if (n + kProducers < nchunks) issue_g(c0 + (int64_t)kProducers * kC);
-        trace_mark(prank, n, 4);
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (has_next) issue_qk(c_next);         // the inverse's scratch is dead
+        trace_mark(prank, n, 6);
 
-        // ---- Z = Lk^T T'^T ----
+        // ---- Yh^T = Rh^T T' (M = key ch) and Wh^T = P' T' (M = token, 64 rows of 128) ----
         if (warp == 0) {
             tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, false, false);
-            const uint64_t a0 = make_desc(sb + P_LK, 16, 1024);
-            const uint64_t b0 = make_desc(sb + hs + H_TP, 16, 1024);
+            const uint32_t id = idesc_bf16(128, 64, false, true);
+            const uint64_t aY = make_desc(sb + P_RH, 16, 1024);
+            const uint64_t aW = make_desc(sb + P_PO, 16, 1024);
+            const uint64_t bT = make_desc(sb + P_TP, 8192, 1024);
+            if (elect_one()) {
 #pragma unroll
-            for (int s = 0; s < 4; ++s) warp_mma(tm + TP_Z, desc_add(a0, s * 32), desc_add(b0, s * 32), id, s > 0);
-            warp_commit(bar_mma);
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tm + TP_Y, desc_add(aY, s * 32), desc_add(bT, s * 2048), id, s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tm + TP_W, desc_add(aW, s * 32), desc_add(bT, s * 2048), id, s > 0);
+                mma_commit(bar_mma);
+            }
+            __syncwarp();
         }
-        if (!wait_mma()) { aborted = true; break; }
-        trace_mark(prank, n, 5);
+        if (tid == 0) bulk_wait_read0();        // the staging is free once the ring store read it
+        if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
+        trace_mark(prank, n, 13);
+        if (has_next) issue_g(c_next);          // R and Rh are dead
+        trace_mark(prank, n, 7);
         tc_fence_after();
-
-        // ---- Z -> bf16 into the hand-off set (local), then hand the chunk over ----
+        if (qt == 0) {
+            float* fs = reinterpret_cast<float*>(sm + P_ST + S_FAC);
+            fs[c] = fac_r;
+            fs[128 + c] = fac_c;
+        }
         {
-            float val[32];
-            tmem_ld32(tm + lane_sel + TP_Z + 32 * wg, val);
+            float val[16];
+            tmem_ld16(tm + lane_sel + TP_Y + 16 * wg, val);
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
-                st16(sm, hs + H_ZO + mnmaj_chunk(row, 4 * wg + qq, 0, 16), pack8(val + 8 * qq));
+            for (int qq = 0; qq < 2; ++qq)
+                st16(sm, P_ST + S_YW + kmaj_chunk(row, 2 * wg + qq, 0, 0), pack8(val + 8 * qq));
+            if ((warp & 3) < 2) {               // lanes 0..63 hold Wh^T
+                tmem_ld16(tm + lane_sel + TP_W + 16 * wg, val);
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq)
+                    st16(sm, P_ST + S_YW + kmaj_chunk(128 + row, 2 * wg + qq, 0, 0), pack8(val + 8 * qq));
+            }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        trace_mark(prank, n, 12);
-        if (n >= 2) {                           // ring slot n % 2 must have been released
-            const bool ok = mbar_wait_cluster_bounded(bar_free, ph_free, kWaitCycles);
-            ph_free ^= 1u;
-            if (!ok) atomicOr(p.err, kErrTimeout);
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
-        trace_mark(prank, n, 6);
+        trace_mark(prank, n, 8);
+
+        // ---- [Gm | Qh] = -Lk^T [Yh | Wh] + Lq^T [0 | I] (M = key ch, N = 192) ----
         if (warp == 0) {
-            // one arrival announcing the bytes, then the bulk copies into the consumer's slot
-            // (one per lane); together they complete that slot's "full" barrier
-            const int lane = tid & 31;
-            const uint32_t dst = c_slot0 + (uint32_t)slot * kSlotBytes;
-            const SlotMap mp = slot_map(slot);
-            const uint32_t full = c_misc + (slot ? M_BAR_B : M_BAR_A);
-            // relaxed: the bytes travel in the bulk copies, which complete the barrier themselves
-            if (lane == 0) mbar_arrive_expect_tx_remote_relaxed(full, kHandoffTx);
+            tc_fence_after();
+            const uint32_t id192 = idesc_bf16(128, 192, false, false, true);
+            const uint32_t id64 = idesc_bf16(128, 64, false, false);
+            const uint64_t aK = make_desc(sb + P_LK, 16, 1024);
+            const uint64_t aQ = make_desc(sb + P_LQ, 16, 1024);
+            const uint64_t bY = make_desc(sb + P_ST + S_YW, 16, 1024);
+            const uint64_t bI = make_desc(sb + P_ID, 16, 1024);
+            if (elect_one()) {
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tm + TP_GQ, desc_add(aK, s * 32), desc_add(bY, s * 32), id192, s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tm + TP_GQ + 128, desc_add(aQ, s * 32), desc_add(bI, s * 32), id64, 1);
+                mma_commit(bar_mma);
+            }
             __syncwarp();
-            if (lane == 0) bulk_copy_to_peer(dst + mp.lq, sb + hs + H_LQ, 16384, full);
-            if (lane == 1) bulk_copy_to_peer(dst + mp.zo, sb + hs + H_ZO, 16384, full);
-            if (lane == 2) bulk_copy_to_peer(dst + mp.rt, sb + hs + H_RT, 16384, full);
-            if (lane == 3) bulk_copy_to_peer(dst + S_TP, sb + hs + H_TP, 8192, full);
-            if (lane == 4) bulk_copy_to_peer(dst + mp.po, sb + hs + H_PO, 8192, full);
-            if (lane == 5) bulk_copy_to_peer(c_fac + (uint32_t)(n % 3) * kFacBytes, sb + hs + H_FAC, kFacBytes, full);
         }
-        trace_mark(prank, n, 7);
+        if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
+        trace_mark(prank, n, 9);
+        tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 3; ++part) {
+            float val[16];
+            const int col0 = 48 * wg + 16 * part;
+            tmem_ld16(tm + lane_sel + TP_GQ + col0, val);
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const int nc = col0 + 8 * qq;
+                st16(sm, P_ST + S_GQ + mnmaj_chunk(row, (nc & 63) >> 3, nc >> 6, 16), pack8(val + 8 * qq));
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        trace_mark(prank, n, 10);
+
+        // ---- hand-off: bulk stores into ring slot n % kRing (once chunk n - kRing was read) ----
+        if (n >= kRing) {
+            const int rs = n % kRing;
+            const bool ok = block_wait(bar_gfree + rs, (ph_gfree >> rs) & 1u, true, p.err);
+            ph_gfree ^= 1u << rs;
+            if (!ok) { aborted = true; break; }
+        }
+        trace_mark(prank, n, 11);
+        announce();                             // the previous chunk, stored a task ago
+        if (tid == 0) {
+            bulk_store(ring + (size_t)(n % kRing) * kSlotBytes, sb + P_ST, kSlotBytes);
+            bulk_commit();
+        }
+        pending = n;
+        trace_mark(prank, n, 12);
     }
+    if (!aborted) announce();
+    if (tid == 0) bulk_wait0();
 }
 
 // ============================== consumer ==============================
@@ -512,234 +630,231 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
     const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, j = tid & 127;
     const uint32_t lane_sel = (uint32_t)(32 * (warp & 3)) << 16;
     uint8_t* misc = sm + C_MISC;
-    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(misc + M_BAR_MMA);
-    uint64_t* bar_full0 = reinterpret_cast<uint64_t*>(misc + M_BAR_A);
-    uint64_t* bar_full1 = reinterpret_cast<uint64_t*>(misc + M_BAR_B);
+    uint64_t* bar_s = reinterpret_cast<uint64_t*>(misc + M_BAR_S);
+    uint64_t* bar_o = reinterpret_cast<uint64_t*>(misc + M_BAR_O);
+    uint64_t* bar_lfull = reinterpret_cast<uint64_t*>(misc + M_LFULL);
+    uint64_t* bar_gfull = reinterpret_cast<uint64_t*>(misc + M_GFULL);
+    uint64_t* bar_v = reinterpret_cast<uint64_t*>(misc + M_BAR_V);
     const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
     const int H = p.H;
     const int nchunks = (int)((eos - bos + kC - 1) / kC);
-    uint32_t ph_mma = 0, ph_full0 = 0, ph_full1 = 0;   // scalars: no run-time indexed arrays
+    uint32_t ph_s = 0, ph_o = 0, ph_lfull = 0, ph_gfull = 0, ph_v = 0;   // bit i: parity of barrier i
+    const uint8_t* ring = p.ring + (size_t)smid() * (kRing * kSlotBytes);
     const int64_t sbase = ((int64_t)n_seq * H + h) * kD * kD;
 
-    float sreg[64];                     // S[64*wg + cc][j]
+    float sreg[32];                     // S[32*wg + cc][j]
 #pragma unroll
-    for (int cc = 0; cc < 64; ++cc)
-        sreg[cc] = p.h0 ? p.h0[sbase + (int64_t)(64 * wg + cc) * kD + j] : 0.f;
+    for (int cc = 0; cc < 32; ++cc)
+        sreg[cc] = p.h0 ? p.h0[sbase + (int64_t)(32 * wg + cc) * kD + j] : 0.f;
 
-    // V tile of chunk nn into its slot by TMA: two (64 channels x 64 tokens) boxes whose
-    // 128B-swizzled image is exactly the MN-major operand layout. Rows past the sequence do
-    // not matter (the matching columns of T' are zero).
-    uint64_t* bar_v0 = reinterpret_cast<uint64_t*>(misc + M_BAR_C);
-    uint64_t* bar_v1 = reinterpret_cast<uint64_t*>(misc + M_BAR_D);
-    uint32_t ph_v0 = 0, ph_v1 = 0;
+    auto wait_bar = [&](uint64_t* bar, uint32_t& ph) -> bool {
+        const bool ok = block_wait(bar, ph & 1u, false, p.err);
+        ph ^= 1u;
+        return ok;
+    };
+    // V tile of chunk nn into ring entry nn % 3 by TMA: two (64 channels x 64 tokens) boxes whose
+    // 128B-swizzled image is exactly the MN-major operand layout. Rows past the sequence do not
+    // matter (the matching rows of Yh and Wh are zero).
+    // Thread kLoader (warp 2) issues every V and ring load, so that it runs beside warp 0's MMA
+    // issue instead of in front of it.
+    constexpr int kLoader = 64;
     auto issue_v = [&](int nn) {
-        if (tid == 0) {
-            uint64_t* bv = (nn & 1) ? bar_v1 : bar_v0;
-            const uint32_t base = sb + C_SLOT0 + (nn & 1) * kSlotBytes + S_VT;
+        if (tid == kLoader) {
+            const int e = nn % 3;
+            const uint32_t base = sb + C_V + (uint32_t)e * 16384;
             const int c0 = (int)(bos + (int64_t)nn * kC);
-            mbar_arrive_expect_tx(bv, 16384u);
-            tma_load_3d(base, &p.tv, 0, h, c0, bv);
-            tma_load_3d(base + 8192, &p.tv, 64, h, c0, bv);
+            mbar_arrive_expect_tx(bar_v + e, 16384u);
+            tma_load_3d(base, &p.tv, 0, h, c0, bar_v + e);
+            tma_load_3d(base + 8192, &p.tv, 64, h, c0, bar_v + e);
         }
     };
     auto wait_v = [&](int nn) -> bool {
-        const int sl = nn & 1;
-        const bool ok = mbar_wait_bounded(sl ? bar_v1 : bar_v0, sl ? ph_v1 : ph_v0, kWaitCycles);
-        if (sl) ph_v1 ^= 1u; else ph_v0 ^= 1u;
-        if (!ok) atomicOr(p.err, kErrTimeout);
-        return __syncthreads_or(!ok) == 0;
+        const int e = nn % 3;
+        const bool ok = block_wait(bar_v + e, (ph_v >> e) & 1u, false, p.err);
+        ph_v ^= 1u << e;
+        return ok;
     };
-    // Output epilogue: O of chunk nn goes from TMEM to a row-major [token][channel] bf16
-    // staging tile (the Ut^T buffer, free once the chunk's last MMAs completed), then to HBM
-    // as one TMA tile store (a ragged last chunk: one bulk copy per valid token, so rows of the
-    // next sequence are never touched), overlapping the next chunk.
-    float oval[32];
-    auto load_o = [&](int nn) { tmem_ld32(tm + lane_sel + ((nn & 1) ? TC_O1 : TC_O0) + 32 * wg, oval); };
-    auto stage_o = [&]() {
-        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + C_UT);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) st[(32 * wg + t) * kD + j] = __float2bfloat16_rn(p.scale * oval[t]);
-    };
-    auto store_o = [&](int nn) {               // warp 1, after the staging writes are fenced
-        const int64_t c0 = bos + (int64_t)nn * kC;
-        const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
-        const int lane = tid & 31;
-        if (L == kC) {
-            if (lane == 0) tma_store_3d(&p.to, 0, h, (int)c0, sb + C_UT);
-        } else {
-            for (int r = lane; r < L; r += 32)
-                bulk_store(p.o + ((c0 + r) * H + h) * kD, sb + C_UT + r * 256, 256);
+    // Operands of chunk nn from its global ring slot into shared slot nn % 2 (thread 0; the
+    // shared slot must be free): waits for the producer's announcement, then bulk loads.
+    auto issue_load = [&](int nn) -> bool {
+        bool ok = true;
+        if (tid == kLoader) {
+            const int rs = nn % kRing;
+            ok = mbar_wait_cluster_bounded(bar_gfull + rs, (ph_gfull >> rs) & 1u, kWaitCycles);
+            ph_gfull ^= 1u << rs;
+            if (ok) {
+                fence_proxy_async_global();
+                uint64_t* bl = bar_lfull + (nn & 1);
+                const uint32_t dst = sb + C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
+                const uint8_t* src = ring + (size_t)rs * kSlotBytes;
+                mbar_arrive_expect_tx(bl, kSlotBytes);
+                bulk_load(dst, src, kSlotBytes, bl);                                 // one copy
+            } else {
+                atomicOr(p.err, kErrTimeout);
+            }
         }
-        bulk_commit();
+        return ok;
     };
-    auto wait_mma = [&]() -> bool {
-        const bool ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitCycles);
-        ph_mma ^= 1u;
-        if (!ok) atomicOr(p.err, kErrTimeout);
-        return __syncthreads_or(!ok) == 0;
-    };
+    // Shared slot nn % 2 holds chunk nn; its ring slot may take chunk nn + kRing.
     auto wait_full = [&](int nn) -> bool {
         const int sl = nn & 1;
-        const bool ok = mbar_wait_cluster_bounded(sl ? bar_full1 : bar_full0,
-                                                  sl ? ph_full1 : ph_full0, kWaitCycles);
-        if (sl) ph_full1 ^= 1u; else ph_full0 ^= 1u;
-        if (!ok) atomicOr(p.err, kErrTimeout);
-        return __syncthreads_or(!ok) == 0;
+        const bool ok = block_wait(bar_lfull + sl, (ph_lfull >> sl) & 1u, false, p.err);
+        ph_lfull ^= 1u << sl;
+        if (!ok) return false;
+        if (tid == 0 && nn + kRing < nchunks)
+            mbar_arrive_remote_relaxed(map_to_rank(sb + P_MISC + M_GFREE + 8u * (uint32_t)(nn % kRing),
+                                                   1 + (nn + kRing) % kProducers));
+        return true;
     };
-    // -U^T = -(V^T T'^T) of chunk nn into its X accumulator (one converged warp).
-    auto issue_u = [&](int nn) {
-        const uint32_t so = C_SLOT0 + (nn & 1) * kSlotBytes;
+    // D(nn) = V^T [Yh | Wh] (one converged warp)
+    auto issue_e = [&](int nn) {
+        const uint32_t so = C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
         tc_fence_after();
-        const uint32_t id_u = idesc_bf16(128, 64, true, false, true);
-        const uint64_t a0 = make_desc(sb + so + S_VT, 8192, 1024);
-        const uint64_t b0 = make_desc(sb + so + S_TP, 16, 1024);
+        const uint32_t id = idesc_bf16(128, 192, true, false);
+        const uint64_t a0 = make_desc(sb + C_V + (uint32_t)(nn % 3) * 16384, 8192, 1024);
+        const uint64_t b0 = make_desc(sb + so + S_YW, 16, 1024);
+        const uint32_t d = tm + ((nn & 1) ? TD1 : TD0);
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            warp_mma(tm + ((nn & 1) ? TC_X1 : TC_X0), desc_add(a0, s * 2048), desc_add(b0, s * 32), id_u, s > 0);
+            for (int s = 0; s < 4; ++s) mma_bf16(d, desc_add(a0, s * 2048), desc_add(b0, s * 32), id, s > 0);
+        }
+        __syncwarp();
     };
-    // Sm(nn) = (diag(e^{gamma_ref(nn)}) S)^T as the bf16 A operand (S already updated).
-    auto write_sm = [&](int nn) {
-        const float* fac = reinterpret_cast<const float*>(sm + C_FAC + (nn % 3) * kFacBytes);
-        const float4* fac4 = reinterpret_cast<const float4*>(fac + 64 * wg);
+    // D(nn) += Sm [Gm | Qh]: the state part first (commit S), then the output part (commit O)
+    auto issue_c = [&](int nn) {
+        const uint32_t so = C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
+        tc_fence_after();
+        const uint32_t idS = idesc_bf16(128, 128, false, true);
+        const uint32_t idO = idesc_bf16(128, 64, false, true);
+        const uint64_t bG = make_desc(sb + so + S_GQ, 16384, 1024);
+        const uint64_t bQ = make_desc(sb + so + S_GQ + 32768, 16384, 1024);
+        const uint32_t d = tm + ((nn & 1) ? TD1 : TD0);
+        if (elect_one()) {
 #pragma unroll
-        for (int qq = 0; qq < 8; ++qq) {
-            const float4 e0 = fac4[2 * qq], e1 = fac4[2 * qq + 1];
-            const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-            float w8[8];
+            for (int s = 0; s < 8; ++s) mma_bf16_ts(d, tm + TC_SM + 8 * s, desc_add(bG, s * 2048), idS, 1);
+            mma_commit(bar_s);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) w8[u] = sreg[8 * qq + u] * ev[u];
-            st16(sm, C_ST + kmaj_chunk(j, qq, wg, 128), pack8(w8));
+            for (int s = 0; s < 8; ++s) mma_bf16_ts(d + 128, tm + TC_SM + 8 * s, desc_add(bQ, s * 2048), idO, 1);
+            mma_commit(bar_o);
+        }
+        __syncwarp();
+    };
+    // Sm(nn) = (S^T diag(e^{gamma_ref(nn)})) as bf16 pairs along the key channel
+    auto pack_sm = [&](int nn, uint32_t* w) {
+        const float* fac = reinterpret_cast<const float*>(sm + C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes + S_FAC);
+        const float4* e4 = reinterpret_cast<const float4*>(fac + 32 * wg);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 e = e4[q4];
+            w[2 * q4] = pack_bf16(sreg[4 * q4] * e.x, sreg[4 * q4 + 1] * e.y);
+            w[2 * q4 + 1] = pack_bf16(sreg[4 * q4 + 2] * e.z, sreg[4 * q4 + 3] * e.w);
+        }
+    };
+    // O of chunk nn: TMEM -> bf16 [token][channel] staging -> one TMA tile store (a ragged last
+    // chunk: one bulk copy per valid token, so rows of the next sequence are never touched)
+    auto epilogue_o = [&](int nn) {
+        tc_fence_after();
+        float ov[16];
+        tmem_ld16(tm + lane_sel + ((nn & 1) ? TD1 : TD0) + 128 + 16 * wg, ov);
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) st[(16 * wg + t) * kD + j] = __float2bfloat16_rn(p.scale * ov[t]);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 1) {
+            const int64_t c0 = bos + (int64_t)nn * kC;
+            const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
+            const int lane = tid & 31;
+            if (L == kC) {
+                if (lane == 0) tma_store_3d(&p.to, 0, h, (int)c0, sb + C_OST);
+            } else {
+                for (int r = lane; r < L; r += 32)
+                    bulk_store(p.o + ((c0 + r) * H + h) * kD, sb + C_OST + r * 256, 256);
+            }
+            bulk_commit();
         }
     };
 
-    // prologue: operands of chunk 0 (and the V tile of chunk 1)
+    // prologue: V tiles of chunks 0..2, Sm(0), then chunk 0's products
     if (nchunks > 0) {
         issue_v(0);
         if (nchunks > 1) issue_v(1);
-        if (!wait_v(0)) aborted = true;
-        if (!aborted && !wait_full(0)) aborted = true;
+        if (nchunks > 2) issue_v(2);
+        // chunk 0 must have arrived (which frees ring slot 0 for chunk 4) before the loader
+        // waits for chunk 1: a producer announces a chunk only when it hands off its next one
+        if (__syncthreads_or(!issue_load(0))) aborted = true;   // (seen by every thread)
+        if (!aborted && (!wait_full(0) || !wait_v(0))) aborted = true;
+        if (!aborted && nchunks > 1 && __syncthreads_or(!issue_load(1))) aborted = true;
         if (!aborted) {
-            write_sm(0);
-            fence_async_smem();
+            uint32_t w[16];
+            pack_sm(0, w);
+            tmem_st16(tm + lane_sel + TC_SM + 16 * wg, w);
+            tmem_wait_st();
             tc_fence_before();
             __syncthreads();
-            if (warp == 0) issue_u(0);
+            if (warp == 0) { issue_e(0); issue_c(0); }
         }
     }
 
     for (int n = 0; n < nchunks && !aborted; ++n) {
-        const int slot = n & 1;
-        const uint32_t so = C_SLOT0 + slot * kSlotBytes;
-        const SlotMap mp = slot_map(slot);
-        const float* fac = reinterpret_cast<const float*>(sm + C_FAC + (n % 3) * kFacBytes);
-        const uint32_t tX = slot ? TC_X1 : TC_X0;
+        const float* fac = reinterpret_cast<const float*>(sm + C_SLOT0 + (uint32_t)(n & 1) * kSlotBytes + S_FAC);
         trace_mark(0, n, 0);
-
-        // ---- [X | O] (+)= Sm [Z | Lq]: X = -Ut^T, O = Sm Lq^T ----
-        if (warp == 0) {
-            tc_fence_after();
-            const uint32_t id64 = idesc_bf16(128, 64, false, true);
-            const uint32_t id128 = idesc_bf16(128, 128, false, true);
-            const uint64_t aS = make_desc(sb + C_ST, 16, 1024);
-            const uint64_t bZ = make_desc(sb + so + mp.zo, 16384, 1024);
-            const uint64_t bQ = make_desc(sb + so + mp.lq, 16384, 1024);
-            // first K step: X accumulates onto -U^T, O starts from zero
-            warp_mma(tm + tX, aS, bZ, id64, 1);
-            warp_mma(tm + (slot ? TC_O1 : TC_O0), aS, bQ, id64, 0);
-            const uint64_t bW = slot ? bQ : bZ;           // the lower of the two adjacent B blocks
-            const uint32_t dW = slot ? TC_O1 : TC_X0;
-#pragma unroll
-            for (int s = 1; s < 8; ++s)
-                warp_mma(tm + dW, desc_add(aS, (s >> 2) * 16384 + (s & 3) * 32), desc_add(bW, s * 2048), id128, 1);
-            warp_commit(bar_mma);
-        }
+        // (1) output of the previous chunk, while this chunk's chain runs
+        if (n > 0) epilogue_o(n - 1);
         trace_mark(0, n, 1);
-        // the staging tile of O(n - 1) is rewritten below: its TMA store must have read it
-        if (warp == 1) bulk_wait_read0();
-        trace_mark(0, n, 2);
-        if (!wait_mma()) { aborted = true; break; }
-        trace_mark(0, n, 10);
-        tc_fence_after();
-        {
-            float val[32];
-            tmem_ld32(tm + lane_sel + tX + 32 * wg, val);
-#pragma unroll
-            for (int t = 0; t < 32; ++t) val[t] = -val[t];
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) st16(sm, C_UT + kmaj_chunk(j, 4 * wg + qq, 0, 128), pack8(val + 8 * qq));
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        trace_mark(0, n, 3);
-
-        // ---- [O | dS^T] (+)= Ut^T [P | R] ----
-        if (warp == 0) {
-            tc_fence_after();
-            const uint32_t id64 = idesc_bf16(128, 64, false, false);
-            const uint32_t id128 = idesc_bf16(128, 128, false, false);
-            const uint32_t id192 = idesc_bf16(128, 192, false, false);
-            const uint64_t aU = make_desc(sb + C_UT, 16, 1024);
-            const uint64_t bP = make_desc(sb + so + mp.po, 16, 1024);
-            const uint64_t bR = make_desc(sb + so + mp.rt, 16, 1024);
-            warp_mma(tm + (slot ? TC_O1 : TC_O0), aU, bP, id64, 1);
-            warp_mma(tm + TC_S, aU, bR, id128, 0);
-            const uint64_t bW = slot ? bR : bP;
-            const uint32_t dW = slot ? TC_S : TC_O0;
-#pragma unroll
-            for (int s = 1; s < 4; ++s) warp_mma(tm + dW, desc_add(aU, s * 32), desc_add(bW, s * 32), id192, 1);
-            warp_commit(bar_mma);
-        }
-        // the V tile of this slot was consumed by -U^T (complete): fetch the one of chunk n + 2
-        if (n + 2 < nchunks) issue_v(n + 2);
-        trace_mark(0, n, 4);
-        if (!wait_mma()) { aborted = true; break; }
-        // every MMA that reads ring slot n % 2 has completed (the chunk's factors live in the
-        // factor ring): tell the producer of chunk n + 2 it may write the slot
-        if (tid == 0 && n + 2 < nchunks)
-            mbar_arrive_remote_relaxed(map_to_rank(sb + P_MISC + M_BAR_A, 1 + (n + 2) % kProducers));
-        trace_mark(0, n, 5);
+        // (2) operands of the next chunk and its V^T products (queued behind this chunk's chain)
         const bool more = n + 1 < nchunks;
         if (more) {
-            // operands of chunk n + 1 (its V tile was requested one chunk earlier)
-            if (!wait_v(n + 1)) { aborted = true; break; }
-            if (!wait_full(n + 1)) { aborted = true; break; }
+            if (!wait_full(n + 1) || !wait_v(n + 1)) { aborted = true; break; }
+            if (warp == 0) issue_e(n + 1);
         }
-        trace_mark(0, n, 6);
+        trace_mark(0, n, 2);
+        // (3) state update S' = e^{gamma_C} S + D_S
+        if (!wait_bar(bar_s, ph_s)) { aborted = true; break; }
+        trace_mark(0, n, 3);
         tc_fence_after();
         {
-            float val[32];
-            const float4* eC4 = reinterpret_cast<const float4*>(fac + 128 + 64 * wg);
-            const float4* eR4 = reinterpret_cast<const float4*>(fac + 256 + 64 * wg);
+            float v32[32];
+            tmem_ld32(tm + lane_sel + ((n & 1) ? TD1 : TD0) + 32 * wg, v32);
+            const float4* eC4 = reinterpret_cast<const float4*>(fac + 128 + 32 * wg);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32(tm + lane_sel + TC_S + 64 * wg + 32 * half, val);
-#pragma unroll
-                for (int t4 = 0; t4 < 8; ++t4) {
-                    const float4 ec = eC4[8 * half + t4], er = eR4[8 * half + t4];
-                    const float ecv[4] = {ec.x, ec.y, ec.z, ec.w}, erv[4] = {er.x, er.y, er.z, er.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int cc = 32 * half + 4 * t4 + u;
-                        sreg[cc] = fmaf(ecv[u], sreg[cc], erv[u] * val[4 * t4 + u]);
-                    }
-                }
+            for (int t4 = 0; t4 < 8; ++t4) {
+                const float4 ec = eC4[t4];
+                const float* v = v32 + 4 * t4;
+                const int cc = 4 * t4;
+                sreg[cc] = fmaf(ec.x, sreg[cc], v[0]);
+                sreg[cc + 1] = fmaf(ec.y, sreg[cc + 1], v[1]);
+                sreg[cc + 2] = fmaf(ec.z, sreg[cc + 2], v[2]);
+                sreg[cc + 3] = fmaf(ec.w, sreg[cc + 3], v[3]);
             }
         }
-        load_o(n);
-        stage_o();
-        if (more) write_sm(n + 1);
-        fence_async_smem();
+        uint32_t w[16];
+        if (more) pack_sm(n + 1, w);
+        if (warp == 1) bulk_wait_read0();       // the staged O tile has been read
+        trace_mark(0, n, 4);
+        if (!wait_bar(bar_o, ph_o)) { aborted = true; break; }
+        trace_mark(0, n, 5);
+        if (more) {
+            tmem_st16(tm + lane_sel + TC_SM + 16 * wg, w);
+            tmem_wait_st();
+        }
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(aborted)) { aborted = true; break; }
+        trace_mark(0, n, 6);
+        // (4) chain of the next chunk; beside it, the loads that the completed chunk n made
+        // possible: shared slot n % 2 takes chunk n + 2, V ring entry n % 3 takes V(n + 3)
+        if (more && warp == 0) issue_c(n + 1);
+        if (n + 2 < nchunks) issue_load(n + 2);   // a failed wait flags the error word; the
+                                                  // consumer then gives up at wait_full(n + 2)
+        if (n + 3 < nchunks) issue_v(n + 3);
         trace_mark(0, n, 7);
-        if (more && warp == 0) issue_u(n + 1);
-        if (warp == 1) store_o(n);
     }
+    if (nchunks > 0 && !aborted) epilogue_o(nchunks - 1);
     if (warp == 1) bulk_wait0();
     if (p.ht && !aborted) {
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) p.ht[sbase + (int64_t)(64 * wg + cc) * kD + j] = sreg[cc];
+        for (int cc = 0; cc < 32; ++cc) p.ht[sbase + (int64_t)(32 * wg + cc) * kD + j] = sreg[cc];
     }
 }
 
@@ -762,19 +877,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
         tmem_relinquish();
     }
     if (threadIdx.x == 0) {
-        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_MMA), 1);
-        // consumer "full" barriers: one producer arrival + the bulk bytes; producer "free"
-        // barrier: one consumer arrival
-        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_A), 1);
-        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_B), 1);
-        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_C), 1);
-        mbar_init(reinterpret_cast<uint64_t*>(misc + M_BAR_D), 1);
+        // every barrier completes once per use: one arrival (plus transaction bytes where a TMA
+        // or bulk copy feeds it)
+        for (uint32_t b = 0; b < kBars; ++b) mbar_init(reinterpret_cast<uint64_t*>(misc + 8 * b), 1);
+        if (is_consumer) {
+            const uint32_t id = smid();
+            *reinterpret_cast<uint32_t*>(misc + M_SMID) = id;
+            if ((int)id >= p.ring_sms) atomicOr(p.err, kErrTimeout);
+        }
     }
     tc_fence_before();
     cluster_sync();                     // barriers of every CTA exist before any remote arrive
     tc_fence_after();
 
-    bool aborted = false;
+    // a consumer SM outside the workspace's ring table (flagged above): nobody touches the ring
+    bool aborted = (int)ld_cluster_u32(map_to_rank(sb + C_MISC + M_SMID, 0)) >= p.ring_sms;
     if (is_consumer) consumer(p, sm, sb, n_seq, h, bos, eos, aborted);
     else producer(p, sm, sb, (int)crank, h, bos, eos, aborted);
 
@@ -789,7 +906,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
 
 }  // namespace
 
-cudaError_t launch_chunk_tcx(const ChunkArgs& a, unsigned int* err, cudaStream_t stream) {
+// Ring tables for SM ids 0 .. kRingSms - 1 (a B200 has 148 SMs).
+constexpr int kRingSms = 160;
+size_t chunk_tcx_workspace_bytes() { return (size_t)kRingSms * kRing * kSlotBytes; }
+
+cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspace_bytes,
+                             unsigned int* err, cudaStream_t stream) {
     const int64_t units = (int64_t)a.N * a.H;
     if (units == 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(chunk_tcx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -803,10 +925,6 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, unsigned int* err, cudaStream_t
         make_tmap_thd(&p.tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, 64, kC, true) &&
         make_tmap_thd(&p.to, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false);
     if (!maps_ok) return cudaErrorInvalidValue;
-    p.q = static_cast<const __nv_bfloat16*>(a.q);
-    p.k = static_cast<const __nv_bfloat16*>(a.k);
-    p.v = static_cast<const __nv_bfloat16*>(a.v);
-    p.g = a.g;
     p.beta = a.beta;
     p.scale = a.scale;
     p.h0 = a.h0;
@@ -817,6 +935,8 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, unsigned int* err, cudaStream_t
     p.N = a.N;
     p.H = a.H;
     p.err = err;
+    p.ring = static_cast<uint8_t*>(workspace);
+    p.ring_sms = (int)(workspace_bytes / ((size_t)kRing * kSlotBytes));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units * kCluster), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

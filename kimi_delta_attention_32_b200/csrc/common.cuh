@@ -104,8 +104,12 @@ __device__ __forceinline__ void trace_mark(int cta, int chunk, int mark, int who
         g_trace[cta][chunk][mark] = t;
     }
 }
+__device__ __forceinline__ void trace_value(int cta, int chunk, int slot, unsigned long long v) {
+    if (threadIdx.x == 0 && blockIdx.x < 4 && chunk < 512) g_trace[cta][chunk][slot] = v;
+}
 #else
 __device__ __forceinline__ void trace_mark(int, int, int, int = 0) {}
+__device__ __forceinline__ void trace_value(int, int, int, unsigned long long) {}
 #endif
 
 }  // namespace kda

@@ -53,7 +53,10 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 // Tensor-core (tcgen05) prefill: bf16 I/O, dk = dv = 128, chunk 64.
 bool chunk_tc_supported(const ChunkArgs& a);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, unsigned int* err, cudaStream_t stream);
-// Same math as a producer/consumer pipeline in one 4-CTA cluster per (sequence, head).
-cudaError_t launch_chunk_tcx(const ChunkArgs& a, unsigned int* err, cudaStream_t stream);
+// Same math as a producer/consumer pipeline in one 4-CTA cluster per (sequence, head). Needs a
+// device workspace of chunk_tcx_workspace_bytes() (16-byte aligned): the per-SM hand-off rings.
+size_t chunk_tcx_workspace_bytes();
+cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspace_bytes,
+                             unsigned int* err, cudaStream_t stream);
 
 }  // namespace kda

@@ -134,8 +134,26 @@ def test_recurrent_step_rejects(lib, kw, status):
 
 def test_workspace_query(lib):
     out = ctypes.c_size_t(123)
+    # bf16, dk = dv = 128, chunk 64: the tensor-core pipeline's fixed hand-off rings
     assert lib.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 128, 64, 1, ctypes.byref(out)) == 0
+    ring = out.value
+    assert ring > 0 and ring % 16 == 0
+    assert lib.kda_chunk_fwd_workspace_size(64, 527241, 32, 128, 128, 64, 1, ctypes.byref(out)) == 0
+    assert out.value == ring                              # independent of the batch
+    for dk, io in ((128, 0), (64, 1), (64, 0)):           # fp32 I/O and d = 64 need none
+        assert lib.kda_chunk_fwd_workspace_size(1, 8192, 32, dk, dk, 64, io, ctypes.byref(out)) == 0
+        assert out.value == 0
     assert lib.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 128, 0, 1, ctypes.byref(out)) == \
         kda.KDA_ERR_INVALID_ARG
     assert lib.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 128, 64, 1, None) == \
         kda.KDA_ERR_INVALID_ARG
+
+
+def test_chunk_fwd_checks_workspace(lib, monkeypatch):
+    monkeypatch.delenv("KDA_CHUNK_KERNEL", raising=False)
+    out = ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_workspace_size(1, 64, 2, 128, 128, 64, 1, ctypes.byref(out)) == 0
+    need = out.value
+    assert _chunk(lib) == kda.KDA_ERR_WORKSPACE                          # missing
+    assert _chunk(lib, ws=MIS, wsb=need) == kda.KDA_ERR_WORKSPACE         # misaligned
+    assert _chunk(lib, ws=FAKE, wsb=need - 16) == kda.KDA_ERR_WORKSPACE   # too small
