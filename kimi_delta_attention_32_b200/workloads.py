@@ -134,8 +134,10 @@ def make_prefill(wl: Workload, device="cpu", T: int | None = None, lengths=None)
     """
     gen = _gen(device, wl.seed)
     dt = io_dtype(wl.io)
-    if wl.varlen:
-        lengths = list(lengths) if lengths is not None else varlen_lengths(wl)
+    if lengths is not None:
+        lengths = list(lengths)
+    elif wl.varlen:
+        lengths = varlen_lengths(wl)
     else:
         lengths = [T if T is not None else wl.T] * wl.N
     cu = cu_seqlens_of(lengths)
