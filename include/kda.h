@@ -145,6 +145,18 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          void* stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd without a caller workspace: the library uses a
+ * device array of its own (reserved when libkda is loaded, one per device), so the call
+ * allocates nothing. Arguments, layouts, results and errors are those of kda_chunk_fwd.
+ * Calls on one device must not run concurrently with each other (they share that array).
+ */
+kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, float scale, const float* h0, float* ht,
+                                 void* o, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                                 int B, int T, int N, int H, int dk, int dv, int chunk,
+                                 kda_io_dtype io, void* stream);
+
+/*
  * kda_recurrent_step -- one decode token per (sequence, head), state updated in place.
  * (sarnas.ru, section "Что именно изменилось"; m.lqnn.cn/news/205170, section
  *  "KDA 与 Gated Attention ...": the per-token loop state = state*exp(gate)+delta.)

@@ -21,7 +21,7 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUD
 KDA_IO_F32, KDA_IO_BF16 = 0, 1
 
 EXPORTED = ("kda_status_string", "kda_version", "kda_conv_fwd", "kda_chunk_fwd_workspace_size",
-            "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error")
+            "kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_recurrent_step", "kda_last_device_error")
 
 _lock = threading.Lock()
 _lib = None
@@ -60,6 +60,10 @@ def load_library(path: str = LIB_PATH):
                                       ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci, ci,
                                       ci, vp, cs, vp]
         lib.kda_chunk_fwd.restype = ci
+        lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, cf, fp, fp, vp, i32p,
+                                              ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci,
+                                              ci, ci, vp]
+        lib.kda_chunk_fwd_noalloc.restype = ci
         lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, cf, fp, vp, ci, ci, ci, ci, ci, vp]
         lib.kda_recurrent_step.restype = ci
         lib.kda_last_device_error.argtypes = [vp]
@@ -161,6 +165,31 @@ def chunk_fwd(q, k, v, g, beta, scale=1.0, h0=None, ht=None, o=None, cu_seqlens=
                            _stream(stream))
     del keep
     _check("kda_chunk_fwd", st)
+    return o, ht
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, scale=1.0, h0=None, ht=None, o=None, cu_seqlens=None,
+                      cu_host=None, chunk=64, stream=None):
+    """chunk_fwd through kda_chunk_fwd_noalloc: no workspace is allocated for the call (o and
+    ht are, unless given). Returns (o, ht)."""
+    lib = load_library()
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape if q.dim() == 4 else (1, *q.shape)
+        N = B
+    else:
+        B, T = 1, 0
+        _, H, dk = q.shape
+        N = len(cu_host) - 1
+    dv = v.shape[-1]
+    o = torch.empty_like(v) if o is None else o
+    if ht is None:
+        ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    keep, cuh = _host_cu(cu_host)
+    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                   _ptr(h0), _ptr(ht), _ptr(o), _ptr(cu_seqlens), cuh, B, T, N, H,
+                                   dk, dv, chunk, _io(q), _stream(stream))
+    del keep
+    _check("kda_chunk_fwd_noalloc", st)
     return o, ht
 
 
