@@ -25,7 +25,7 @@
 // state in registers and writes the next Sm back to tensor memory; O leaves through a TMA
 // store. Ranks 1..3 are producers, each preparing every third chunk. A chunk's operands travel
 // through L2, not DSMEM (bulk copies between SMs of a cluster move ~30-60 GB/s, TMA loads from
-// L2 150-220 GB/s): the producer bulk-stores them into a four-slot ring in global memory owned
+// L2 150-220 GB/s): the producer bulk-stores them into a six-slot ring in global memory owned
 // by the consumer's SM, the consumer TMA-loads them two chunks ahead into a two-slot ring in its
 // shared memory. Only the flags use cluster barriers: "gfull" (ring slot written) in the
 // consumer, "gfree" (ring slot read) in each producer. Every wait is bounded.
@@ -55,7 +55,7 @@ constexpr uint32_t S_YW = 0;          // [Yh^T (rows key ch 0..127) | Wh^T (rows
 constexpr uint32_t S_GQ = 24576;      // [Gm | Qh]: MN-major (K = key ch), three 64-wide N atoms
 constexpr uint32_t S_FAC = 73728;     // e^{gamma_ref}[128], e^{gamma_C}[128] (fp32)
 constexpr uint32_t kSlotBytes = 74752;
-constexpr int kRing = 4;                                // global ring slots per consumer SM
+constexpr int kRing = 6;                                // global ring slots per consumer SM
 
 // ---- consumer shared memory ----
 constexpr uint32_t C_SLOT0 = 0;                       // two slots
@@ -80,25 +80,25 @@ constexpr uint32_t kSmemBytes = (P_MISC > C_MISC ? P_MISC : C_MISC) + kMiscBytes
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(2 * kC * kLd * 4 + 4 * 16 * kLdY * 4 <= P_LK, "inverse scratch");
 
-// misc areas: 12 mbarriers at 8-byte steps, then scalars
-constexpr uint32_t kBars = 12;
-constexpr uint32_t M_TMEM = 96;
-constexpr uint32_t M_TMP = 100;       // unit_of scratch
-constexpr uint32_t M_SMID = 104;      // consumer: its SM id (selects the global ring)
+// misc areas: 16 mbarriers at 8-byte steps, then scalars
+constexpr uint32_t kBars = 16;
+constexpr uint32_t M_TMEM = 128;
+constexpr uint32_t M_TMP = 132;       // unit_of scratch
+constexpr uint32_t M_SMID = 136;      // consumer: its SM id (selects the global ring)
 // consumer
 constexpr uint32_t M_BAR_S = 0;       // chain MMAs up to the state part
 constexpr uint32_t M_BAR_O = 8;       // chain MMAs up to the output part
 constexpr uint32_t M_LFULL = 16;      // shared slot [2] loaded from the ring
 constexpr uint32_t M_BAR_V = 32;      // V ring [3]
-constexpr uint32_t M_GFULL = 56;      // global ring slot [4] written (producer arrival)
+constexpr uint32_t M_GFULL = 80;      // global ring slot [kRing] written (producer arrival)
 // producer
 constexpr uint32_t M_BAR_MMA = 0;
 constexpr uint32_t M_BAR_QK = 8;
 constexpr uint32_t M_BAR_G = 16;
-constexpr uint32_t M_GFREE = 24;      // [4] per ring slot: its previous chunk was read (one barrier
+constexpr uint32_t M_GFREE = 24;      // [kRing] per ring slot: its previous chunk was read (one barrier
                                       // per slot, so arrivals for later chunks never overrun)
-constexpr uint32_t M_BETA = 128;      // beta[64]
-constexpr uint32_t M_GSUM = 384;      // [4][128] token-quarter decay sums
+constexpr uint32_t M_BETA = 192;      // beta[64]
+constexpr uint32_t M_GSUM = 448;      // [4][128] token-quarter decay sums
 static_assert(M_GSUM + 4 * 128 * 4 <= kMiscBytes && M_GFULL + 8 * kRing <= 8 * kBars &&
               M_GFREE + 8 * kRing <= M_GFULL, "misc area");
 
@@ -235,14 +235,16 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
 
     const uint32_t c_misc = map_to_rank(sb + C_MISC, 0);
     uint8_t* ring = p.ring + (size_t)ld_cluster_u32(c_misc + M_SMID) * (kRing * kSlotBytes);
-    // Chunk whose ring store (one bulk copy by thread 0) was issued but not yet announced (-1:
-    // none). It is announced when the next chunk is handed off, a whole task later, so the wait
-    // for its completion is normally free: thread 0 waits for its bulk group, then arrives on
-    // the consumer's "gfull" barrier of that ring slot.
+    // Chunk whose ring stores were issued but not yet announced (-1: none). Thread 0 stores a
+    // chunk as two bulk groups, [Yh^T|Wh^T] right after its staging and [Gm|Qh|factors] at the
+    // hand-off, and announces it when it hands off its next chunk, a whole task later: it waits
+    // until only the newest group (the next chunk's first) may still be in flight, then
+    // arrives on the consumer's "gfull" barrier of that ring slot.
     int pending = -1;
-    auto announce = [&]() {
+    auto announce = [&](bool last) {
         if (tid == 0 && pending >= 0) {
-            bulk_wait0();
+            if (last) bulk_wait0();
+            else asm volatile("cp.async.bulk.wait_group 1;" ::: "memory");
             fence_proxy_async_global();
             mbar_arrive_remote(c_misc + M_GFULL + 8u * (uint32_t)(pending % kRing));
         }
@@ -281,17 +283,22 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
     }
 
     int n = prank - 1;
+    float beta_nx = 0.f;                    // beta of the next task, loaded a task ahead
     if (n < nchunks) {
         const int64_t c0 = bos + (int64_t)n * kC;
         issue_qk(c0);
         issue_g(c0);
+        if (tid < kC && c0 + tid < eos) beta_nx = p.beta[(c0 + tid) * H + h];
     }
     for (int task = 0; n < nchunks && !aborted; n += kProducers, ++task) {
         const int64_t c0 = bos + (int64_t)n * kC;
         const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
         const bool has_next = n + kProducers < nchunks;
         const int64_t c_next = c0 + (int64_t)kProducers * kC;
-        if (tid < kC) s_beta[tid] = tid < L ? p.beta[(c0 + tid) * H + h] : 0.f;
+        trace_mark(prank, n, 14);
+        if (tid < kC) s_beta[tid] = beta_nx;    // (zero past the sequence)
+        beta_nx = 0.f;
+        if (has_next && tid < kC && c_next + tid < eos) beta_nx = p.beta[(c_next + tid) * H + h];
         if (!wait_local(bar_qk, ph_qk) || !wait_local(bar_g, ph_g)) { aborted = true; break; }
         trace_mark(prank, n, 0);
 
@@ -536,17 +543,13 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             }
             __syncwarp();
         }
-        if (tid == 0) bulk_wait_read0();        // the staging is free once the ring store read it
+        // the [Yh^T|Wh^T] staging is free once the previous chunk's first ring store read it
+        if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
         if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
         trace_mark(prank, n, 13);
         if (has_next) issue_g(c_next);          // R and Rh are dead
         trace_mark(prank, n, 7);
         tc_fence_after();
-        if (qt == 0) {
-            float* fs = reinterpret_cast<float*>(sm + P_ST + S_FAC);
-            fs[c] = fac_r;
-            fs[128 + c] = fac_c;
-        }
         {
             float val[16];
             tmem_ld16(tm + lane_sel + TP_Y + 16 * wg, val);
@@ -564,6 +567,18 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         tc_fence_before();
         __syncthreads();
         trace_mark(prank, n, 8);
+        // ring slot n % kRing must have been read by the consumer (chunk n - kRing), then the
+        // first group of this chunk's ring stores goes out while the [Gm | Qh] products run
+        if (n >= kRing) {
+            const int rs = n % kRing;
+            const bool ok = block_wait(bar_gfree + rs, (ph_gfree >> rs) & 1u, true, p.err);
+            ph_gfree ^= 1u << rs;
+            if (!ok) { aborted = true; break; }
+        }
+        if (tid == 0) {
+            bulk_store(ring + (size_t)(n % kRing) * kSlotBytes + S_YW, sb + P_ST + S_YW, S_GQ - S_YW);
+            bulk_commit();
+        }
 
         // ---- [Gm | Qh] = -Lk^T [Yh | Wh] + Lq^T [0 | I] (M = key ch, N = 192) ----
         if (warp == 0) {
@@ -585,9 +600,16 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             }
             __syncwarp();
         }
+        // the [Gm | Qh | factors] staging is free once the previous chunk's second store read it
+        if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
         if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
         trace_mark(prank, n, 9);
         tc_fence_after();
+        if (qt == 0) {
+            float* fs = reinterpret_cast<float*>(sm + P_ST + S_FAC);
+            fs[c] = fac_r;
+            fs[128 + c] = fac_c;
+        }
 #pragma unroll
         for (int part = 0; part < 3; ++part) {
             float val[16];
@@ -604,23 +626,17 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         __syncthreads();
         trace_mark(prank, n, 10);
 
-        // ---- hand-off: bulk stores into ring slot n % kRing (once chunk n - kRing was read) ----
-        if (n >= kRing) {
-            const int rs = n % kRing;
-            const bool ok = block_wait(bar_gfree + rs, (ph_gfree >> rs) & 1u, true, p.err);
-            ph_gfree ^= 1u << rs;
-            if (!ok) { aborted = true; break; }
-        }
+        // ---- hand-off: announce the previous chunk, then the second group of this one ----
         trace_mark(prank, n, 11);
-        announce();                             // the previous chunk, stored a task ago
+        announce(false);                        // the previous chunk, stored a task ago
         if (tid == 0) {
-            bulk_store(ring + (size_t)(n % kRing) * kSlotBytes, sb + P_ST, kSlotBytes);
+            bulk_store(ring + (size_t)(n % kRing) * kSlotBytes + S_GQ, sb + P_ST + S_GQ, kSlotBytes - S_GQ);
             bulk_commit();
         }
         pending = n;
         trace_mark(prank, n, 12);
     }
-    if (!aborted) announce();
+    if (!aborted) announce(true);
     if (tid == 0) bulk_wait0();
 }
 
