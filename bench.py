@@ -58,6 +58,16 @@ def measured_traffic(workload):
     return nbytes if h.hexdigest() == digest else None
 
 
+def max_over_ranks(dist, torch, value, device, world):
+    """The largest `value` over all ranks (every rank gets it); `value` itself when world == 1.
+    Timings of a multi-GPU run are the slowest rank's."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -337,11 +347,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms_total = sum(times)
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(dist, torch, sum(times), dev, world)
     ms_step = ms_total / args.steps
     value = units * world * args.steps / (ms_total / 1e3)
     achieved = algo_bytes / (statistics.mean(times) / 1e3) / 1e9
@@ -376,11 +382,7 @@ def run_ours(args):
             o_host.copy_(o, non_blocking=True)
             ht_host.copy_(ht, non_blocking=True)
         et = _events_time(torch, e2e_step, max(2, args.steps // 2), 2, stream=stream)
-        ems = sum(et)
-        if world > 1:
-            tt = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = max_over_ranks(dist, torch, sum(et), dev, world)
         e2e = {"value": units * world * len(et) / (ems / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ems / len(et)}

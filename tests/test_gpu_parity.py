@@ -284,3 +284,18 @@ def test_device_error_word_is_clear():
     d = make_prefill(small("prefill_8k", N=1, H=2, T=64, seed=35), DEV)
     run_chunk(d)
     assert kda.last_device_error() == kda.KDA_OK
+
+
+@pytest.mark.parametrize("n_seq,max_len,scale", [(600, 70, 0.125), (40, 300, 2.0)])
+def test_chunk_scale_and_many_sequences(n_seq, max_len, scale):
+    """Output scale on the tensor-core path (applied when O leaves tensor memory), and more
+    packed sequences than the kernel orders by length (it orders at most one per thread)."""
+    rng = np.random.default_rng(n_seq)
+    lens = [int(x) for x in rng.integers(0, max_len + 1, size=n_seq)]
+    wl = small("prefill_8k", N=n_seq, H=2, io="bf16", h0_std=0.02, seed=39)
+    d = make_prefill(wl, DEV, lengths=lens)
+    d["scale"] = scale
+    o, ht = run_chunk(d)
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == kda.KDA_OK
+    check_prefill(d, d["q"], d["k"], d["v"], o, ht)
