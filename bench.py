@@ -36,9 +36,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # It is reported only while that kernel's sources hash to what was profiled.
 MEASURED_TRAFFIC = {
     "prefill_8k": (("chunk_tcx.cu", "tc.cuh", "common.cuh", "tma_host.h"),
-                   "b401fbb50e36e0f02159f88cb55684a769df0539635903b04c4c4b6754b66ee9", 392316416),
+                   "1f0cbb6b8afe311f2be7b3692bea42c8b2498688bca971080afa3bc5ea9b5adb", 392788480),
     "conv_8k": (("conv.cu", "common.cuh"),
-                "fe0d33018f85dfbb956b4758e5422eb013df5d6703f26c1e77d2b01afd8281d0", 359109376),
+                "57851013be10bf43df46ad41c337896a25884525ab4b3b12a15eae74d91c97b3", 357546240),
     "decode_256x32": (("recurrent_step.cu", "common.cuh"),
                       "77c4ec89d7d467c1f5a8ac71bee67eacdc51b3a44d5a73ae884d6db155449850", 1030215424),
 }
