@@ -107,7 +107,7 @@ kda_status kda_conv_fwd(const void* q_raw, const void* k_raw, const void* v_raw,
  * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd needs
  * for these sizes (written to *bytes, host). Zero means none; the call then
  * accepts workspace == NULL. The bf16, dk = dv = 128, chunk-64 prefill needs a
- * fixed ~71.8 MB whatever the batch: per-SM hand-off rings through which the
+ * fixed ~56.0 MB whatever the batch: per-SM hand-off rings through which the
  * kernel's producer CTAs pass each chunk's operands to its consumer CTA via L2.
  * The contents need no initialisation and are dead after the call; one
  * workspace may serve consecutive calls on one stream, not concurrent ones.

@@ -4,31 +4,34 @@
 // The recurrence (sarnas.ru, "Яндекс открыл веса AliceAI-Foundation-80B-A3B-Base ...", section
 // "Что именно изменилось"; m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...") is
 // linear in the state, so one chunk maps the state at its start, S, to the state at its end by
-// S' = M S + N with M, N built from the chunk's inputs alone. This kernel splits exactly along
-// that line: producers build everything that does not depend on S; the consumer applies it.
-// With gamma the within-chunk cumulative log-decay, gamma_C its last row and gamma_ref a
+// S' = M S + N with M, N built from the chunk's inputs alone. This kernel splits along that
+// line: producers build the chunk's factors, which do not depend on S; the consumer applies
+// them. With gamma the within-chunk cumulative log-decay, gamma_C its last row and gamma_ref a
 // per-chunk reference (the chunk middle, or 0 when a half chunk decays by more than 80 in some
 // channel), per chunk:
 //   Lk = k e^{gamma - gamma_ref},  Lq = q e^{gamma - gamma_ref}
 //   R = k e^{gamma_ref - gamma},   Rh = k e^{gamma_C - gamma}              (every Rh <= |k|)
 //   [A ; P] = [Lk ; Lq] R^T   (strictly / inclusively lower triangular parts)
 //   T' = (I + diag(beta) A)^-1 diag(beta)
-//   Yh^T = Rh^T T',  Wh^T = P T',  Gm = -Lk^T Yh,  Qh = Lq^T - Lk^T Wh
+//   Yh^T = Rh^T T',  Wh^T = P T'
 // and with Sm = S^T diag(e^{gamma_ref}) (bf16), on the consumer:
-//   S'^T = S^T diag(e^{gamma_C}) + V^T Yh + Sm Gm        (fp32 state, fp32 decay term)
-//   O^T  = scale (V^T Wh + Sm Qh)
-// A chunk that fails the range test forms A and P' exactly on CUDA cores (gamma_ref = 0, so
+//   X = Sm Lk^T,  U = V^T - X                            (the part of V the state misses)
+//   S'^T = S^T diag(e^{gamma_C}) + U Yh                  (fp32 state, fp32 decay term)
+//   O^T  = scale (Sm Lq^T + U Wh)
+// A chunk that fails the range test forms A and P exactly on CUDA cores (gamma_ref = 0, so
 // every factor is <= 1).
 //
-// Cluster of 4 CTAs: rank 0 is the consumer. Per chunk it issues V^T [Yh | Wh] as soon as the
-// operands are in, then the chain Sm [Gm | Qh] (A operand Sm in tensor memory), updates the fp32
-// state in registers and writes the next Sm back to tensor memory; O leaves through a TMA
-// store. Ranks 1..3 are producers, each preparing every third chunk. A chunk's operands travel
-// through L2, not DSMEM (bulk copies between SMs of a cluster move ~30-60 GB/s, TMA loads from
-// L2 150-220 GB/s): the producer bulk-stores them into a six-slot ring in global memory owned
-// by the consumer's SM, the consumer TMA-loads them two chunks ahead into a two-slot ring in its
-// shared memory. Only the flags use cluster barriers: "gfull" (ring slot written) in the
-// consumer, "gfree" (ring slot read) in each producer. Every wait is bounded.
+// Cluster of 4 CTAs: rank 0 is the consumer, ranks 1..3 are producers, each preparing every
+// third chunk. Per chunk the consumer runs two tensor-core groups with the A operand in tensor
+// memory: Sm [Lk^T | Lq^T] into [X | O], then, once U is written back, U [Yh | Wh] into the
+// state delta and O. It keeps the fp32 state in registers; O leaves through a TMA store. A
+// chunk's factors (57 KB) travel through L2, not DSMEM (bulk copies between SMs of a cluster
+// move ~30-60 GB/s, TMA loads from L2 150-220 GB/s): the producer bulk-stores them into a
+// six-slot ring in global memory owned by the consumer's SM (Lk and Lq straight from its own
+// A|P operand tiles, which have the consumer's layout), and the consumer TMA-loads them two
+// chunks ahead into a two-slot ring in its shared memory. Only the flags use cluster
+// barriers: "gfull" (ring slot written) in the consumer, "gfree" (ring slot read) in each
+// producer. Every wait is bounded.
 #include "common.cuh"
 #include "launchers.h"
 #include "tc.cuh"
@@ -49,12 +52,13 @@ constexpr long long kWaitCycles = 4000000000LL;
 constexpr int kLd = 68;                // fp32 row stride of the 64x64 scratch (16-byte rows)
 constexpr int kLdY = 24;               // row stride of the per-warp 16x16 merge scratch
 
-// ---- one chunk's hand-off (identical image in the producer's staging and a consumer slot) ----
-constexpr uint32_t S_YW = 0;          // [Yh^T (rows key ch 0..127) | Wh^T (rows token 0..63)]:
+// ---- one chunk's hand-off (identical image in a global ring slot and a consumer slot) ----
+constexpr uint32_t S_LK = 0;          // [Lk | Lq]: MN-major (K = key ch, N = token), two
+constexpr uint32_t S_LQ = 16384;      //   64-wide N atoms; the producer's A|P operand image
+constexpr uint32_t S_YW = 32768;      // [Yh^T (rows key ch 0..127) | Wh^T (rows token 0..63)]:
                                       //   K-major (K = token), one 128B-swizzled atom column
-constexpr uint32_t S_GQ = 24576;      // [Gm | Qh]: MN-major (K = key ch), three 64-wide N atoms
-constexpr uint32_t S_FAC = 73728;     // e^{gamma_ref}[128], e^{gamma_C}[128] (fp32)
-constexpr uint32_t kSlotBytes = 74752;
+constexpr uint32_t S_FAC = 57344;     // e^{gamma_ref}[128], e^{gamma_C}[128] (fp32)
+constexpr uint32_t kSlotBytes = 58368;
 constexpr int kRing = 6;                                // global ring slots per consumer SM
 
 // ---- consumer shared memory ----
@@ -65,20 +69,24 @@ constexpr uint32_t C_MISC = C_OST + 16384;
 // ---- producer shared memory ----
 constexpr uint32_t P_X = 0;           // raw q, k [64][128] bf16 (folds), then the inverse's
                                       // scratch Nm, Tm [64][68], Y [3][16][24] (fp32)
-constexpr uint32_t P_LK = 40960;      // Lk : rows key ch, K = token (A|P A block 0; K-major A)
-constexpr uint32_t P_LQ = 57344;      // Lq: same layout (A|P A block 1; K-major A)
+constexpr uint32_t P_LK = 40960;      // Lk : rows key ch, N = token (A|P A block 0, MN-major)
+constexpr uint32_t P_LQ = 57344;      // Lq : same layout (A|P A block 1)
 constexpr uint32_t P_RT = 73728;      // R  : B of A|P. Raw g (fp32, 32 KB) spans P_RT..P_RH
 constexpr uint32_t P_RH = 90112;      // Rh : K-major A of Yh^T
 constexpr uint32_t P_PO = 106496;     // P' : rows token, K = token (K-major A of Wh^T; the
                                       //      M = 128 padding rows read T' below)
 constexpr uint32_t P_TP = 114688;     // T' : rows token, columns token (MN-major B)
-constexpr uint32_t P_ID = 122880;     // identity 64x64 (K-major B of the Lq term)
-constexpr uint32_t P_ST = 131072;     // hand-off staging (S_YW, S_GQ); exact path: Aex, gamma
-constexpr uint32_t P_MISC = P_ST + kSlotBytes;
+constexpr uint32_t P_AEX = 122880;    // exact path: diag(beta) A, fp32 [64][64]
+constexpr uint32_t P_GX = 139264;     // exact path: natural-log gamma, fp32 [64][128]
+constexpr uint32_t P_ST = 172032;     // hand-off staging: [Yh^T | Wh^T], then the factors
+constexpr uint32_t P_MISC = P_ST + (kSlotBytes - S_YW);
 constexpr uint32_t kMiscBytes = 2560;
 constexpr uint32_t kSmemBytes = (P_MISC > C_MISC ? P_MISC : C_MISC) + kMiscBytes + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(2 * kC * kLd * 4 + 4 * 16 * kLdY * 4 <= P_LK, "inverse scratch");
+static_assert(P_LQ - P_LK == S_LQ - S_LK && S_LQ + 16384 == S_YW && S_FAC - S_YW == 24576 &&
+              P_GX + kC * kD * 4 <= P_ST, "producer layout");
+static_assert(kSlotBytes % 1024 == 0 && S_FAC + 1024 <= kSlotBytes, "slot layout");
 
 // misc areas: 16 mbarriers at 8-byte steps, then scalars
 constexpr uint32_t kBars = 16;
@@ -86,10 +94,11 @@ constexpr uint32_t M_TMEM = 128;
 constexpr uint32_t M_TMP = 132;       // unit_of scratch
 constexpr uint32_t M_SMID = 136;      // consumer: its SM id (selects the global ring)
 // consumer
-constexpr uint32_t M_BAR_S = 0;       // chain MMAs up to the state part
-constexpr uint32_t M_BAR_O = 8;       // chain MMAs up to the output part
+constexpr uint32_t M_BAR_S = 0;       // U Yh (the state delta) done
+constexpr uint32_t M_BAR_O = 8;       // U Wh (the output) done
 constexpr uint32_t M_LFULL = 16;      // shared slot [2] loaded from the ring
 constexpr uint32_t M_BAR_V = 32;      // V ring [3]
+constexpr uint32_t M_BAR_X = 56;      // Sm [Lk^T | Lq^T] done
 constexpr uint32_t M_GFULL = 80;      // global ring slot [kRing] written (producer arrival)
 // producer
 constexpr uint32_t M_BAR_MMA = 0;
@@ -100,12 +109,13 @@ constexpr uint32_t M_GFREE = 24;      // [kRing] per ring slot: its previous chu
 constexpr uint32_t M_BETA = 192;      // beta[64]
 constexpr uint32_t M_GSUM = 448;      // [4][128] token-quarter decay sums
 static_assert(M_GSUM + 4 * 128 * 4 <= kMiscBytes && M_GFULL + 8 * kRing <= 8 * kBars &&
-              M_GFREE + 8 * kRing <= M_GFULL, "misc area");
+              M_GFREE + 8 * kRing <= M_GFULL && M_BAR_X + 8 <= M_GFULL, "misc area");
 
-// consumer TMEM columns: D0 = [S part (128) | O part (64)], D1 likewise, Sm (64 cols of bf16 pairs)
-constexpr uint32_t TD0 = 0, TD1 = 256, TC_SM = 448, kTmemC = 512;
+// consumer TMEM columns: [X | O] (64 + 64) for even and odd chunks, the state delta (128),
+// Sm (64 columns of bf16 pairs), U (32 columns of bf16 pairs)
+constexpr uint32_t TXO0 = 0, TXO1 = 128, TC_DS = 256, TC_SM = 384, TC_U = 448, kTmemC = 512;
 // producer TMEM columns
-constexpr uint32_t TP_AP = 0, TP_Y = 64, TP_W = 128, TP_GQ = 256, kTmemP = 512;
+constexpr uint32_t TP_AP = 0, TP_Y = 64, TP_W = 128, kTmemP = 256;
 
 struct Params {
     CUtensorMap tq, tk, tg, tv, to;   // TMA maps: q, k, o [T,H,128] bf16 and g [T,H,128] f32 in
@@ -150,6 +160,54 @@ __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, bool 
     return __syncthreads_or(fail) == 0;
 }
 
+// The same with a flag of the caller's that is OR-ed into the result.
+__device__ __forceinline__ bool block_wait_or(uint64_t* bar, uint32_t parity, int fail,
+                                              unsigned int* err) {
+    if (threadIdx.x == kPoller && !mbar_wait_bounded(bar, parity, kWaitCycles)) {
+        atomicOr(err, kErrTimeout);
+        fail = 1;
+    }
+    return __syncthreads_or(fail) == 0;
+}
+// Named barrier 1 over warps 1..15 (warp 0 issues the consumer's MMAs meanwhile), with an
+// OR-reduction of `pred`.
+constexpr int kGroupThreads = kThreads - 32;
+__device__ __forceinline__ int group_sync_or(int pred) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.s32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, 1, %2, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred), "n"(kGroupThreads)
+        : "memory");
+    return r;
+}
+__device__ __forceinline__ void group_sync() {
+    asm volatile("barrier.cta.sync 1, %0;" ::"n"(kGroupThreads) : "memory");
+}
+// Bounded wait of warps 1..15 for up to two barriers (the poller is in warp 15).
+__device__ __forceinline__ bool group_wait(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1,
+                                           unsigned int* err) {
+    int fail = 0;
+    if (threadIdx.x == kPoller) {
+        const bool ok = mbar_wait_bounded(b0, p0, kWaitCycles) &&
+                        (b1 == nullptr || mbar_wait_bounded(b1, p1, kWaitCycles));
+        if (!ok) {
+            atomicOr(err, kErrTimeout);
+            fail = 1;
+        }
+    }
+    return group_sync_or(fail) == 0;
+}
+// Bounded wait of warp 0 on its own (every lane observes the barrier).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned int* err) {
+    const bool ok = mbar_wait_bounded(bar, parity, kWaitCycles);
+    if (!ok && (threadIdx.x & 31) == 0) atomicOr(err, kErrTimeout);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // Sequence / head of this cluster. Packed batches with at most 256 sequences are processed
 // longest first: cluster u takes the sequence of descending-length rank u / H (ties by index).
 // Every thread of the CTA must call this (it synchronises the CTA once).
@@ -182,16 +240,16 @@ __device__ void unit_of(const Params& p, int unit, int* s_tmp, int& n, int& h, i
 }
 
 // Exact A and P on CUDA cores for a chunk whose decay fails the range test (one warp per (r, i)
-// pair, lanes over channels): A (times beta) into an fp32 [64][64] scratch in the hand-off
-// staging, P into its bf16 operand. Rare, so kept out of line, away from the common path's
+// pair, lanes over channels): A (times beta) into an fp32 [64][64] scratch, P into its bf16
+// operand. Rare, so kept out of line, away from the common path's
 // instruction stream. Every thread of the CTA calls it.
 __device__ __noinline__ void exact_ap(uint8_t* sm, const float* s_beta, int L) {
     const int tid = threadIdx.x, warp = tid >> 5;
     const __nv_bfloat16* Xq = reinterpret_cast<const __nv_bfloat16*>(sm + P_X);
     const __nv_bfloat16* Xk = reinterpret_cast<const __nv_bfloat16*>(sm + P_X + 16384);
     __nv_bfloat16* Pop = reinterpret_cast<__nv_bfloat16*>(sm + P_PO);
-    const float* Gx = reinterpret_cast<const float*>(sm + P_ST + S_GQ);
-    float* Aex = reinterpret_cast<float*>(sm + P_ST + S_YW);        // [64][64]
+    const float* Gx = reinterpret_cast<const float*>(sm + P_GX);
+    float* Aex = reinterpret_cast<float*>(sm + P_AEX);              // [64][64]
     const int lane = tid & 31;
     for (int pidx = warp; pidx < kC * (kC + 1) / 2; pidx += kThreads / 32) {
         int r = (int)((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
@@ -236,10 +294,10 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
     const uint32_t c_misc = map_to_rank(sb + C_MISC, 0);
     uint8_t* ring = p.ring + (size_t)ld_cluster_u32(c_misc + M_SMID) * (kRing * kSlotBytes);
     // Chunk whose ring stores were issued but not yet announced (-1: none). Thread 0 stores a
-    // chunk as two bulk groups, [Yh^T|Wh^T] right after its staging and [Gm|Qh|factors] at the
-    // hand-off, and announces it when it hands off its next chunk, a whole task later: it waits
-    // until only the newest group (the next chunk's first) may still be in flight, then
-    // arrives on the consumer's "gfull" barrier of that ring slot.
+    // chunk as two bulk groups, [Lk | Lq] from the A|P operand tiles right after the folds and
+    // [Yh^T | Wh^T | factors] from the staging at the end of the task, and announces it in the
+    // producer's next task once only that task's first group may still be in flight: it
+    // then arrives on the consumer's "gfull" barrier of that ring slot.
     int pending = -1;
     auto announce = [&](bool last) {
         if (tid == 0 && pending >= 0) {
@@ -273,15 +331,6 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         }
     };
 
-    // identity (B operand of the Lq term of Qh), written once
-    for (int e = tid; e < kC * 8; e += kThreads) {
-        const int r = e >> 3, q8 = e & 7;
-        float v8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v8[u] = (8 * q8 + u == r) ? 1.f : 0.f;
-        st16(sm, P_ID + kmaj_chunk(r, q8, 0, 64), pack8(v8));
-    }
-
     int n = prank - 1;
     float beta_nx = 0.f;                    // beta of the next task, loaded a task ahead
     if (n < nchunks) {
@@ -300,6 +349,17 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         beta_nx = 0.f;
         if (has_next && tid < kC && c_next + tid < eos) beta_nx = p.beta[(c_next + tid) * H + h];
         if (!wait_local(bar_qk, ph_qk) || !wait_local(bar_g, ph_g)) { aborted = true; break; }
+        // ring slot n % kRing must have been read by the consumer (chunk n - kRing)
+        if (n >= kRing) {
+            const int rs = n % kRing;
+            const bool ok = block_wait(bar_gfree + rs, (ph_gfree >> rs) & 1u, true, p.err);
+            ph_gfree ^= 1u << rs;
+            if (!ok) { aborted = true; break; }
+        }
+        uint8_t* slot = ring + (size_t)(n % kRing) * kSlotBytes;
+        // the previous task's [Lk | Lq] store must have read the operand tiles before the folds
+        // below overwrite them (its second group may still be in flight)
+        if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
         trace_mark(prank, n, 0);
 
         // ---- cumulative decay (thread: channel c = row, tokens [16*qt, 16*qt + 16)) ----
@@ -333,18 +393,14 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         const float gr = bad ? 0.f : gA;        // reference for Lk, Lq, R (token 31, or 0)
         const float gs = bad ? gC : gA;         // R's reference (the exact path does not use R)
         const float rhf = ex2_approx(gC - gs);  // Rh = R * rhf
-        // this chunk's factors, written into the staging once the previous ring store read it
-        const float fac_r = ex2_approx(gr), fac_c = ex2_approx(gC);
-        if (bad) {
-            // exact path: natural-log gamma goes to the hand-off staging, which the previous
-            // chunk's ring store must have read
-            if (tid == 0) bulk_wait_read0();
-            __syncthreads();
-            float* Gx = reinterpret_cast<float*>(sm + P_ST + S_GQ);
+        const float fac_r = ex2_approx(gr), fac_c = ex2_approx(gC);   // staged with Yh, Wh
+        if (bad) {                              // exact path: natural-log gamma
+            float* Gx = reinterpret_cast<float*>(sm + P_GX);
 #pragma unroll
             for (int t = 0; t < 16; ++t) Gx[(16 * qt + t) * kD + c] = gam[t] * (1.f / kLog2e);
         }
-        // ---- folded operands Lk, Lq (A of A|P), R (B of A|P), Rh: 8 tokens per 16-byte store ----
+        // ---- folded operands Lk, Lq (A of A|P, and the consumer's B of Sm [Lk^T | Lq^T]),
+        // R (B of A|P), Rh: 8 tokens per 16-byte store ----
 #pragma unroll
         for (int q8 = 0; q8 < 2; ++q8) {
             float lk[8], lq[8], rr[8];
@@ -359,19 +415,23 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                 lk[u] = kv * a; lq[u] = qv * a; rr[u] = kv * b;
             }
             const int ch = 2 * qt + q8;         // 8-token chunk index within the 64 tokens
-            st16(sm, P_LK + mnmaj_chunk(c, ch, 0, 16), pack8(lk));
-            st16(sm, P_LQ + mnmaj_chunk(c, ch, 0, 16), pack8(lq));
-            st16(sm, P_RT + mnmaj_chunk(c, ch, 0, 16), pack8(rr));
+            const uint32_t o16 = mnmaj_chunk(c, ch, 0, 16);
+            st16(sm, P_LK + o16, pack8(lk));
+            st16(sm, P_LQ + o16, pack8(lq));
+            st16(sm, P_RT + o16, pack8(rr));
 #pragma unroll
             for (int u = 0; u < 8; ++u) rr[u] *= rhf;
-            st16(sm, P_RH + mnmaj_chunk(c, ch, 0, 16), pack8(rr));
+            st16(sm, P_RH + o16, pack8(rr));
         }
         fence_async_smem();
         __syncthreads();
+        if (tid == 0) {                         // first group: [Lk | Lq]
+            bulk_store(slot + S_LK, sb + P_LK, S_YW - S_LK);
+            bulk_commit();
+        }
         trace_mark(prank, n, 1);
 
         float* Nm = reinterpret_cast<float*>(sm + P_X);
-        __nv_bfloat16* Pop = reinterpret_cast<__nv_bfloat16*>(sm + P_PO);
         if (!bad) {
             if (warp == 0) {
                 tc_fence_after();
@@ -416,7 +476,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             }
         } else {
             exact_ap(sm, s_beta, L);
-            const float* Aex = reinterpret_cast<const float*>(sm + P_ST + S_YW);
+            const float* Aex = reinterpret_cast<const float*>(sm + P_AEX);
             // the raw tiles are dead: move diag(beta) A into the inverse's scratch
             for (int e = tid; e < kC * kC; e += kThreads) Nm[(e >> 6) * kLd + (e & 63)] = Aex[e];
         }
@@ -523,6 +583,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         tc_fence_before();
         __syncthreads();
         if (has_next) issue_qk(c_next);         // the inverse's scratch is dead
+        announce(false);                        // the previous chunk, stored a task ago
         trace_mark(prank, n, 6);
 
         // ---- Yh^T = Rh^T T' (M = key ch) and Wh^T = P' T' (M = token, 64 rows of 128) ----
@@ -543,98 +604,39 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             }
             __syncwarp();
         }
-        // the [Yh^T|Wh^T] staging is free once the previous chunk's first ring store read it
+        // the staging is free once the previous chunk's second group has read it
         if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
         if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
-        trace_mark(prank, n, 13);
-        if (has_next) issue_g(c_next);          // R and Rh are dead
         trace_mark(prank, n, 7);
+        if (has_next) issue_g(c_next);          // R and Rh are dead
         tc_fence_after();
         {
             float val[16];
             tmem_ld16(tm + lane_sel + TP_Y + 16 * wg, val);
 #pragma unroll
             for (int qq = 0; qq < 2; ++qq)
-                st16(sm, P_ST + S_YW + kmaj_chunk(row, 2 * wg + qq, 0, 0), pack8(val + 8 * qq));
+                st16(sm, P_ST + kmaj_chunk(row, 2 * wg + qq, 0, 0), pack8(val + 8 * qq));
             if ((warp & 3) < 2) {               // lanes 0..63 hold Wh^T
                 tmem_ld16(tm + lane_sel + TP_W + 16 * wg, val);
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq)
-                    st16(sm, P_ST + S_YW + kmaj_chunk(128 + row, 2 * wg + qq, 0, 0), pack8(val + 8 * qq));
+                    st16(sm, P_ST + kmaj_chunk(128 + row, 2 * wg + qq, 0, 0), pack8(val + 8 * qq));
+            }
+            if (qt == 0) {
+                float* fs = reinterpret_cast<float*>(sm + P_ST + (S_FAC - S_YW));
+                fs[c] = fac_r;
+                fs[128 + c] = fac_c;
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        trace_mark(prank, n, 8);
-        // ring slot n % kRing must have been read by the consumer (chunk n - kRing), then the
-        // first group of this chunk's ring stores goes out while the [Gm | Qh] products run
-        if (n >= kRing) {
-            const int rs = n % kRing;
-            const bool ok = block_wait(bar_gfree + rs, (ph_gfree >> rs) & 1u, true, p.err);
-            ph_gfree ^= 1u << rs;
-            if (!ok) { aborted = true; break; }
-        }
-        if (tid == 0) {
-            bulk_store(ring + (size_t)(n % kRing) * kSlotBytes + S_YW, sb + P_ST + S_YW, S_GQ - S_YW);
-            bulk_commit();
-        }
-
-        // ---- [Gm | Qh] = -Lk^T [Yh | Wh] + Lq^T [0 | I] (M = key ch, N = 192) ----
-        if (warp == 0) {
-            tc_fence_after();
-            const uint32_t id192 = idesc_bf16(128, 192, false, false, true);
-            const uint32_t id64 = idesc_bf16(128, 64, false, false);
-            const uint64_t aK = make_desc(sb + P_LK, 16, 1024);
-            const uint64_t aQ = make_desc(sb + P_LQ, 16, 1024);
-            const uint64_t bY = make_desc(sb + P_ST + S_YW, 16, 1024);
-            const uint64_t bI = make_desc(sb + P_ID, 16, 1024);
-            if (elect_one()) {
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tm + TP_GQ, desc_add(aK, s * 32), desc_add(bY, s * 32), id192, s > 0);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tm + TP_GQ + 128, desc_add(aQ, s * 32), desc_add(bI, s * 32), id64, 1);
-                mma_commit(bar_mma);
-            }
-            __syncwarp();
-        }
-        // the [Gm | Qh | factors] staging is free once the previous chunk's second store read it
-        if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-        if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
-        trace_mark(prank, n, 9);
-        tc_fence_after();
-        if (qt == 0) {
-            float* fs = reinterpret_cast<float*>(sm + P_ST + S_FAC);
-            fs[c] = fac_r;
-            fs[128 + c] = fac_c;
-        }
-#pragma unroll
-        for (int part = 0; part < 3; ++part) {
-            float val[16];
-            const int col0 = 48 * wg + 16 * part;
-            tmem_ld16(tm + lane_sel + TP_GQ + col0, val);
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const int nc = col0 + 8 * qq;
-                st16(sm, P_ST + S_GQ + mnmaj_chunk(row, (nc & 63) >> 3, nc >> 6, 16), pack8(val + 8 * qq));
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        trace_mark(prank, n, 10);
-
-        // ---- hand-off: announce the previous chunk, then the second group of this one ----
-        trace_mark(prank, n, 11);
-        announce(false);                        // the previous chunk, stored a task ago
-        if (tid == 0) {
-            bulk_store(ring + (size_t)(n % kRing) * kSlotBytes + S_GQ, sb + P_ST + S_GQ, kSlotBytes - S_GQ);
+        if (tid == 0) {                         // second group: [Yh^T | Wh^T | factors]
+            bulk_store(slot + S_YW, sb + P_ST, kSlotBytes - S_YW);
             bulk_commit();
         }
         pending = n;
-        trace_mark(prank, n, 12);
+        trace_mark(prank, n, 8);
     }
     if (!aborted) announce(true);
     if (tid == 0) bulk_wait0();
@@ -646,6 +648,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
     const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, j = tid & 127;
     const uint32_t lane_sel = (uint32_t)(32 * (warp & 3)) << 16;
     uint8_t* misc = sm + C_MISC;
+    uint64_t* bar_x = reinterpret_cast<uint64_t*>(misc + M_BAR_X);
     uint64_t* bar_s = reinterpret_cast<uint64_t*>(misc + M_BAR_S);
     uint64_t* bar_o = reinterpret_cast<uint64_t*>(misc + M_BAR_O);
     uint64_t* bar_lfull = reinterpret_cast<uint64_t*>(misc + M_LFULL);
@@ -654,7 +657,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
     const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
     const int H = p.H;
     const int nchunks = (int)((eos - bos + kC - 1) / kC);
-    uint32_t ph_s = 0, ph_o = 0, ph_lfull = 0, ph_gfull = 0, ph_v = 0;   // bit i: parity of barrier i
+    uint32_t ph_x = 0, ph_s = 0, ph_lfull = 0, ph_gfull = 0, ph_v = 0;   // bit i: barrier i
     const uint8_t* ring = p.ring + (size_t)smid() * (kRing * kSlotBytes);
     const int64_t sbase = ((int64_t)n_seq * H + h) * kD * kD;
 
@@ -663,16 +666,9 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
     for (int cc = 0; cc < 32; ++cc)
         sreg[cc] = p.h0 ? p.h0[sbase + (int64_t)(32 * wg + cc) * kD + j] : 0.f;
 
-    auto wait_bar = [&](uint64_t* bar, uint32_t& ph) -> bool {
-        const bool ok = block_wait(bar, ph & 1u, false, p.err);
-        ph ^= 1u;
-        return ok;
-    };
-    // V tile of chunk nn into ring entry nn % 3 by TMA: two (64 channels x 64 tokens) boxes whose
-    // 128B-swizzled image is exactly the MN-major operand layout. Rows past the sequence do not
-    // matter (the matching rows of Yh and Wh are zero).
-    // Thread kLoader (warp 2) issues every V and ring load, so that it runs beside warp 0's MMA
-    // issue instead of in front of it.
+    // V tile of chunk nn into ring entry nn % 3 by TMA: two (64 channels x 64 tokens) boxes,
+    // 128B-swizzled. Rows past the sequence do not matter (the matching rows of Lk, Yh and Wh
+    // are zero). Thread kLoader (warp 2) issues every V and ring load, beside warp 0's MMA issue.
     constexpr int kLoader = 64;
     auto issue_v = [&](int nn) {
         if (tid == kLoader) {
@@ -684,14 +680,8 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             tma_load_3d(base + 8192, &p.tv, 64, h, c0, bar_v + e);
         }
     };
-    auto wait_v = [&](int nn) -> bool {
-        const int e = nn % 3;
-        const bool ok = block_wait(bar_v + e, (ph_v >> e) & 1u, false, p.err);
-        ph_v ^= 1u << e;
-        return ok;
-    };
-    // Operands of chunk nn from its global ring slot into shared slot nn % 2 (thread 0; the
-    // shared slot must be free): waits for the producer's announcement, then bulk loads.
+    // Factors of chunk nn from its global ring slot into shared slot nn % 2 (the shared slot
+    // must be free): waits for the producer's announcement, then one bulk load.
     auto issue_load = [&](int nn) -> bool {
         bool ok = true;
         if (tid == kLoader) {
@@ -702,55 +692,64 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 fence_proxy_async_global();
                 uint64_t* bl = bar_lfull + (nn & 1);
                 const uint32_t dst = sb + C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
-                const uint8_t* src = ring + (size_t)rs * kSlotBytes;
                 mbar_arrive_expect_tx(bl, kSlotBytes);
-                bulk_load(dst, src, kSlotBytes, bl);                                 // one copy
+                bulk_load(dst, ring + (size_t)rs * kSlotBytes, kSlotBytes, bl);
             } else {
                 atomicOr(p.err, kErrTimeout);
             }
         }
         return ok;
     };
-    // Shared slot nn % 2 holds chunk nn; its ring slot may take chunk nn + kRing.
-    auto wait_full = [&](int nn) -> bool {
-        const int sl = nn & 1;
-        const bool ok = block_wait(bar_lfull + sl, (ph_lfull >> sl) & 1u, false, p.err);
+    // Factors and V tile of chunk nn both in (one polling thread, one block barrier); then
+    // its ring slot may take chunk nn + kRing.
+    auto wait_next = [&](int nn) -> bool {
+        const int sl = nn & 1, e = nn % 3;
+        int fail = 0;
+        if (tid == kPoller) {
+            const bool ok = mbar_wait_bounded(bar_lfull + sl, (ph_lfull >> sl) & 1u, kWaitCycles) &&
+                            mbar_wait_bounded(bar_v + e, (ph_v >> e) & 1u, kWaitCycles);
+            if (!ok) {
+                atomicOr(p.err, kErrTimeout);
+                fail = 1;
+            }
+        }
         ph_lfull ^= 1u << sl;
-        if (!ok) return false;
+        ph_v ^= 1u << e;
+        if (__syncthreads_or(fail)) return false;
         if (tid == 0 && nn + kRing < nchunks)
             mbar_arrive_remote_relaxed(map_to_rank(sb + P_MISC + M_GFREE + 8u * (uint32_t)(nn % kRing),
                                                    1 + (nn + kRing) % kProducers));
         return true;
     };
-    // D(nn) = V^T [Yh | Wh] (one converged warp)
-    auto issue_e = [&](int nn) {
+    // [X | O](nn) = Sm(nn) [Lk^T | Lq^T] (one converged warp; A operand Sm in tensor memory)
+    auto issue_xo = [&](int nn) {
         const uint32_t so = C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
         tc_fence_after();
-        const uint32_t id = idesc_bf16(128, 192, true, false);
-        const uint64_t a0 = make_desc(sb + C_V + (uint32_t)(nn % 3) * 16384, 8192, 1024);
-        const uint64_t b0 = make_desc(sb + so + S_YW, 16, 1024);
-        const uint32_t d = tm + ((nn & 1) ? TD1 : TD0);
+        const uint32_t id = idesc_bf16(128, 128, false, true);
+        const uint64_t b0 = make_desc(sb + so + S_LK, S_LQ - S_LK, 1024);
+        const uint32_t d = tm + ((nn & 1) ? TXO1 : TXO0);
         if (elect_one()) {
 #pragma unroll
-            for (int s = 0; s < 4; ++s) mma_bf16(d, desc_add(a0, s * 2048), desc_add(b0, s * 32), id, s > 0);
+            for (int s = 0; s < 8; ++s) mma_bf16_ts(d, tm + TC_SM + 8 * s, desc_add(b0, s * 2048), id, s > 0);
+            mma_commit(bar_x);
         }
         __syncwarp();
     };
-    // D(nn) += Sm [Gm | Qh]: the state part first (commit S), then the output part (commit O)
-    auto issue_c = [&](int nn) {
+    // state delta U Yh (commit S), then O(nn) += U Wh (commit O); A operand U in tensor memory
+    auto issue_u = [&](int nn) {
         const uint32_t so = C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
         tc_fence_after();
-        const uint32_t idS = idesc_bf16(128, 128, false, true);
-        const uint32_t idO = idesc_bf16(128, 64, false, true);
-        const uint64_t bG = make_desc(sb + so + S_GQ, 16384, 1024);
-        const uint64_t bQ = make_desc(sb + so + S_GQ + 32768, 16384, 1024);
-        const uint32_t d = tm + ((nn & 1) ? TD1 : TD0);
+        const uint32_t idS = idesc_bf16(128, 128, false, false);
+        const uint32_t idO = idesc_bf16(128, 64, false, false);
+        const uint64_t bY = make_desc(sb + so + S_YW, 16, 1024);
+        const uint64_t bW = make_desc(sb + so + S_YW + 128 * 128, 16, 1024);
+        const uint32_t dO = tm + ((nn & 1) ? TXO1 : TXO0) + 64;
         if (elect_one()) {
 #pragma unroll
-            for (int s = 0; s < 8; ++s) mma_bf16_ts(d, tm + TC_SM + 8 * s, desc_add(bG, s * 2048), idS, 1);
+            for (int s = 0; s < 4; ++s) mma_bf16_ts(tm + TC_DS, tm + TC_U + 8 * s, desc_add(bY, s * 32), idS, s > 0);
             mma_commit(bar_s);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) mma_bf16_ts(d + 128, tm + TC_SM + 8 * s, desc_add(bQ, s * 2048), idO, 1);
+            for (int s = 0; s < 4; ++s) mma_bf16_ts(dO, tm + TC_U + 8 * s, desc_add(bW, s * 32), idO, 1);
             mma_commit(bar_o);
         }
         __syncwarp();
@@ -766,18 +765,45 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             w[2 * q4 + 1] = pack_bf16(sreg[4 * q4 + 2] * e.z, sreg[4 * q4 + 3] * e.w);
         }
     };
-    // O of chunk nn: TMEM -> bf16 [token][channel] staging -> one TMA tile store (a ragged last
-    // chunk: one bulk copy per valid token, so rows of the next sequence are never touched)
-    auto epilogue_o = [&](int nn) {
+    // U(nn) = V(nn)^T - X(nn) for value channel j and tokens [16 wg, 16 wg + 16), as bf16
+    // pairs along the token into tensor memory. V[t][j] sits in box j / 64, row t, 16-byte
+    // chunk ((j % 64) / 8) ^ (t % 8) of the 128B-swizzled tile.
+    auto make_u = [&](int nn) {
         tc_fence_after();
-        float ov[16];
-        tmem_ld16(tm + lane_sel + ((nn & 1) ? TD1 : TD0) + 128 + 16 * wg, ov);
-        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
+        float xv[16];
+        tmem_ld16(tm + lane_sel + ((nn & 1) ? TXO1 : TXO0) + 16 * wg, xv);
+        const uint8_t* vt = sm + C_V + (uint32_t)(nn % 3) * 16384 + 8192 * (j >> 6) + (j & 7) * 2;
+        const int jc = (j & 63) >> 3;
+        uint32_t w[8];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) st[(16 * wg + t) * kD + j] = __float2bfloat16_rn(p.scale * ov[t]);
+        for (int u = 0; u < 8; ++u) {
+            const int t0 = 16 * wg + 2 * u;
+            const float v0 = bf(reinterpret_cast<const __nv_bfloat16*>(vt + t0 * 128 + ((jc ^ (t0 & 7)) << 4)));
+            const float v1 = bf(reinterpret_cast<const __nv_bfloat16*>(vt + (t0 + 1) * 128 + ((jc ^ ((t0 + 1) & 7)) << 4)));
+            w[u] = pack_bf16(v0 - xv[2 * u], v1 - xv[2 * u + 1]);
+        }
+        tmem_st8(tm + lane_sel + TC_U + 8 * wg, w);
+        tmem_wait_st();
+    };
+    // O of chunk nn, by warps 1..15 (warp 4 also takes warp 0's share): TMEM -> bf16
+    // [token][channel] staging -> one TMA tile store (a ragged last chunk: one bulk copy per
+    // valid token, so rows of the next sequence are never touched)
+    auto epilogue_o = [&](int nn) -> bool {
+        if (warp == 1) bulk_wait_read0();       // the previous O tile has left the staging
+        const bool ok = group_wait(bar_o, (uint32_t)(nn & 1), nullptr, 0, p.err);   // once per chunk
+        tc_fence_after();
+        const uint32_t to = tm + lane_sel + ((nn & 1) ? TXO1 : TXO0) + 64;
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
+        for (int part = (warp == 4 ? 0 : 1); part < 2; ++part) {
+            const int t0 = part ? 16 * wg : 0;
+            float ov[16];
+            tmem_ld16(to + t0, ov);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) st[(t0 + t) * kD + j] = __float2bfloat16_rn(p.scale * ov[t]);
+        }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        group_sync();
         if (warp == 1) {
             const int64_t c0 = bos + (int64_t)nn * kC;
             const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
@@ -790,17 +816,18 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             }
             bulk_commit();
         }
+        return ok;
     };
 
-    // prologue: V tiles of chunks 0..2, Sm(0), then chunk 0's products
+    // prologue: V tiles of chunks 0..2, factors of chunks 0 and 1, Sm(0), then [X | O](0)
     if (nchunks > 0) {
         issue_v(0);
         if (nchunks > 1) issue_v(1);
         if (nchunks > 2) issue_v(2);
-        // chunk 0 must have arrived (which frees ring slot 0 for chunk 4) before the loader
-        // waits for chunk 1: a producer announces a chunk only when it hands off its next one
+        // chunk 0 must have arrived (which frees ring slot 0 for chunk kRing) before the loader
+        // waits for chunk 1: a producer announces a chunk only during its next task
         if (__syncthreads_or(!issue_load(0))) aborted = true;   // (seen by every thread)
-        if (!aborted && (!wait_full(0) || !wait_v(0))) aborted = true;
+        if (!aborted && !wait_next(0)) aborted = true;
         if (!aborted && nchunks > 1 && __syncthreads_or(!issue_load(1))) aborted = true;
         if (!aborted) {
             uint32_t w[16];
@@ -809,30 +836,53 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             tmem_wait_st();
             tc_fence_before();
             __syncthreads();
-            if (warp == 0) { issue_e(0); issue_c(0); }
+            if (warp == 0) issue_xo(0);
         }
     }
 
+    // Warp 0 issues the MMAs and blocks for about their execution time, so after each issue
+    // warps 1..15 go on alone (named barrier 1) and warp 0 catches up at the next block-wide
+    // barrier. A failed wait only raises `fail`; the block leaves the loop together at the
+    // next block-wide barrier.
+    int fail = 0;
     for (int n = 0; n < nchunks && !aborted; ++n) {
         const float* fac = reinterpret_cast<const float*>(sm + C_SLOT0 + (uint32_t)(n & 1) * kSlotBytes + S_FAC);
-        trace_mark(0, n, 0);
-        // (1) output of the previous chunk, while this chunk's chain runs
-        if (n > 0) epilogue_o(n - 1);
-        trace_mark(0, n, 1);
-        // (2) operands of the next chunk and its V^T products (queued behind this chunk's chain)
         const bool more = n + 1 < nchunks;
-        if (more) {
-            if (!wait_full(n + 1) || !wait_v(n + 1)) { aborted = true; break; }
-            if (warp == 0) issue_e(n + 1);
-        }
+        const int n1 = n + 1, sl1 = n1 & 1, e1 = n1 % 3;
+        trace_mark(0, n, 0);
+        // (1) U(n) = V(n)^T - X(n), then U [Yh | Wh]
+        if (!block_wait_or(bar_x, ph_x & 1u, fail, p.err)) { aborted = true; break; }
+        ph_x ^= 1u;
+        trace_mark(0, n, 1);
+        make_u(n);
+        tc_fence_before();
+        __syncthreads();
         trace_mark(0, n, 2);
-        // (3) state update S' = e^{gamma_C} S + D_S
-        if (!wait_bar(bar_s, ph_s)) { aborted = true; break; }
-        trace_mark(0, n, 3);
+        // (2) the next chunk's operands and this chunk's state delta
+        if (warp == 0) {
+            issue_u(n);
+            trace_mark(0, n, 3);
+            if (more && !warp_wait(bar_lfull + sl1, (ph_lfull >> sl1) & 1u, p.err)) fail = 1;
+            if (!warp_wait(bar_s, ph_s & 1u, p.err)) fail = 1;
+        } else {
+            if (more && !group_wait(bar_lfull + sl1, (ph_lfull >> sl1) & 1u, bar_v + e1, (ph_v >> e1) & 1u, p.err))
+                fail = 1;
+            if (more && tid == 32 && n1 + kRing < nchunks)    // ring slot of n + 1 may take n + 1 + kRing
+                mbar_arrive_remote_relaxed(map_to_rank(sb + P_MISC + M_GFREE + 8u * (uint32_t)(n1 % kRing),
+                                                       1 + (n1 + kRing) % kProducers));
+            if (!group_wait(bar_s, ph_s & 1u, nullptr, 0, p.err)) fail = 1;
+        }
+        if (more) {
+            ph_lfull ^= 1u << sl1;
+            ph_v ^= 1u << e1;
+        }
+        ph_s ^= 1u;
+        trace_mark(0, n, 4);
+        // (3) state update S' = e^{gamma_C} S + U Yh, then Sm(n + 1)
         tc_fence_after();
         {
             float v32[32];
-            tmem_ld32(tm + lane_sel + ((n & 1) ? TD1 : TD0) + 32 * wg, v32);
+            tmem_ld32(tm + lane_sel + TC_DS + 32 * wg, v32);
             const float4* eC4 = reinterpret_cast<const float4*>(fac + 128 + 32 * wg);
 #pragma unroll
             for (int t4 = 0; t4 < 8; ++t4) {
@@ -845,28 +895,31 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 sreg[cc + 3] = fmaf(ec.w, sreg[cc + 3], v[3]);
             }
         }
-        uint32_t w[16];
-        if (more) pack_sm(n + 1, w);
-        if (warp == 1) bulk_wait_read0();       // the staged O tile has been read
-        trace_mark(0, n, 4);
-        if (!wait_bar(bar_o, ph_o)) { aborted = true; break; }
-        trace_mark(0, n, 5);
         if (more) {
+            uint32_t w[16];
+            pack_sm(n1, w);
             tmem_st16(tm + lane_sel + TC_SM + 16 * wg, w);
             tmem_wait_st();
         }
+        trace_mark(0, n, 5);
         tc_fence_before();
-        if (__syncthreads_or(aborted)) { aborted = true; break; }
+        if (__syncthreads_or(fail)) { aborted = true; break; }
         trace_mark(0, n, 6);
-        // (4) chain of the next chunk; beside it, the loads that the completed chunk n made
-        // possible: shared slot n % 2 takes chunk n + 2, V ring entry n % 3 takes V(n + 3)
-        if (more && warp == 0) issue_c(n + 1);
-        if (n + 2 < nchunks) issue_load(n + 2);   // a failed wait flags the error word; the
-                                                  // consumer then gives up at wait_full(n + 2)
-        if (n + 3 < nchunks) issue_v(n + 3);
-        trace_mark(0, n, 7);
+        if (warp == 0) {
+            // (4) the next chunk's [X | O]
+            if (more) issue_xo(n1);
+            trace_mark(0, n, 7);
+        } else {
+            // (4') output of chunk n, then the loads that the completed chunk n made possible:
+            // shared slot n % 2 takes chunk n + 2, V ring entry n % 3 takes V(n + 3)
+            if (!epilogue_o(n)) fail = 1;
+            trace_mark(0, n, 8, 32);
+            if (n + 2 < nchunks) issue_load(n + 2);   // a failed wait flags the error word; the
+                                                      // consumer then gives up at the next wait
+            if (n + 3 < nchunks) issue_v(n + 3);
+            trace_mark(0, n, 9, 32);
+        }
     }
-    if (nchunks > 0 && !aborted) epilogue_o(nchunks - 1);
     if (warp == 1) bulk_wait0();
     if (p.ht && !aborted) {
 #pragma unroll

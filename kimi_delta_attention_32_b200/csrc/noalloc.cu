@@ -14,9 +14,9 @@
 #define KDA_API extern "C" __attribute__((visibility("default")))
 
 namespace {
-// Ring tables for 160 SM ids x 6 slots x 74752 bytes: what kda_chunk_fwd_workspace_size reports
+// Ring tables for 160 SM ids x 6 slots x 58368 bytes: what kda_chunk_fwd_workspace_size reports
 // for the bf16, dk = dv = 128, chunk-64 prefill (checked at every call).
-constexpr size_t kStaticWorkspaceBytes = (size_t)160 * 6 * 74752;
+constexpr size_t kStaticWorkspaceBytes = (size_t)160 * 6 * 58368;
 __device__ __align__(256) uint8_t g_static_workspace[kStaticWorkspaceBytes];
 }  // namespace
 
