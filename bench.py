@@ -36,7 +36,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # It is reported only while that kernel's sources hash to what was profiled.
 MEASURED_TRAFFIC = {
     "prefill_8k": (("chunk_tcx.cu", "tc.cuh", "common.cuh", "tma_host.h"),
-                   "1f0cbb6b8afe311f2be7b3692bea42c8b2498688bca971080afa3bc5ea9b5adb", 392788480),
+                   "0716dc2e7752154918079bf0d08a5f9add4073aca64e868a6b4dd04c972ee6fe", 392807168),
     "conv_8k": (("conv.cu", "common.cuh"),
                 "57851013be10bf43df46ad41c337896a25884525ab4b3b12a15eae74d91c97b3", 357546240),
     "decode_256x32": (("recurrent_step.cu", "common.cuh"),
