@@ -90,3 +90,70 @@ def chunk_fwd(q, k, v, g, beta, scale=1.0, h0=None, cu_seqlens=None, chunk=64, s
                 S = np.exp(last)[:, None] * S + (kc * np.exp(last - gam)).T @ Ut
             ht[n, h] = S
     return o, ht
+
+
+def split_chunk_fwd(q, k, v, g, beta, scale=1.0, h0=None, chunk=64, half_range=80.0,
+                    rounding=None):
+    """The state-transition split that the bf16 prefill kernel computes, for one sequence.
+
+    Per chunk, with gamma the within-chunk cumulative log-decay, gamma_C its last row and
+    gamma_ref = gamma at the chunk middle (or 0 when some channel decays by more than
+    `half_range` in either half of the chunk, the kernel's range test):
+      Lk = k e^{gamma-gamma_ref}, Lq = q e^{gamma-gamma_ref}, R = k e^{gamma_ref-gamma},
+      Rh = k e^{gamma_C-gamma};  A = strict lower part of Lk R^T, P = lower part of Lq R^T
+      (formed exactly from e^{gamma_r-gamma_i} when the range test fails);
+      T' = (I + diag(beta) A)^-1 diag(beta);  Yh^T = Rh^T T',  Wh^T = P T';
+      Sm = S^T diag(e^{gamma_ref}),  X = Sm Lk^T,  U = V^T - X;
+      S'^T = S^T diag(e^{gamma_C}) + U Yh,  O^T = scale (Sm Lq^T + U Wh).
+    `rounding`, if given, is applied where the kernel rounds to bf16 (every tensor-core
+    operand). Returns (o [T, H, dv], ht [1, H, dk, dv], number of chunks that failed the
+    range test).
+    """
+    rnd = rounding or (lambda x: x)
+    q, k, v, g, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    o = np.zeros((T, H, dv))
+    ht = np.zeros((1, H, dk, dv))
+    nbad = 0
+    for h in range(H):
+        S = np.zeros((dk, dv)) if h0 is None else np.array(h0[0, h], dtype=np.float64)
+        for c0 in range(0, T, chunk):
+            L = min(chunk, T - c0)
+
+            def pad(x, width):
+                out = np.zeros((chunk, width))
+                out[:L] = x[c0:c0 + L, h]
+                return out
+
+            qc, kc, vc, gc = pad(q, dk), pad(k, dk), pad(v, dv), pad(g, dk)
+            bc = np.zeros(chunk)
+            bc[:L] = beta[c0:c0 + L, h]
+            gam = np.cumsum(gc, axis=0)
+            g_half, g_last = gam[chunk // 2 - 1], gam[chunk - 1]
+            bad = bool(np.any(g_half < -half_range) or np.any(g_last - g_half < -half_range))
+            nbad += bad
+            g_ref = np.zeros(dk) if bad else g_half
+            Lk = rnd(kc * np.exp(gam - g_ref))
+            Lq = rnd(qc * np.exp(gam - g_ref))
+            Rh = rnd(kc * np.exp(g_last - gam))
+            if bad:
+                E = np.exp(gam[:, None, :] - gam[None, :, :])
+                A = np.einsum('rc,ic,ric->ri', kc, kc, E)
+                P = np.einsum('rc,ic,ric->ri', qc, kc, E)
+            else:
+                R = rnd(kc * np.exp(g_ref - gam))
+                A = Lk @ R.T
+                P = Lq @ R.T
+            A = np.tril(A, -1)
+            P = rnd(np.tril(P))
+            Tp = rnd(np.linalg.inv(np.eye(chunk) + bc[:, None] * A) * bc[None, :])
+            Yt = rnd(Rh.T @ Tp)                      # Yh^T [dk, chunk]
+            Wt = rnd(P @ Tp)                         # Wh^T [chunk, chunk]
+            Sm = rnd(S.T * np.exp(g_ref)[None, :])   # [dv, dk]
+            U = rnd(vc.T - Sm @ Lk.T)                # [dv, chunk]
+            Ot = scale * (Sm @ Lq.T + U @ Wt.T)      # [dv, chunk]
+            o[c0:c0 + L, h] = Ot.T[:L]
+            S = (S.T * np.exp(g_last)[None, :] + U @ Yt.T).T
+        ht[0, h] = S
+    return o, ht, nbad
