@@ -54,6 +54,13 @@ def _declare(lib):
     lib.kda_oracle_conv_silu.restype = None
     lib.kda_oracle_l2norm.argtypes = [_dp, ctypes.c_int64, ctypes.c_int, ctypes.c_double]
     lib.kda_oracle_l2norm.restype = None
+    lib.kda_oracle_gate.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
+    lib.kda_oracle_gate.restype = None
+    lib.kda_oracle_sigmoid.argtypes = [_dp, _dp, ctypes.c_int64]
+    lib.kda_oracle_sigmoid.restype = None
+    lib.kda_oracle_gated_rmsnorm.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int,
+                                             ctypes.c_double]
+    lib.kda_oracle_gated_rmsnorm.restype = None
     return lib
 
 
@@ -182,3 +189,34 @@ def prologue(q_raw, k_raw, v_raw, w_q, w_k, w_v, conv_state=None, cu_seqlens=Non
     k = l2norm(parts[1].reshape(T_tot, H, dk), l2_eps, lib=lib)
     v = parts[2].reshape(T_tot, H, dv)
     return q, k, v, np.concatenate(outs_cache, axis=1)
+
+
+def gate(x, A_log, dt_bias, lib=None):
+    """Per-channel log-decay from raw gate logits: g = -exp(A_log[h]) softplus(x + dt_bias).
+    x: [T_tot, H, dk]; A_log: [H]; dt_bias: [H*dk] (or [H, dk]). Returns g (float64)."""
+    lib = lib or load()
+    x = _f64(x)
+    T_tot, H, dk = x.shape
+    A_log, dt_bias = _f64(A_log).reshape(H), _f64(dt_bias).reshape(H * dk)
+    g = np.zeros_like(x)
+    lib.kda_oracle_gate(_ptr(x), _ptr(A_log), _ptr(dt_bias), _ptr(g), T_tot, H, dk)
+    return g
+
+
+def sigmoid(b_raw, lib=None):
+    """beta = sigmoid(b_raw), elementwise (float64)."""
+    lib = lib or load()
+    b = _f64(b_raw)
+    out = np.zeros_like(b)
+    lib.kda_oracle_sigmoid(_ptr(b), _ptr(out), b.size)
+    return out
+
+
+def gated_rmsnorm(o, z, w, eps=1e-6, lib=None):
+    """y = o / sqrt(mean(o^2) + eps) * w * sigmoid(z) over the last axis (dv); w: [dv]."""
+    lib = lib or load()
+    o, z, w = _f64(o), _f64(z), _f64(w)
+    dv = o.shape[-1]
+    y = np.zeros_like(o)
+    lib.kda_oracle_gated_rmsnorm(_ptr(o), _ptr(z), _ptr(w), _ptr(y), o.size // dv, dv, float(eps))
+    return y

@@ -260,3 +260,58 @@ void kda_oracle_l2norm(double* x, int64_t rows, int d, double eps) {
         for (int i = 0; i < d; ++i) x[(size_t)r * d + i] *= inv;
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Gate activation ([P4]: the gate is computed from a_log_bias and dt_bias;  */
+/* delta is the residual times sigmoid(beta)).                               */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The pages name only the inputs of the gate. Reading: per token t, head h and key channel c,
+ *     g[t, h, c] = -exp(A_log[h]) * softplus(x[t, h, c] + dt_bias[h * dk + c]),
+ *     softplus(z) = log(1 + exp(z)),
+ * so g <= 0 and exp(g) is the per-row forgetting factor of [P1].
+ * x, g : [T_tot, H, dk];  A_log : [H];  dt_bias : [H * dk].
+ */
+void kda_oracle_gate(const double* x, const double* A_log, const double* dt_bias, double* g,
+                     int64_t T_tot, int H, int dk) {
+    for (int64_t t = 0; t < T_tot; ++t)
+        for (int h = 0; h < H; ++h) {
+            const double a = exp(A_log[h]);
+            for (int c = 0; c < dk; ++c) {
+                const size_t i = ((size_t)t * H + h) * dk + c;
+                const double z = x[i] + dt_bias[(size_t)h * dk + c];
+                const double sp = z > 30.0 ? z + log1p(exp(-z)) : log1p(exp(z));
+                g[i] = -a * sp;
+            }
+        }
+}
+
+/* beta = sigmoid(b_raw), elementwise over n values ([P4]). */
+void kda_oracle_sigmoid(const double* b_raw, double* beta, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) beta[i] = 1.0 / (1.0 + exp(-b_raw[i]));
+}
+
+/* ------------------------------------------------------------------------ */
+/* Gated RMSNorm of the output ([P1], "Отвергнутые решения": every norm but   */
+/* the QK norms is a gated RMSNorm).                                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Reading: per token and head, over the dv output channels,
+ *     y = o / sqrt(mean(o^2) + eps) * w * sigmoid(z),
+ * with a weight w [dv] shared by the heads and a gate z of o's shape.
+ * o, z, y : [rows, dv].
+ */
+void kda_oracle_gated_rmsnorm(const double* o, const double* z, const double* w, double* y,
+                              int64_t rows, int dv, double eps) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double ss = 0.0;
+        for (int j = 0; j < dv; ++j) ss += o[(size_t)r * dv + j] * o[(size_t)r * dv + j];
+        const double inv = 1.0 / sqrt(ss / dv + eps);
+        for (int j = 0; j < dv; ++j) {
+            const size_t i = (size_t)r * dv + j;
+            y[i] = o[i] * inv * w[j] * (1.0 / (1.0 + exp(-z[i])));
+        }
+    }
+}

@@ -309,9 +309,81 @@ def pin_prologue_composition(lib):
         _close(cso[0, lo:hi], e[-3:].T, what="prologue cache slice")
 
 
+# --------------------------------------------------------------------------- #
+# Gate activation and output norm                                             #
+# --------------------------------------------------------------------------- #
+# m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...": the gate comes from a_log_bias
+# and dt_bias, and delta is the residual times sigmoid(beta). sarnas.ru, section "Отвергнутые
+# решения": every norm except the QK norms is a gated RMSNorm. The formulas are readings (the
+# pages give only the inputs); the pins below fix them against closed forms and torch's CPU
+# routines.
+
+def pin_gate_closed_form(lib):
+    """x + dt_bias = 0 and A_log = 0 give g = -log 2; A_log = log 3 triples it; a very negative
+    A_log switches the decay off (g -> 0); a large logit makes softplus the identity."""
+    x = np.zeros((2, 3, 4))
+    _close(oracle.gate(x, np.zeros(3), np.zeros(12), lib=lib), -np.log(2.0) * np.ones_like(x),
+           tol=1e-15, what="gate at zero")
+    g = oracle.gate(x, np.log([1.0, 3.0, 1e-30]), np.zeros(12), lib=lib)
+    _close(g[:, 1], -3 * np.log(2.0) * np.ones((2, 4)), tol=1e-14, what="gate A_log scale")
+    assert np.all(np.abs(g[:, 2]) < 1e-29), "gate with A_log -> -inf"
+    big = oracle.gate(np.full((1, 1, 2), 40.0), np.zeros(1), np.array([0.0, 5.0]), lib=lib)
+    _close(big[0, 0], [-40.0, -45.0], tol=1e-15, what="gate softplus linear branch")
+
+
+def pin_gate_matches_torch(lib):
+    """Random logits, per-head A_log and per-channel dt_bias against torch's fp64 softplus."""
+    import torch
+    rng = np.random.default_rng(41)
+    T, H, dk = 9, 3, 8
+    x = rng.normal(0.0, 3.0, (T, H, dk))
+    A_log = rng.normal(0.0, 1.0, H)
+    dt = rng.normal(0.0, 1.0, (H, dk))
+    ref = -(torch.exp(torch.from_numpy(A_log))[None, :, None] *
+            torch.nn.functional.softplus(torch.from_numpy(x) + torch.from_numpy(dt)[None]))
+    g = oracle.gate(x, A_log, dt.reshape(-1), lib=lib)
+    _close(g, ref.numpy(), tol=1e-13, what="gate vs torch softplus")
+    assert np.all(g <= 0.0), "gate must be a decay (g <= 0)"
+
+
+def pin_sigmoid(lib):
+    """beta = sigmoid(b): 1/2 at 0, sigmoid(-b) = 1 - sigmoid(b), and torch's fp64 sigmoid."""
+    import torch
+    b = np.random.default_rng(43).normal(0.0, 4.0, 50)
+    s = oracle.sigmoid(b, lib=lib)
+    _close(oracle.sigmoid(np.zeros(1), lib=lib), [0.5], tol=1e-16, what="sigmoid(0)")
+    _close(s + oracle.sigmoid(-b, lib=lib), np.ones_like(b), tol=1e-15, what="sigmoid symmetry")
+    _close(s, torch.sigmoid(torch.from_numpy(b)).numpy(), tol=1e-15, what="sigmoid vs torch")
+
+
+def pin_gated_rmsnorm(lib):
+    """A constant row normalises to its sign; a large gate passes the plain RMSNorm (torch's
+    rms_norm); a zero gate halves it; and the norm is scale-free."""
+    import torch
+    rng = np.random.default_rng(47)
+    dv = 16
+    w = rng.normal(1.0, 0.2, dv)
+    o = np.full((1, dv), -2.5)
+    y = oracle.gated_rmsnorm(o, np.full((1, dv), 60.0), w, eps=0.0, lib=lib)
+    _close(y[0], -w, tol=1e-14, what="rmsnorm of a constant row")
+    o = rng.normal(0.0, 3.0, (5, 2, dv))
+    z = rng.normal(0.0, 2.0, (5, 2, dv))
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(o), (dv,), torch.from_numpy(w), 1e-6)
+    _close(oracle.gated_rmsnorm(o, np.full_like(o, 60.0), w, 1e-6, lib=lib), ref.numpy(),
+           tol=1e-13, what="rmsnorm vs torch")
+    _close(oracle.gated_rmsnorm(o, np.zeros_like(o), w, 1e-6, lib=lib), 0.5 * ref.numpy(),
+           tol=1e-13, what="gate sigmoid(0) = 1/2")
+    gref = ref * torch.sigmoid(torch.from_numpy(z))
+    _close(oracle.gated_rmsnorm(o, z, w, 1e-6, lib=lib), gref.numpy(), tol=1e-13,
+           what="gated rmsnorm vs torch")
+    _close(oracle.gated_rmsnorm(7.0 * o, z, w, 0.0, lib=lib), oracle.gated_rmsnorm(o, z, w, 0.0, lib=lib),
+           tol=1e-13, what="scale invariance")
+
+
 ALL_PINS = [
     pin_orthonormal_write_read, pin_same_key_last_value_wins, pin_beta_zero_pure_decay,
     pin_equal_gates_are_gated_deltanet, pin_T1_closed_form, pin_T2_closed_form, pin_linearity,
     pin_column_permutation, pin_varlen_equals_separate, pin_split_resume, pin_contraction,
     pin_conv_matches_torch, pin_conv_varlen_and_cache, pin_l2norm, pin_prologue_composition,
+    pin_gate_closed_form, pin_gate_matches_torch, pin_sigmoid, pin_gated_rmsnorm,
 ]

@@ -69,6 +69,19 @@ MUTANTS = {
                        "const double inv = 1.0 / (sqrt(ss) + eps);"),
     "gdn_gate_missing": ("at * (S[(size_t)i * dv + j] - bt * kt[i] * kS[j])",
                          "(S[(size_t)i * dv + j] - bt * kt[i] * kS[j])"),
+    "gate_positive": ("g[i] = -a * sp;", "g[i] = a * sp;"),
+    "gate_dt_bias_dropped": ("const double z = x[i] + dt_bias[(size_t)h * dk + c];",
+                             "const double z = x[i];"),
+    "gate_dt_bias_per_head": ("const double z = x[i] + dt_bias[(size_t)h * dk + c];",
+                              "const double z = x[i] + dt_bias[h];"),
+    "gate_softplus_as_exp": ("log1p(exp(-z)) : log1p(exp(z));", "log1p(exp(-z)) : exp(z);"),
+    "gate_without_exp": ("const double a = exp(A_log[h]);", "const double a = A_log[h];"),
+    "sigmoid_sign": ("beta[i] = 1.0 / (1.0 + exp(-b_raw[i]));", "beta[i] = 1.0 / (1.0 + exp(b_raw[i]));"),
+    "rmsnorm_sum_not_mean": ("const double inv = 1.0 / sqrt(ss / dv + eps);",
+                             "const double inv = 1.0 / sqrt(ss + eps);"),
+    "rmsnorm_weight_dropped": ("y[i] = o[i] * inv * w[j] * (1.0", "y[i] = o[i] * inv * (1.0"),
+    "rmsnorm_gate_silu": ("y[i] = o[i] * inv * w[j] * (1.0 / (1.0 + exp(-z[i])));",
+                          "y[i] = o[i] * inv * w[j] * (z[i] / (1.0 + exp(-z[i])));"),
 }
 
 
