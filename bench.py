@@ -9,8 +9,9 @@ gates/beta/state, chunk 64): prefill tokens/s of kda_chunk_fwd with inputs resid
 HBM, timed per step with CUDA events on the launching stream, L2 flushed between steps.
 `e2e` is the same metric through the C ABI with pinned HOST buffers (host->device copy of
 the step's inputs and device->host copy of o and the final state inside the timed region).
-`rows` adds the other steps of the path measured in the same run: the conv prologue on
-the packed 64-sequence workload and the decode step on 256 x 32 states.
+`rows` adds every other config of the path measured in the same run: the conv prologue and
+the packed 64-sequence prefill with its prologue, the 262,144-token prefill, and the decode
+step (alone and with its conv step) on 256 x 32 states.
 Under torchrun (N > 1) every rank runs its own replica (weak scaling, no collective on
 the data path); time is the max over ranks.
 """
@@ -41,6 +42,15 @@ MEASURED_TRAFFIC = {
                 "57851013be10bf43df46ad41c337896a25884525ab4b3b12a15eae74d91c97b3", 357546240),
     "decode_256x32": (("recurrent_step.cu", "common.cuh"),
                       "77c4ec89d7d467c1f5a8ac71bee67eacdc51b3a44d5a73ae884d6db155449850", 1030215424),
+}
+
+
+# One description per workload, printed by both arms in config.workload.
+WL_DESC = {
+    "prefill_8k": "prefill_8k: B=1,H=32,T=8192,dk=dv=128,bf16 q/k/v/o,fp32 g/beta/state,chunk 64,"
+                  "zero h0,final state returned",
+    "long_256k": "long_256k: B=1,H=32,T=262144,dk=dv=128,bf16 q/k/v/o,fp32 g/beta/state,chunk 64,"
+                 "13/128 channels per head with exp(g)<0.5,final state returned",
 }
 
 
@@ -202,7 +212,8 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "prefill_8k: B=1,H=32,T=8192,dk=dv=128,chunk 64"},
+            "config": {"workload": WL_DESC["prefill_8k"], "parallelism": "1 GPU" if args.gpus <= 1
+                       else f"replicas x{args.gpus} (rank 0 times the oracle)"},
             "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -320,13 +331,10 @@ def run_ours(args):
                           stream=stream)
         units = T_tot
         algo_bytes = prefill_bytes(T_tot, H, dk, dv, N, h0=d["h0"] is not None)
-        wl_desc = {"prefill_8k": "prefill_8k: B=1,H=32,T=8192,dk=dv=128,bf16 q/k/v/o,fp32 g/beta/"
-                                 "state,chunk 64,zero h0,final state returned",
-                   "varlen_prologue": f"varlen_prologue: 64 packed sequences U[128,16384] "
-                                      f"(T_tot={T_tot}),H=32,dk=dv=128,bf16,h0~N(0,0.02) "
-                                      "(timed: chunked prefill on the prologue's outputs)",
-                   "long_256k": "long_256k: B=1,H=32,T=262144,dk=dv=128,bf16,skewed gates"
-                   }.get(args.workload, args.workload)
+        wl_desc = dict(WL_DESC, varlen_prologue=f"varlen_prologue: 64 packed sequences "
+                       f"U[128,16384] (T_tot={T_tot}),H=32,dk=dv=128,bf16,h0~N(0,0.02) "
+                       "(timed: chunked prefill on the prologue's outputs)").get(args.workload,
+                                                                                 args.workload)
         flops = prefill_flops(T_tot, H, dk, dv)
         dtype = "f32" if wl.io == "f32" else "bf16-io/f32"
 
@@ -398,6 +406,8 @@ def run_ours(args):
         if rate is not None:
             cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                    "sample": sample}
+            r1, s1 = oracle_one_core_rate()
+            cpu["one_core"] = {"value": r1, "unit": "tokens/s", "cores": 1, "sample": s1}
 
     if world > 1:
         dist.barrier()
@@ -417,8 +427,55 @@ def run_ours(args):
     return 0
 
 
+def _prefill_row(torch, kda, dev, flush, hbm_peak, stream, name, with_prologue=False, steps=5):
+    """One prefill workload timed as in the headline: chunk pass alone, and for the packed
+    workload also conv prologue + chunk pass (the config as stated)."""
+    from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_prefill
+    wl = WORKLOADS[name]
+    d = make_prefill(wl, dev)
+    T_tot, N, H, dk, dv = d["T_tot"], d["N"], d["H"], d["dk"], d["dv"]
+    o = torch.empty((T_tot, H, dv), dtype=torch.bfloat16, device=dev)
+    ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(kda.chunk_fwd_workspace_size(N, T_tot, H, dk, dv), dtype=torch.uint8,
+                     device=dev)
+    if with_prologue:
+        q, k, v = (torch.empty_like(d[n]) for n in ("q_raw", "k_raw", "v_raw"))
+    else:
+        q, k, v = d["q"], d["k"], d["v"]
+
+    def conv():
+        kda.conv_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["w_q"], d["w_k"], d["w_v"], q, k, v,
+                     cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], stream=stream)
+
+    def chunk():
+        kda.chunk_fwd(q, k, v, d["g"], d["beta"], 1.0, h0=d["h0"], ht=ht, o=o,
+                      cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], workspace=ws, stream=stream)
+
+    if with_prologue:
+        conv()
+    algo = prefill_bytes(T_tot, H, dk, dv, N, h0=d["h0"] is not None)
+    ms = statistics.mean(_events_time(torch, chunk, steps, 2, flush=flush, stream=stream))
+    row = {"workload": WL_DESC.get(name, f"{name}: {N} packed sequences (T_tot={T_tot}),H={H},"
+                                          f"dk=dv={dk},bf16,h0~N(0,0.02)"),
+           "chunk_ms": ms, "chunk_tokens/s": T_tot / ms * 1e3,
+           "algorithmic_bytes": algo, "chunk_frac_hbm": algo / ms / 1e6 / hbm_peak}
+    if with_prologue:
+        def both():
+            conv()
+            chunk()
+        ms2 = statistics.mean(_events_time(torch, both, steps, 2, flush=flush, stream=stream))
+        # the config's own bytes: raw q/k/v in instead of the normalised ones (same size)
+        row.update({"conv_plus_chunk_ms": ms2, "tokens/s": T_tot / ms2 * 1e3,
+                    "frac_hbm": algo / ms2 / 1e6 / hbm_peak})
+    else:
+        row.update({"tokens/s": T_tot / ms * 1e3, "frac_hbm": algo / ms / 1e6 / hbm_peak})
+    return row
+
+
 def measure_rows(torch, kda, dev, flush, hbm_peak, stream):
-    """Conv prologue (packed 64-sequence workload) and decode step (256 x 32 states)."""
+    """Every other config of the path, measured in the same run: the conv prologue and the
+    packed prefill with its prologue (64 sequences), the long-context prefill, and the decode
+    step alone and paired with its conv step (256 x 32 states)."""
     from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_decode, make_prefill
     out = {}
     wl = WORKLOADS["varlen_prologue"]
@@ -438,6 +495,12 @@ def measure_rows(torch, kda, dev, flush, hbm_peak, stream):
     del d, qo, ko, vo
     torch.cuda.empty_cache()
 
+    out["varlen_prologue"] = _prefill_row(torch, kda, dev, flush, hbm_peak, stream,
+                                          "varlen_prologue", with_prologue=True, steps=3)
+    torch.cuda.empty_cache()
+    out["long_256k"] = _prefill_row(torch, kda, dev, flush, hbm_peak, stream, "long_256k", steps=3)
+    torch.cuda.empty_cache()
+
     wl = WORKLOADS["decode_256x32"]
     steps = 16
     dd = make_decode(wl, dev, steps=steps)
@@ -455,20 +518,54 @@ def measure_rows(torch, kda, dev, flush, hbm_peak, stream):
     b = decode_bytes(wl.N, wl.H, wl.dk, wl.dv)
     ms = statistics.mean(t)
     it2 = iter(range(10 ** 9))
+    bufs = [torch.empty_like(dd[n][0]).unsqueeze(1) for n in ("q_raw", "k_raw", "v_raw")]
 
     def pair():
         s = next(it2) % steps
         x = [dd[n][s].unsqueeze(1) for n in ("q_raw", "k_raw", "v_raw")]
-        qq, kk, vv = kda.conv_fwd(*x, dd["w_q"], dd["w_k"], dd["w_v"], conv_state=cache,
+        qq, kk, vv = kda.conv_fwd(*x, dd["w_q"], dd["w_k"], dd["w_v"], *bufs, conv_state=cache,
                                   stream=stream)
         kda.recurrent_step(qq[:, 0], kk[:, 0], vv[:, 0], dd["g"][s], dd["beta"][s], state,
                            stream=stream)
-    tp = _events_time(torch, pair, 20, 3, flush=flush, stream=stream)
+    tp = statistics.mean(_events_time(torch, pair, 20, 3, flush=flush, stream=stream))
+    it3 = iter(range(10 ** 9))
+
+    def fused():
+        s = next(it3) % steps
+        kda.conv_recurrent_step(dd["q_raw"][s], dd["k_raw"][s], dd["v_raw"][s], dd["w_q"],
+                                dd["w_k"], dd["w_v"], cache, dd["g"][s], dd["beta"][s], state,
+                                stream=stream)
+    tf = statistics.mean(_events_time(torch, fused, 20, 3, flush=flush, stream=stream))
+    # the pair's own bytes: the step's, with raw q/k/v in place of the normalised ones, plus
+    # the width-3 conv cache read and written
+    cache_rw = 2 * wl.N * wl.H * (2 * wl.dk + wl.dv) * 3 * 2
     out["a5_decode_step"] = {"workload": "decode_256x32: 256 seq x 32 heads, fp32 128x128 state",
                              "ms": ms, "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm_peak,
                              "tokens/s": wl.N / ms * 1e3,
-                             "conv_plus_step_ms": statistics.mean(tp)}
+                             "conv_plus_step_ms": tp,
+                             "conv_plus_step_GB/s": (b + cache_rw) / tp / 1e6,
+                             "conv_plus_step_frac_hbm": (b + cache_rw) / tp / 1e6 / hbm_peak,
+                             "fused_conv_step_ms": tf,
+                             "fused_conv_step_GB/s": (b + cache_rw) / tf / 1e6,
+                             "fused_conv_step_frac_hbm": (b + cache_rw) / tf / 1e6 / hbm_peak}
     return out
+
+
+def oracle_one_core_rate(heads=4):
+    """The fp64 oracle on ONE host thread over a bounded sample of prefill_8k (the first
+    `heads` heads, all 8192 tokens). Returns (tokens/s normalised to H=32, sample)."""
+    import oracle
+    from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_prefill
+    d = make_prefill(WORKLOADS["prefill_8k"], "cpu")
+    f64 = lambda t: t[:, :heads].double().numpy()       # noqa: E731
+    args = [f64(d[n]) for n in ("q", "k", "v", "g", "beta")]
+    oracle.load()
+    t0 = time.perf_counter()
+    oracle.kda_fwd(*args, 1.0, None, d["cu_host"], nthreads=1)
+    el = time.perf_counter() - t0
+    rate = d["T_tot"] * heads / el / d["H"]
+    return rate, (f"heads 0..{heads - 1} of prefill_8k (8192 tokens each) on 1 host thread, "
+                  f"{el:.1f} s, scaled to H={d['H']}")
 
 
 def main():

@@ -145,6 +145,31 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          void* stream);
 
 /*
+ * kda_chunk_fwd_gated -- kda_chunk_fwd with the gate and beta formed from raw logits inside the
+ * kernel, and optionally the gated RMSNorm of the output before it is stored.
+ * (m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...": the gate is computed from
+ *  a_log_bias and dt_bias, delta is the residual times sigmoid(beta); sarnas.ru, section
+ *  "Отвергнутые решения": every norm except the QK norms is a gated RMSNorm.)
+ *
+ *     g[t, h, c]  = -exp(A_log[h]) * softplus(g_raw[t, h, c] + dt_bias[h * dk + c])
+ *     beta[t, h]  = sigmoid(beta_raw[t, h])
+ *     o'[t, h, :] = o / sqrt(mean_j o_j^2 + norm_eps) * w_norm * sigmoid(z[t, h, :])   (z != NULL)
+ *
+ *  g_raw : [T_tot, H, dk] bf16      beta_raw : [T_tot, H] bf16 (2-byte aligned)
+ *  A_log : [H] fp32                 dt_bias  : [H*dk] fp32
+ *  z     : [T_tot, H, dv] bf16 or NULL (no output norm)    w_norm : [dv] fp32 (with z)
+ *  other arguments, the workspace and the errors as for kda_chunk_fwd.
+ *  Supported: bf16 I/O, dk == dv == 128, chunk 64 (KDA_ERR_UNSUPPORTED otherwise).
+ */
+kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v, const void* g_raw,
+                               const void* beta_raw, const float* A_log, const float* dt_bias,
+                               const void* z, const float* w_norm, float norm_eps, float scale,
+                               const float* h0, float* ht, void* o, const int32_t* cu_seqlens,
+                               const int32_t* cu_seqlens_host, int B, int T, int N, int H,
+                               int dk, int dv, int chunk, kda_io_dtype io, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd without a caller workspace: the library uses a
  * device array of its own (reserved when libkda is loaded, one per device), so the call
  * allocates nothing. Arguments, layouts, results and errors are those of kda_chunk_fwd.
@@ -170,6 +195,72 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, co
 kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
                               const float* beta, float scale, float* state, void* o,
                               int N, int H, int dk, int dv, kda_io_dtype io, void* stream);
+
+/*
+ * kda_conv_recurrent_step -- one decode token per (sequence, head) from RAW q, k, v: the conv
+ * prologue and the state update in one kernel, with the conv cache advanced in place.
+ * (m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...": q/k/v pass a kernel-4 causal
+ *  conv whose cache is advanced per step, then the loop state = state*exp(gate)+delta;
+ *  sarnas.ru, section "Что именно изменилось".)
+ *
+ * Computes exactly kda_conv_fwd in decode form (T == 1 per sequence) followed by
+ * kda_recurrent_step, except that the conv outputs stay in fp32 inside the kernel instead of
+ * being rounded to the io dtype and written out (they are not returned).
+ *
+ *  q_raw, k_raw : [N, H, dk] io dtype   v_raw : [N, H, dv] io dtype (this step's raw inputs)
+ *  w_q, w_k     : [H*dk, K] fp32        w_v   : [H*dv, K] fp32 (tap K-1 = current token)
+ *  conv_state   : [N, H*(2*dk+dv), K-1] io dtype, channels q, k, v; read and overwritten with
+ *                 the last K-1 raw inputs (required: the decode history)
+ *  g    : [N, H, dk] fp32   beta : [N, H] fp32   scale: multiplies the output
+ *  state: [N, H, dk, dv] fp32, read and overwritten with the state after the token
+ *  o    : [N, H, dv] io dtype; must not overlap any input
+ *  l2_eps: the epsilon of the q, k L2 norm (x / sqrt(sum x^2 + eps))
+ *  Supported: dk, dv in {64, 128}; K == 4.
+ */
+kda_status kda_conv_recurrent_step(const void* q_raw, const void* k_raw, const void* v_raw,
+                                   const float* w_q, const float* w_k, const float* w_v,
+                                   void* conv_state, const float* g, const float* beta,
+                                   float scale, float* state, void* o, int N, int H, int dk,
+                                   int dv, int K, float l2_eps, kda_io_dtype io, void* stream);
+
+/*
+ * kda_fused_recurrent_step -- the whole decode step of a KDA layer from raw projections, in one
+ * kernel: conv prologue (cache advanced in place), gate activation, the state update, and
+ * optionally the gated RMSNorm of the output.
+ * (m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...": kernel-4 causal conv with a
+ *  cache advanced per step; the gate is computed from a_log_bias and dt_bias; delta is the
+ *  residual times sigmoid(beta). sarnas.ru, section "Отвергнутые решения": every norm except
+ *  the QK norms is a gated RMSNorm.)
+ *
+ * As kda_conv_recurrent_step, except that the gate and beta arrive as raw logits:
+ *     g[n, h, c] = -exp(A_log[h]) * softplus(g_raw[n, h, c] + dt_bias[h * dk + c]),
+ *     beta[n, h] = sigmoid(beta_raw[n, h]),
+ * and, when z is not NULL, the output is o' = o / sqrt(mean_j o_j^2 + norm_eps) * w_norm *
+ * sigmoid(z) over the dv channels of each (sequence, head).
+ *
+ *  g_raw   : [N, H, dk] io dtype        beta_raw : [N, H] io dtype (element-aligned)
+ *  A_log   : [H] fp32                   dt_bias  : [H*dk] fp32
+ *  z       : [N, H, dv] io dtype or NULL (no output norm)   w_norm : [dv] fp32 (with z)
+ *  other arguments as for kda_conv_recurrent_step.
+ *  Supported: dk, dv in {64, 128}; K == 4.
+ */
+kda_status kda_fused_recurrent_step(const void* q_raw, const void* k_raw, const void* v_raw,
+                                    const void* g_raw, const void* beta_raw, const float* w_q,
+                                    const float* w_k, const float* w_v, void* conv_state,
+                                    const float* A_log, const float* dt_bias, const void* z,
+                                    const float* w_norm, float norm_eps, float scale,
+                                    float* state, void* o, int N, int H, int dk, int dv, int K,
+                                    float l2_eps, kda_io_dtype io, void* stream);
+
+/*
+ * kda_set_wait_limit -- bound, in SM clock cycles, of every device-side wait of the prefill
+ * kernels launched after this call on any device (0 restores the default of ~2 s). A wait that
+ * runs out sets the device error word (KDA_ERR_TIMEOUT from kda_last_device_error) and the
+ * kernel ends without finishing the call; its outputs are then undefined. A diagnostic for
+ * failure handling: a short bound makes the cross-CTA hand-off waits give up. Not thread-safe
+ * against concurrent launches. KDA_ERR_INVALID_ARG for a negative bound.
+ */
+kda_status kda_set_wait_limit(int64_t cycles);
 
 /*
  * kda_last_device_error -- synchronises `stream`, then returns and clears the

@@ -6,8 +6,6 @@
 #include "kda.h"
 
 #include <stdint.h>
-#include <stdlib.h>
-#include <string.h>
 
 #define KDA_API extern "C" __attribute__((visibility("default")))
 
@@ -47,13 +45,6 @@ bool batch_geometry(const int32_t* cu, const int32_t* cu_host, int B, int T, int
 }
 
 kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
-
-// Tensor-core prefill variant: the 4-CTA cluster pipeline unless KDA_CHUNK_KERNEL=single
-// selects the one-CTA-per-(sequence, head) kernel.
-bool use_cluster_prefill() {
-    const char* e = getenv("KDA_CHUNK_KERNEL");
-    return !(e != nullptr && strcmp(e, "single") == 0);
-}
 
 // The bf16, dk = dv = 128, chunk-64 prefill runs on the cluster pipeline, which needs a workspace.
 bool cluster_prefill_path(kda_io_dtype io, int dk, int dv, int chunk) {
@@ -148,17 +139,58 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
     a.N = Nn; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk;
     a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
     if (kda::chunk_tc_supported(a)) {
-        const bool cluster = use_cluster_prefill();
-        if (cluster && (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0 ||
-                        workspace_bytes < kda::chunk_tcx_workspace_bytes()))
+        if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0 ||
+            workspace_bytes < kda::chunk_tcx_workspace_bytes())
             return KDA_ERR_WORKSPACE;
         unsigned int* err = device_error_word();
         if (err == nullptr) return KDA_ERR_CUDA;
-        cudaStream_t st = static_cast<cudaStream_t>(stream);
-        if (!cluster) return from_cuda(kda::launch_chunk_tc(a, err, st));
-        return from_cuda(kda::launch_chunk_tcx(a, workspace, workspace_bytes, err, st));
+        return from_cuda(kda::launch_chunk_tcx(a, workspace, workspace_bytes, err,
+                                               static_cast<cudaStream_t>(stream)));
     }
     return from_cuda(kda::launch_chunk_simt(a, static_cast<cudaStream_t>(stream)));
+}
+
+KDA_API kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v,
+                                       const void* g_raw, const void* beta_raw, const float* A_log,
+                                       const float* dt_bias, const void* z, const float* w_norm,
+                                       float norm_eps, float scale, const float* h0, float* ht,
+                                       void* o, const int32_t* cu_seqlens,
+                                       const int32_t* cu_seqlens_host, int B, int T, int N, int H,
+                                       int dk, int dv, int chunk, kda_io_dtype io, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+    if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
+    if (H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0) return KDA_ERR_INVALID_ARG;
+    int64_t T_tot = 0;
+    int Nn = 0;
+    if (!batch_geometry(cu_seqlens, cu_seqlens_host, B, T, N, &T_tot, &Nn)) return KDA_ERR_INVALID_ARG;
+    const void* req[] = {q, k, v, g_raw, o};
+    for (const void* p : req)
+        if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
+    if (A_log == nullptr || !aligned4(A_log) || dt_bias == nullptr || !aligned4(dt_bias))
+        return KDA_ERR_INVALID_ARG;
+    if (beta_raw == nullptr || (reinterpret_cast<uintptr_t>(beta_raw) & 1u) != 0)   // bf16 elements
+        return KDA_ERR_INVALID_ARG;
+    if (!ok_opt(h0) || !ok_opt(ht) || !ok_opt(cu_seqlens) || !ok_opt(z)) return KDA_ERR_INVALID_ARG;
+    if (z != nullptr && (w_norm == nullptr || !aligned4(w_norm) || !(norm_eps >= 0.f)))
+        return KDA_ERR_INVALID_ARG;
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = nullptr; a.beta = nullptr; a.scale = scale;
+    a.h0 = h0; a.ht = ht; a.o = o;
+    a.cu = cu_seqlens; a.cu_host = cu_seqlens_host;
+    a.T_tot = T_tot;
+    a.T_pad = cu_seqlens ? 0 : T;
+    a.N = Nn; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk;
+    a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
+    a.g_raw = g_raw; a.beta_raw = beta_raw; a.A_log = A_log; a.dt_bias = dt_bias;
+    a.z = z; a.w_norm = w_norm; a.norm_eps = norm_eps;
+    if (!kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0 ||
+        workspace_bytes < kda::chunk_tcx_workspace_bytes())
+        return KDA_ERR_WORKSPACE;
+    unsigned int* err = device_error_word();
+    if (err == nullptr) return KDA_ERR_CUDA;
+    return from_cuda(kda::launch_chunk_tcx(a, workspace, workspace_bytes, err,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 KDA_API kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
@@ -177,6 +209,67 @@ KDA_API kda_status kda_recurrent_step(const void* q, const void* k, const void* 
     a.N = N; a.H = H; a.dk = dk; a.dv = dv;
     a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
     return from_cuda(kda::launch_recurrent_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+KDA_API kda_status kda_conv_recurrent_step(const void* q_raw, const void* k_raw, const void* v_raw,
+                                           const float* w_q, const float* w_k, const float* w_v,
+                                           void* conv_state, const float* g, const float* beta,
+                                           float scale, float* state, void* o, int N, int H, int dk,
+                                           int dv, int K, float l2_eps, kda_io_dtype io,
+                                           void* stream) {
+    if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0 || K < 2 || !(l2_eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+    const void* req[] = {q_raw, k_raw, v_raw, w_q, w_k, w_v, conv_state, g, state, o};
+    for (const void* p : req)
+        if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
+    if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
+    if (K != 4 || !head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    kda::StepArgs a;
+    a.q = q_raw; a.k = k_raw; a.v = v_raw; a.g = g; a.beta = beta; a.scale = scale;
+    a.state = state; a.o = o;
+    a.N = N; a.H = H; a.dk = dk; a.dv = dv;
+    a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
+    a.w[0] = w_q; a.w[1] = w_k; a.w[2] = w_v;
+    a.conv_state = conv_state;
+    a.eps = l2_eps;
+    return from_cuda(kda::launch_recurrent_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+KDA_API kda_status kda_fused_recurrent_step(
+    const void* q_raw, const void* k_raw, const void* v_raw, const void* g_raw,
+    const void* beta_raw, const float* w_q, const float* w_k, const float* w_v, void* conv_state,
+    const float* A_log, const float* dt_bias, const void* z, const float* w_norm, float norm_eps,
+    float scale, float* state, void* o, int N, int H, int dk, int dv, int K, float l2_eps,
+    kda_io_dtype io, void* stream) {
+    if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0 || K < 2 || !(l2_eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+    const void* req[] = {q_raw, k_raw, v_raw, g_raw, w_q, w_k, w_v, conv_state, A_log, dt_bias,
+                         state, o};
+    for (const void* p : req)
+        if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
+    const uintptr_t esz = io == KDA_IO_BF16 ? 2u : 4u;     // beta_raw: element alignment
+    if (beta_raw == nullptr || (reinterpret_cast<uintptr_t>(beta_raw) & (esz - 1)) != 0)
+        return KDA_ERR_INVALID_ARG;
+    if (!ok_opt(z) || (z != nullptr && (w_norm == nullptr || !(norm_eps >= 0.f))))
+        return KDA_ERR_INVALID_ARG;
+    if (K != 4 || !head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    kda::StepArgs a;
+    a.q = q_raw; a.k = k_raw; a.v = v_raw; a.g = nullptr; a.beta = nullptr; a.scale = scale;
+    a.state = state; a.o = o;
+    a.N = N; a.H = H; a.dk = dk; a.dv = dv;
+    a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
+    a.w[0] = w_q; a.w[1] = w_k; a.w[2] = w_v;
+    a.conv_state = conv_state;
+    a.eps = l2_eps;
+    a.g_raw = g_raw; a.beta_raw = beta_raw; a.A_log = A_log; a.dt_bias = dt_bias;
+    a.z = z; a.w_norm = w_norm; a.norm_eps = norm_eps;
+    return from_cuda(kda::launch_recurrent_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+KDA_API kda_status kda_set_wait_limit(int64_t cycles) {
+    if (cycles < 0) return KDA_ERR_INVALID_ARG;
+    kda::g_chunk_wait_cycles = cycles;
+    return KDA_OK;
 }
 
 KDA_API kda_status kda_last_device_error(void* stream) {

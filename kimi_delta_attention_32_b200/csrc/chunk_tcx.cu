@@ -3,123 +3,161 @@
 //
 // The recurrence (sarnas.ru, "Яндекс открыл веса AliceAI-Foundation-80B-A3B-Base ...", section
 // "Что именно изменилось"; m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...") is
-// linear in the state, so one chunk maps the state at its start, S, to the state at its end by
-// S' = M S + N with M, N built from the chunk's inputs alone. This kernel splits along that
-// line: producers build the chunk's factors, which do not depend on S; the consumer applies
-// them. With gamma the within-chunk cumulative log-decay, gamma_C its last row and gamma_ref a
-// per-chunk reference (the chunk middle, or 0 when a half chunk decays by more than 80 in some
-// channel), per chunk:
-//   Lk = k e^{gamma - gamma_ref},  Lq = q e^{gamma - gamma_ref}
-//   R = k e^{gamma_ref - gamma},   Rh = k e^{gamma_C - gamma}              (every Rh <= |k|)
-//   [A ; P] = [Lk ; Lq] R^T   (strictly / inclusively lower triangular parts)
+// linear in the state, so one chunk maps the state at its start, S (dk x dv, row = key
+// channel), to the state at its end by S' = M S + N with M, N built from the chunk's inputs
+// alone. This kernel splits along that line: producers build the chunk's factors, which do not
+// depend on S; the consumer applies them. With gamma the within-chunk cumulative log-decay,
+// gamma_C its last row and gamma_ref a per-chunk reference (token 31, or 0 when a half chunk
+// decays by more than e^-80 in some channel), per chunk (rows = tokens):
+//   Lk = k e^{gamma - gamma_ref},  Lq = q e^{gamma - gamma_ref},  R = k e^{gamma_s - gamma}
+//   [A ; P] = [Lk ; Lq] R^T        (strictly / inclusively lower triangular parts)
 //   T' = (I + diag(beta) A)^-1 diag(beta)
-//   Yh^T = Rh^T T',  Wh^T = P T'
-// and with Sm = S^T diag(e^{gamma_ref}) (bf16), on the consumer:
-//   X = Sm Lk^T,  U = V^T - X                            (the part of V the state misses)
-//   S'^T = S^T diag(e^{gamma_C}) + U Yh                  (fp32 state, fp32 decay term)
-//   O^T  = scale (Sm Lq^T + U Wh)
+//   Yh^T = diag(e^{gamma_C - gamma_s}) R^T T',   Wh^T = P T'
+// (gamma_s = gamma_ref, or gamma_C on the exact path) and with Sm = diag(e^{gamma_ref}) S:
+//   X = Lk Sm,  U = V - X                      (the part of V the decayed state misses)
+//   S' = diag(e^{gamma_C}) S + Yh^T U          (fp32 state, fp32 decay term)
+//   O  = scale (Lq Sm + Wh^T U)
 // A chunk that fails the range test forms A and P exactly on CUDA cores (gamma_ref = 0, so
 // every factor is <= 1).
 //
-// Cluster of 4 CTAs: rank 0 is the consumer, ranks 1..3 are producers, each preparing every
-// third chunk. Per chunk the consumer runs two tensor-core groups with the A operand in tensor
-// memory: Sm [Lk^T | Lq^T] into [X | O], then, once U is written back, U [Yh | Wh] into the
-// state delta and O. It keeps the fp32 state in registers; O leaves through a TMA store. A
-// chunk's factors (57 KB) travel through L2, not DSMEM (bulk copies between SMs of a cluster
-// move ~30-60 GB/s, TMA loads from L2 150-220 GB/s): the producer bulk-stores them into a
-// six-slot ring in global memory owned by the consumer's SM (Lk and Lq straight from its own
-// A|P operand tiles, which have the consumer's layout), and the consumer TMA-loads them two
-// chunks ahead into a two-slot ring in its shared memory. Only the flags use cluster
-// barriers: "gfull" (ring slot written) in the consumer, "gfree" (ring slot read) in each
-// producer. Every wait is bounded.
+// Cluster of 4 CTAs of 17 warps: rank 0 is the consumer, ranks 1..3 are producers, each
+// preparing every third chunk. A chunk's factors (57 KB) travel through L2, not DSMEM: the
+// producer's I/O lane bulk-stores them into a ring in global memory owned by the consumer's SM
+// and announces them on a cluster barrier ("gfull"); the consumer's loader warp bulk-loads them
+// into shared memory and hands the ring slot back ("gfree").
+//
+// The consumer runs the value columns as two independent halves of 64 (state columns do not
+// interact), each on its own 8 warps with its own MMA issuer, so that one half's tensor-core
+// products overlap the other half's CUDA-core work. Per half and chunk: [X ; Lq Sm] = [Lk ; Lq]
+// Sm (M = 128 token rows, N = 64), U = V - X, then the state delta Yh^T U and the output term
+// Wh^T U; the fp32 state stays in registers (thread = key channel x 32 value columns).
+//
+// Two compile-time variants serve kda_chunk_fwd_gated. kGate: the producers form g from raw
+// gate logits, g = -exp(A_log[h]) softplus(x + dt_bias) (m.lqnn.cn/news/205170: the gate comes
+// from a_log_bias and dt_bias), in the fold, and beta = sigmoid(b) from raw logits. kNorm: the
+// consumer's output warps apply the gated RMSNorm o / sqrt(mean(o^2) + eps) * w * sigmoid(z)
+// (sarnas.ru, section "Отвергнутые решения") before the store, the two value halves exchanging
+// their per-token sums of squares through shared memory.
+//
+// Every wait is bounded (a launch parameter); a wait that gives up sets the error word, and the
+// CTA leaves its loop, waits for its own copies and products in flight, and frees its tensor
+// memory.
 #include "common.cuh"
 #include "launchers.h"
 #include "tc.cuh"
 #include "tma_host.h"
 
 namespace kda {
+
+long long g_chunk_wait_cycles = 0;   // 0: the default bound
+
 namespace {
 
 using namespace tc;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 512;          // 16 warps: latency hiding for the CUDA-core phases
+constexpr int kWarps = 17;
+constexpr int kThreads = 32 * kWarps;     // 16 compute warps + 1 I/O (producer) or loader warp
+constexpr int kCompute = 512;
+constexpr int kIoWarp = 16;
 constexpr int kProducers = 3;
 constexpr int kCluster = 1 + kProducers;
-constexpr float kHalfRange = 80.f;
-constexpr long long kWaitCycles = 4000000000LL;
-constexpr int kLd = 68;                // fp32 row stride of the 64x64 scratch (16-byte rows)
-constexpr int kLdY = 24;               // row stride of the per-warp 16x16 merge scratch
+constexpr float kHalfRange = 80.f;       // largest natural-log decay allowed per half chunk
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr long long kDefaultWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
+constexpr int kGate = 1, kNorm = 2;      // variant bits
+constexpr float kLn2 = 0.6931471805599453f;
 
-// ---- one chunk's hand-off (identical image in a global ring slot and a consumer slot) ----
-constexpr uint32_t S_LK = 0;          // [Lk | Lq]: MN-major (K = key ch, N = token), two
-constexpr uint32_t S_LQ = 16384;      //   64-wide N atoms; the producer's A|P operand image
-constexpr uint32_t S_YW = 32768;      // [Yh^T (rows key ch 0..127) | Wh^T (rows token 0..63)]:
-                                      //   K-major (K = token), one 128B-swizzled atom column
-constexpr uint32_t S_FAC = 57344;     // e^{gamma_ref}[128], e^{gamma_C}[128] (fp32)
-constexpr uint32_t kSlotBytes = 58368;
-constexpr int kRing = 6;                                // global ring slots per consumer SM
+// ---- one chunk's hand-off (identical image in a global ring slot and the consumer's slots) ----
+constexpr uint32_t S_LKQ = 0;            // [Lk ; Lq]: K-major, 2 atom columns (channels) x 128 rows
+constexpr uint32_t S_FAC = 32768;        // e^{gamma_ref}[128], e^{gamma_C}[128] (fp32)
+constexpr uint32_t kAPart = 33792;       // [Lk ; Lq | factors]
+constexpr uint32_t S_YW = kAPart;        // [Yh^T (rows key ch 0..127) ; Wh^T (rows token)]: K-major
+constexpr uint32_t kBPart = 24576;
+constexpr uint32_t kSlotBytes = kAPart + kBPart;
+constexpr int kRing = kTcxRingSlots;
+static_assert(kSlotBytes == kTcxSlotBytes, "slot size");
+static_assert(kAPart % 1024 == 0 && kBPart % 1024 == 0, "slot parts stay swizzle-atom aligned");
+
+// ---- producer shared memory ----
+constexpr uint32_t P_Q = 0;              // raw q tile [64][128] bf16 (TMA, unswizzled)
+constexpr uint32_t P_K = 16384;          // raw k tile
+constexpr uint32_t P_G = 32768;          // raw g tile [64][128] fp32
+constexpr uint32_t P_LKQ = 65536;        // [Lk ; Lq | factors]: the slot's A part image
+constexpr uint32_t P_R = P_LKQ + kAPart; // R: K-major, 2 atom columns x 64 token rows
+constexpr uint32_t P_PO = P_R + 16384;   // P': K-major, 64 token rows x 64 (A of Wh^T; its M = 128
+                                         //     padding rows read T' and give unused rows)
+constexpr uint32_t P_TP = P_PO + 8192;   // T': rows r (K), 64 columns i (N): MN-major B
+constexpr int kLd = 68;                  // fp32 row stride of the 64 x 64 inverse scratch
+constexpr int kLdY = 24;                 // row stride of the per-warp 16 x 16 products
+constexpr uint32_t P_NM = P_TP + 8192;   // N = diag(beta) A (fp32 [64][kLd])
+constexpr uint32_t P_TM = P_NM + 64 * kLd * 4;   // T (fp32 [64][kLd])
+constexpr uint32_t P_Y = P_TM + 64 * kLd * 4;    // [4][16][kLdY] fp32
+constexpr uint32_t P_ST = ((P_Y + 4 * 16 * kLdY * 4 + 1023) / 1024) * 1024;   // [Yh^T ; Wh^T] staging
+constexpr uint32_t P_GX = P_TM;          // exact path: natural-log gamma fp32 [64][128] (32 KB over
+                                         //   T, Y and the staging, all idle at that point)
+constexpr uint32_t P_MISC = P_ST + kBPart;
+static_assert(P_R % 1024 == 0 && P_PO % 1024 == 0 && P_TP % 1024 == 0 && P_ST % 1024 == 0,
+              "operand tiles are swizzle-atom aligned");
+static_assert(P_GX + 64 * 128 * 4 <= P_MISC, "exact-path scratch");
 
 // ---- consumer shared memory ----
-constexpr uint32_t C_SLOT0 = 0;                       // two slots
-constexpr uint32_t C_V = 2 * kSlotBytes;              // V ring, 3 x (two 64-ch SW128 boxes)
-constexpr uint32_t C_OST = C_V + 3 * 16384;           // O staging [64 tokens][128 ch] bf16
-constexpr uint32_t C_MISC = C_OST + 16384;
-// ---- producer shared memory ----
-constexpr uint32_t P_X = 0;           // raw q, k [64][128] bf16 (folds), then the inverse's
-                                      // scratch Nm, Tm [64][68], Y [3][16][24] (fp32)
-constexpr uint32_t P_LK = 40960;      // Lk : rows key ch, N = token (A|P A block 0, MN-major)
-constexpr uint32_t P_LQ = 57344;      // Lq : same layout (A|P A block 1)
-constexpr uint32_t P_RT = 73728;      // R  : B of A|P. Raw g (fp32, 32 KB) spans P_RT..P_RH
-constexpr uint32_t P_RH = 90112;      // Rh : K-major A of Yh^T
-constexpr uint32_t P_PO = 106496;     // P' : rows token, K = token (K-major A of Wh^T; the
-                                      //      M = 128 padding rows read T' below)
-constexpr uint32_t P_TP = 114688;     // T' : rows token, columns token (MN-major B)
-constexpr uint32_t P_AEX = 122880;    // exact path: diag(beta) A, fp32 [64][64]
-constexpr uint32_t P_GX = 139264;     // exact path: natural-log gamma, fp32 [64][128]
-constexpr uint32_t P_ST = 172032;     // hand-off staging: [Yh^T | Wh^T], then the factors
-constexpr uint32_t P_MISC = P_ST + (kSlotBytes - S_YW);
-constexpr uint32_t kMiscBytes = 2560;
-constexpr uint32_t kSmemBytes = (P_MISC > C_MISC ? P_MISC : C_MISC) + kMiscBytes + 1024;
+constexpr uint32_t C_A = 0;                        // A parts of chunks n % 2
+constexpr uint32_t C_B = 2 * kAPart;               // B parts of chunks n % 2
+constexpr uint32_t C_V = C_B + 2 * kBPart;         // V tiles [half][n % 2] (64 ch x 64 tokens, SW128)
+constexpr uint32_t C_SM = C_V + 4 * 8192;          // Sm per half: MN-major B (K = key ch, N = 64)
+constexpr uint32_t C_U = C_SM + 2 * 16384;         // U per half: MN-major B (K = token, N = 64)
+constexpr uint32_t C_OST = C_U + 2 * 8192;         // O staging per half (64 ch x 64 tokens, SW128)
+constexpr uint32_t C_MISC = C_OST + 2 * 8192;
+static_assert(C_V % 1024 == 0 && C_SM % 1024 == 0 && C_U % 1024 == 0 && C_OST % 1024 == 0,
+              "consumer tiles are swizzle-atom aligned");
+
+// ---- misc areas: mbarriers (8 bytes each) from offset 0, scalars from 256 ----
+constexpr uint32_t M_TMEM = 256;      // TMEM base address (both roles)
+constexpr uint32_t M_TMP = 260;       // unit_of scratch
+constexpr uint32_t M_SMID = 264;      // consumer: its SM id (selects the global ring)
+// producer barriers
+constexpr uint32_t M_QK_FULL = 0, M_G_FULL = 8, M_RAW_FREE = 16, M_LKQ_READY = 24, M_LKQ_FREE = 32,
+                   M_ST_READY = 40, M_ST_FREE = 48, M_AP = 56, M_YW = 64, M_GFREE = 72;
+constexpr int kBarsP = 9 + kRing;
+constexpr uint32_t M_BETA = 512;      // beta[64]
+constexpr uint32_t M_GA = 768;        // gamma at token 31, per channel (log2 units)
+constexpr uint32_t M_GC = 1280;       // gamma at token 63 (log2 units)
+constexpr uint32_t M_RHF = 1792;      // e^{gamma_C - gamma_s} per channel
+constexpr uint32_t M_WSUM = 2304;     // [16 warps][128] decay sums, then their exclusive prefix
+constexpr uint32_t M_DT = M_WSUM + 16 * 128 * 4;   // kGate: dt_bias of this head [128]
+constexpr uint32_t kMiscP = M_DT + 512;
+// consumer barriers ([X ; O] and delta per half; A, B parts per slot; V per half and slot)
+constexpr uint32_t M_XO = 0, M_DS = 16, M_AFULL = 32, M_BFULL = 48, M_AFREE = 64, M_BFREE = 80,
+                   M_VFULL = 96, M_VFREE = 128, M_GFULL = 160, M_NRM = 208;
+constexpr int kBarsC = 28;
+constexpr uint32_t M_WN = 512;        // kNorm: the norm weight [128]
+constexpr uint32_t M_SS = 1024;       // kNorm: sums of squares [chunk % 2][half][column part][64]
+constexpr uint32_t kMiscC = M_SS + 2 * 2 * 2 * 64 * 4;
+static_assert(M_GFREE + 8 * kRing <= M_TMEM && M_NRM + 16 <= M_TMEM && M_GFULL + 8 * kRing <= M_NRM &&
+              8 * kBarsC == M_NRM + 16, "barrier area");
+
+constexpr uint32_t kSmemBytes =
+    ((P_MISC + kMiscP) > (C_MISC + kMiscC) ? (P_MISC + kMiscP) : (C_MISC + kMiscC)) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(2 * kC * kLd * 4 + 4 * 16 * kLdY * 4 <= P_LK, "inverse scratch");
-static_assert(P_LQ - P_LK == S_LQ - S_LK && S_LQ + 16384 == S_YW && S_FAC - S_YW == 24576 &&
-              P_GX + kC * kD * 4 <= P_ST, "producer layout");
-static_assert(kSlotBytes % 1024 == 0 && S_FAC + 1024 <= kSlotBytes, "slot layout");
 
-// misc areas: 16 mbarriers at 8-byte steps, then scalars
-constexpr uint32_t kBars = 16;
-constexpr uint32_t M_TMEM = 128;
-constexpr uint32_t M_TMP = 132;       // unit_of scratch
-constexpr uint32_t M_SMID = 136;      // consumer: its SM id (selects the global ring)
-// consumer
-constexpr uint32_t M_BAR_S = 0;       // U Yh (the state delta) done
-constexpr uint32_t M_BAR_O = 8;       // U Wh (the output) done
-constexpr uint32_t M_LFULL = 16;      // shared slot [2] loaded from the ring
-constexpr uint32_t M_BAR_V = 32;      // V ring [3]
-constexpr uint32_t M_BAR_X = 56;      // Sm [Lk^T | Lq^T] done
-constexpr uint32_t M_GFULL = 80;      // global ring slot [kRing] written (producer arrival)
-// producer
-constexpr uint32_t M_BAR_MMA = 0;
-constexpr uint32_t M_BAR_QK = 8;
-constexpr uint32_t M_BAR_G = 16;
-constexpr uint32_t M_GFREE = 24;      // [kRing] per ring slot: its previous chunk was read (one barrier
-                                      // per slot, so arrivals for later chunks never overrun)
-constexpr uint32_t M_BETA = 192;      // beta[64]
-constexpr uint32_t M_GSUM = 448;      // [4][128] token-quarter decay sums
-static_assert(M_GSUM + 4 * 128 * 4 <= kMiscBytes && M_GFULL + 8 * kRing <= 8 * kBars &&
-              M_GFREE + 8 * kRing <= M_GFULL && M_BAR_X + 8 <= M_GFULL, "misc area");
-
-// consumer TMEM columns: [X | O] (64 + 64) for even and odd chunks, the state delta (128),
-// Sm (64 columns of bf16 pairs), U (32 columns of bf16 pairs)
-constexpr uint32_t TXO0 = 0, TXO1 = 128, TC_DS = 256, TC_SM = 384, TC_U = 448, kTmemC = 512;
-// producer TMEM columns
+// producer TMEM columns: A|P (M = 128: rows 0..63 A, 64..127 P; N = 64), Yh^T, Wh^T
 constexpr uint32_t TP_AP = 0, TP_Y = 64, TP_W = 128, kTmemP = 256;
+// consumer TMEM columns: per half h, [X ; Lq Sm] for even / odd chunks at 128 h + 64 b, the
+// state delta at 256 + 64 h
+constexpr uint32_t kTmemC = 512;
+
+// named barriers: 1 = producer compute warps, 5 = its inverse warps; 1 + h = consumer half h,
+// 3 + h = that half's output warps
+constexpr int kBarCompute = 1, kBarInverse = 5;
 
 struct Params {
-    CUtensorMap tq, tk, tg, tv, to;   // TMA maps: q, k, o [T,H,128] bf16 and g [T,H,128] f32 in
-                                      // (128, 1, 64) boxes; v in (64, 1, 64) boxes, 128B swizzle
+    CUtensorMap tq, tk, tg;           // q, k [T,H,128] bf16, g [T,H,128] f32: (128, 1, 64) boxes
+    CUtensorMap tv, to;               // v, o [T,H,128] bf16: (64, 1, 64) boxes, 128B swizzle
+    const __nv_bfloat16* q;           // the exact path reads q, k, g directly
+    const __nv_bfloat16* k;
+    const float* g;
     const float* beta;
     float scale;
     const float* h0;
@@ -131,84 +169,68 @@ struct Params {
     int T_pad;
     int N, H;
     unsigned int* err;
+    long long wait_cycles;            // bound of every wait in the main loops
+    // kGate: raw gate logits (the tg map covers them, bf16), raw beta logits, A_log [H],
+    // dt_bias [H*128]
+    const __nv_bfloat16* g_raw;
+    const __nv_bfloat16* beta_raw;
+    const float* A_log;
+    const float* dt_bias;
+    // kNorm: the output norm's gate z [T,H,128] bf16, weight [128], epsilon
+    const __nv_bfloat16* z;
+    const float* w_norm;
+    float norm_eps;
 };
+
+// softplus(x) = log(1 + e^x) = max(x, 0) + log(1 + e^-|x|), one ex2 and one lg2 on the SFU
+// (for e^-|x| below fp32 resolution next to 1 the second term is lost, an absolute error
+// below 1e-7).
+__device__ __forceinline__ float softplus_fast(float x) {
+    float l;
+    const float e = ex2_approx(-fabsf(x) * kLog2e);
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.f + e));
+    return fmaxf(x, 0.f) + l * kLn2;
+}
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
 
 __device__ __forceinline__ void st16(uint8_t* base, uint32_t off, uint4 v) {
     *reinterpret_cast<uint4*>(base + off) = v;
 }
-__device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ uint4 ld16(const uint8_t* base, uint32_t off) {
+    return *reinterpret_cast<const uint4*>(base + off);
+}
 __device__ __forceinline__ uint4 pack8(const float* v) {
     return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
                       pack_bf16(v[6], v[7]));
 }
-
-// Block-wide bounded wait for the phase of `bar` with the given parity: one thread polls (the
-// other 15 warps sleep in the block barrier instead of taking issue slots from the warp that
-// issues MMAs); false for every thread if the wait gave up.
-constexpr int kPoller = kThreads - 32;
-__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, bool cluster_scope,
-                                           unsigned int* err) {
-    int fail = 0;
-    if (threadIdx.x == kPoller) {
-        const bool ok = cluster_scope ? mbar_wait_cluster_bounded(bar, parity, kWaitCycles)
-                                      : mbar_wait_bounded(bar, parity, kWaitCycles);
-        if (!ok) {
-            atomicOr(err, kErrTimeout);
-            fail = 1;
-        }
+__device__ __forceinline__ void unpack8(uint4 w, float* v) {
+    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = unpack_bf16(a[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
     }
-    return __syncthreads_or(fail) == 0;
 }
-
-// The same with a flag of the caller's that is OR-ed into the result.
-__device__ __forceinline__ bool block_wait_or(uint64_t* bar, uint32_t parity, int fail,
-                                              unsigned int* err) {
-    if (threadIdx.x == kPoller && !mbar_wait_bounded(bar, parity, kWaitCycles)) {
-        atomicOr(err, kErrTimeout);
-        fail = 1;
-    }
-    return __syncthreads_or(fail) == 0;
+__device__ __forceinline__ uint64_t* bar_at(uint8_t* misc, uint32_t off) {
+    return reinterpret_cast<uint64_t*>(misc + off);
 }
-// Named barrier 1 over warps 1..15 (warp 0 issues the consumer's MMAs meanwhile), with an
-// OR-reduction of `pred`.
-constexpr int kGroupThreads = kThreads - 32;
-__device__ __forceinline__ int group_sync_or(int pred) {
-    int r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.s32 p, %1, 0;\n\t"
-        "barrier.cta.red.or.pred q, 1, %2, p;\n\t"
-        "selp.s32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(pred), "n"(kGroupThreads)
-        : "memory");
-    return r;
+// A bounded wait whose result every lane of the warp agrees on; a failure sets the error word.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const Params& p) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, p.wait_cycles));
+    if (!ok && (threadIdx.x & 31) == 0) atomicOr(p.err, kErrTimeout);
+    return ok;
 }
-__device__ __forceinline__ void group_sync() {
-    asm volatile("barrier.cta.sync 1, %0;" ::"n"(kGroupThreads) : "memory");
-}
-// Bounded wait of warps 1..15 for up to two barriers (the poller is in warp 15).
-__device__ __forceinline__ bool group_wait(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1,
-                                           unsigned int* err) {
-    int fail = 0;
-    if (threadIdx.x == kPoller) {
-        const bool ok = mbar_wait_bounded(b0, p0, kWaitCycles) &&
-                        (b1 == nullptr || mbar_wait_bounded(b1, p1, kWaitCycles));
-        if (!ok) {
-            atomicOr(err, kErrTimeout);
-            fail = 1;
-        }
-    }
-    return group_sync_or(fail) == 0;
-}
-// Bounded wait of warp 0 on its own (every lane observes the barrier).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned int* err) {
-    const bool ok = mbar_wait_bounded(bar, parity, kWaitCycles);
-    if (!ok && (threadIdx.x & 31) == 0) atomicOr(err, kErrTimeout);
-    return __all_sync(0xffffffffu, ok);
+// The same for one thread.
+__device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, const Params& p,
+                                         bool cluster_scope = false) {
+    const bool ok = cluster_scope ? mbar_wait_cluster(bar, parity, p.wait_cycles)
+                                  : mbar_wait(bar, parity, p.wait_cycles);
+    if (!ok) atomicOr(p.err, kErrTimeout);
+    return ok;
 }
 
-// Sequence / head of this cluster. Packed batches with at most 256 sequences are processed
+// Sequence / head of this cluster. Packed batches with at most kThreads sequences are processed
 // longest first: cluster u takes the sequence of descending-length rank u / H (ties by index).
 // Every thread of the CTA must call this (it synchronises the CTA once).
 __device__ void unit_of(const Params& p, int unit, int* s_tmp, int& n, int& h, int64_t& bos,
@@ -239,222 +261,437 @@ __device__ void unit_of(const Params& p, int unit, int* s_tmp, int& n, int& h, i
     }
 }
 
-// Exact A and P on CUDA cores for a chunk whose decay fails the range test (one warp per (r, i)
-// pair, lanes over channels): A (times beta) into an fp32 [64][64] scratch, P into its bf16
-// operand. Rare, so kept out of line, away from the common path's
-// instruction stream. Every thread of the CTA calls it.
-__device__ __noinline__ void exact_ap(uint8_t* sm, const float* s_beta, int L) {
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const __nv_bfloat16* Xq = reinterpret_cast<const __nv_bfloat16*>(sm + P_X);
-    const __nv_bfloat16* Xk = reinterpret_cast<const __nv_bfloat16*>(sm + P_X + 16384);
-    __nv_bfloat16* Pop = reinterpret_cast<__nv_bfloat16*>(sm + P_PO);
-    const float* Gx = reinterpret_cast<const float*>(sm + P_GX);
-    float* Aex = reinterpret_cast<float*>(sm + P_AEX);              // [64][64]
-    const int lane = tid & 31;
-    for (int pidx = warp; pidx < kC * (kC + 1) / 2; pidx += kThreads / 32) {
+// ============================== producer ==============================
+
+// Exact A and P on CUDA cores for a chunk whose decay fails the range test: natural-log gamma
+// from the global g (thread = channel), then one warp per (r, i) pair with lanes over channels,
+// reading q and k from global memory. Writes N = diag(beta) A into the inverse's scratch and P
+// into its operand. Rare, so kept out of line. Every compute thread calls it.
+template <int MODE>
+__device__ __noinline__ void exact_ap(const Params& p, uint8_t* sm, const float* s_beta, int h,
+                                      int64_t c0, int L) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* Gx = reinterpret_cast<float*>(sm + P_GX);
+    float* Nm = reinterpret_cast<float*>(sm + P_NM);
+    __nv_bfloat16* Po = reinterpret_cast<__nv_bfloat16*>(sm + P_PO);
+    const int64_t rs = (int64_t)p.H * kD;
+    if (tid < kD) {
+        float a = 0.f;
+        for (int t = 0; t < kC; ++t) {
+            if (t < L) {
+                if constexpr ((MODE & kGate) != 0) {
+                    const float x = __bfloat162float(p.g_raw[(c0 + t) * rs + (int64_t)h * kD + tid]) +
+                                    p.dt_bias[h * kD + tid];
+                    a -= expf(p.A_log[h]) * (x > 20.f ? x : log1pf(expf(x)));
+                } else {
+                    a += p.g[(c0 + t) * rs + (int64_t)h * kD + tid];
+                }
+            }
+            Gx[t * kD + tid] = a;
+        }
+    }
+    bar_sync(kBarCompute, kCompute);
+    for (int pidx = warp; pidx < kC * (kC + 1) / 2; pidx += kCompute / 32) {
         int r = (int)((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
         while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
         while (r * (r + 1) / 2 > pidx) --r;
         const int i = pidx - r * (r + 1) / 2;
         float a = 0.f, pp = 0.f;
-        for (int cc = lane; cc < kD && r < L; cc += 32) {
-            const float ki = bf(Xk + i * kD + cc) * expf(Gx[r * kD + cc] - Gx[i * kD + cc]);
-            a = fmaf(bf(Xk + r * kD + cc), ki, a);
-            pp = fmaf(bf(Xq + r * kD + cc), ki, pp);
+        if (r < L) {
+            const __nv_bfloat16* kr = p.k + (c0 + r) * rs + (int64_t)h * kD;
+            const __nv_bfloat16* qr = p.q + (c0 + r) * rs + (int64_t)h * kD;
+            const __nv_bfloat16* ki = p.k + (c0 + i) * rs + (int64_t)h * kD;
+            for (int cc = lane; cc < kD; cc += 32) {
+                const float kd = __bfloat162float(ki[cc]) * expf(Gx[r * kD + cc] - Gx[i * kD + cc]);
+                a = fmaf(__bfloat162float(kr[cc]), kd, a);
+                pp = fmaf(__bfloat162float(qr[cc]), kd, pp);
+            }
         }
         a = warp_sum(a);
         pp = warp_sum(pp);
         if (lane == 0) {
-            Aex[r * 64 + i] = (i < r) ? s_beta[r] * a : 0.f;
-            Aex[i * 64 + r] = (i < r) ? 0.f : Aex[i * 64 + r];
-            Pop[(kmaj_chunk(r, i >> 3, 0, 64) + (i & 7) * 2) / 2] = __float2bfloat16_rn(pp);
-            if (i < r) Pop[(kmaj_chunk(i, r >> 3, 0, 64) + (r & 7) * 2) / 2] = __float2bfloat16_rn(0.f);
+            Nm[r * kLd + i] = (i < r) ? s_beta[r] * a : 0.f;
+            if (i < r) Nm[i * kLd + r] = 0.f;
+            Po[(sw128(r, i >> 3, 0, 0) + (i & 7) * 2) / 2] = __float2bfloat16_rn(pp);
+            if (i < r) Po[(sw128(i, r >> 3, 0, 0) + (r & 7) * 2) / 2] = __float2bfloat16_rn(0.f);
         }
     }
-    __syncthreads();
 }
 
-// ============================== producer ==============================
+// T' = T diag(beta) of one 16 x 16 block held as an mma accumulator (rows R0.., cols C0..),
+// times `sign`, written as bf16 into the T' operand.
+__device__ __forceinline__ void store_tp16(uint8_t* sm, int R0, int C0, const float (*acc)[4],
+                                           float sign, const float* s_beta) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int col = C0 + 8 * nt + 2 * t;
+        const float b0 = sign * s_beta[col], b1 = sign * s_beta[col + 1];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int row = R0 + g + 8 * hh;
+            *reinterpret_cast<uint32_t*>(sm + P_TP + sw128(row, col >> 3, 0, 0) + (col & 7) * 2) =
+                pack_bf16(acc[nt][2 * hh] * b0, acc[nt][2 * hh + 1] * b1);
+        }
+    }
+}
+// scale * (a 16 x 16 mma accumulator) into an fp32 block with row stride ld.
+__device__ __forceinline__ void store_f16(float* C, int ld, const float (*acc)[4], float scale) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        C[g * ld + 8 * nt + 2 * t] = scale * acc[nt][0];
+        C[g * ld + 8 * nt + 2 * t + 1] = scale * acc[nt][1];
+        C[(g + 8) * ld + 8 * nt + 2 * t] = scale * acc[nt][2];
+        C[(g + 8) * ld + 8 * nt + 2 * t + 1] = scale * acc[nt][3];
+    }
+}
+
+// T' = (I + N)^-1 diag(beta) for the strictly lower triangular N in the scratch, by block
+// recursion on the unit lower triangular matrix (the inverse of [[A, 0], [B, C]] is
+// [[A^-1, 0], [-C^-1 B A^-1, C^-1]]): 8 x 8 diagonal blocks by substitution and their 16 x 16
+// merges in fp32 inside one warp per 16-block, then 16 -> 32 -> 64 as warp-level tensor-core
+// products (TF32 inputs, fp32 sums). Run by warps 0..3; T' is written as bf16 as each block
+// becomes final (its blocks above the diagonal stay zero from the kernel start).
+__device__ void inverse(uint8_t* sm, const float* s_beta) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* Nm = reinterpret_cast<float*>(sm + P_NM);
+    float* Tm = reinterpret_cast<float*>(sm + P_TM);
+    float* Y = reinterpret_cast<float*>(sm + P_Y);
+    float* Yw = Y + warp * 16 * kLdY;
+    const int o16 = 16 * warp;
+    // level 0: the two 8 x 8 diagonal blocks of this warp's 16-block, one column per lane
+    if (lane < 16) {
+        const int o = o16 + 8 * (lane >> 3), i = lane & 7;
+        const float* Nb = Nm + o * kLd + o;
+        float x[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            float s0 = 0.f;
+#pragma unroll
+            for (int m = 0; m < r; ++m) s0 = fmaf(Nb[r * kLd + m], x[m], s0);
+            x[r] = (r < i) ? 0.f : (r == i ? 1.f : -s0);
+            Tm[(o + r) * kLd + o + i] = x[r];
+        }
+    }
+    __syncwarp();
+    // level 1: Y = N21 T11 (8 x 8), then T21 = -T22 Y; the upper-right 8 x 8 is zero
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2) {
+        const int e = lane + 32 * e2, r = e >> 3, j = e & 7;
+        float y = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) y = fmaf(Nm[(o16 + 8 + r) * kLd + o16 + m], Tm[(o16 + m) * kLd + o16 + j], y);
+        Yw[r * 8 + j] = y;
+        Tm[(o16 + r) * kLd + o16 + 8 + j] = 0.f;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2) {
+        const int e = lane + 32 * e2, r = e >> 3, j = e & 7;
+        float t = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) t = fmaf(Tm[(o16 + 8 + r) * kLd + o16 + 8 + m], Yw[m * 8 + j], t);
+        Tm[(o16 + 8 + r) * kLd + o16 + j] = -t;
+    }
+    __syncwarp();
+    {   // T' of the diagonal 16-block: lane = (row, 8-column half)
+        const int rr = o16 + (lane >> 1), c8 = o16 + 8 * (lane & 1);
+        float w8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            w8[u] = (c8 + u <= rr) ? Tm[rr * kLd + c8 + u] * s_beta[c8 + u] : 0.f;
+        st16(sm, P_TP + sw128(rr, c8 >> 3, 0, 0), pack8(w8));
+    }
+    bar_sync(kBarInverse, 128);
+    // level 2: 16 -> 32 on warps 0, 1 (32-block = warp)
+    if (warp < 2) {
+        const int o = 32 * warp;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        warp_block_mma16(acc, Nm + (o + 16) * kLd + o, kLd, Tm + o * kLd + o, kLd);
+        store_f16(Yw, kLdY, acc, 1.f);
+        __syncwarp();
+        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        warp_block_mma16(acc2, Tm + (o + 16) * kLd + o + 16, kLd, Yw, kLdY);
+        store_f16(Tm + (o + 16) * kLd + o, kLd, acc2, -1.f);
+        store_tp16(sm, o + 16, o, acc2, -1.f, s_beta);
+    }
+    bar_sync(kBarInverse, 128);
+    // level 3: the lower-left 32 x 32 as 2 x 2 blocks of 16, warp = (a, b)
+    const int a = warp >> 1, b = warp & 1;
+    {
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int k2 = b; k2 < 2; ++k2)            // Y_ab = sum_k N21_ak T11_kb
+            warp_block_mma16(acc, Nm + (32 + 16 * a) * kLd + 16 * k2, kLd, Tm + (16 * k2) * kLd + 16 * b, kLd);
+        store_f16(Yw, kLdY, acc, 1.f);
+    }
+    bar_sync(kBarInverse, 128);
+    {
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int k2 = 0; k2 <= a; ++k2)           // T21_ab = -sum_k T22_ak Y_kb
+            warp_block_mma16(acc, Tm + (32 + 16 * a) * kLd + 32 + 16 * k2, kLd, Y + (2 * k2 + b) * 16 * kLdY, kLdY);
+        store_tp16(sm, 32 + 16 * a, 16 * b, acc, -1.f, s_beta);
+    }
+}
+
+template <int MODE>
 __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, int h,
-                         int64_t bos, int64_t eos, bool& aborted) {
-    const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
-    const uint32_t lane_sel = (uint32_t)(32 * (warp & 3)) << 16;
+                         int64_t bos, int64_t eos, bool aborted) {
+    constexpr bool kG = (MODE & kGate) != 0;
+    constexpr uint32_t kGBytes = kG ? 16384u : 32768u;   // raw logits bf16, or g fp32
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* misc = sm + P_MISC;
-    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(misc + M_BAR_MMA);
-    uint64_t* bar_qk = reinterpret_cast<uint64_t*>(misc + M_BAR_QK);
-    uint64_t* bar_g = reinterpret_cast<uint64_t*>(misc + M_BAR_G);
-    uint64_t* bar_gfree = reinterpret_cast<uint64_t*>(misc + M_GFREE);
-    float* s_beta = reinterpret_cast<float*>(misc + M_BETA);
-    float* s_gsum = reinterpret_cast<float*>(misc + M_GSUM);
     const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
     const int H = p.H;
     const int nchunks = (int)((eos - bos + kC - 1) / kC);
-    uint32_t ph_mma = 0, ph_qk = 0, ph_g = 0, ph_gfree = 0;   // ph_gfree: bit per ring slot
-
+    const int ntasks = nchunks >= prank ? (nchunks - prank) / kProducers + 1 : 0;
     const uint32_t c_misc = map_to_rank(sb + C_MISC, 0);
-    uint8_t* ring = p.ring + (size_t)ld_cluster_u32(c_misc + M_SMID) * (kRing * kSlotBytes);
-    // Chunk whose ring stores were issued but not yet announced (-1: none). Thread 0 stores a
-    // chunk as two bulk groups, [Lk | Lq] from the A|P operand tiles right after the folds and
-    // [Yh^T | Wh^T | factors] from the staging at the end of the task, and announces it in the
-    // producer's next task once only that task's first group may still be in flight: it
-    // then arrives on the consumer's "gfull" barrier of that ring slot.
-    int pending = -1;
-    auto announce = [&](bool last) {
-        if (tid == 0 && pending >= 0) {
-            if (last) bulk_wait0();
-            else asm volatile("cp.async.bulk.wait_group 1;" ::: "memory");
-            fence_proxy_async_global();
-            mbar_arrive_remote(c_misc + M_GFULL + 8u * (uint32_t)(pending % kRing));
-        }
-        pending = -1;
-    };
+    auto chunk_of = [&](int task) { return prank - 1 + kProducers * task; };
 
-    auto wait_local = [&](uint64_t* bar, uint32_t& ph) -> bool {
-        const bool ok = block_wait(bar, ph, false, p.err);
-        ph ^= 1u;
-        return ok;
-    };
-    // raw q, k tiles of a chunk (into P_X) and its g tile (into P_RT..P_RH), by TMA from one
-    // thread. Rows past the sequence are masked where they are read; rows past the whole
-    // batch arrive as zeros.
-    auto issue_qk = [&](int64_t c0) {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar_qk, 32768u);
-            tma_load_3d(sb + P_X, &p.tq, 0, h, (int)c0, bar_qk);
-            tma_load_3d(sb + P_X + 16384, &p.tk, 0, h, (int)c0, bar_qk);
+    if (warp == kIoWarp) {
+        // ---------------- I/O warp: lane 0 loads tiles, lane 1 stores and announces ----------
+        if (lane == 0 && !aborted && ntasks > 0) {
+            auto issue = [&](int task) {
+                const int c0 = (int)(bos + (int64_t)chunk_of(task) * kC);
+                mbar_arrive_expect_tx(bar_at(misc, M_QK_FULL), 32768u);
+                tma_load_3d(sb + P_Q, &p.tq, 0, h, c0, bar_at(misc, M_QK_FULL));
+                tma_load_3d(sb + P_K, &p.tk, 0, h, c0, bar_at(misc, M_QK_FULL));
+                mbar_arrive_expect_tx(bar_at(misc, M_G_FULL), kGBytes);
+                tma_load_3d(sb + P_G, &p.tg, 0, h, c0, bar_at(misc, M_G_FULL));
+            };
+            issue(0);
+            int last = 0;
+            for (int task = 0; task + 1 < ntasks; ++task) {
+                if (!wait_one(bar_at(misc, M_RAW_FREE), task & 1, p)) break;
+                issue(task + 1);
+                last = task + 1;
+            }
+            // the tiles of the last load must land before the CTA may leave
+            mbar_wait(bar_at(misc, M_QK_FULL), last & 1, kDefaultWaitCycles);
+            mbar_wait(bar_at(misc, M_G_FULL), last & 1, kDefaultWaitCycles);
+        } else if (lane == 1 && !aborted && ntasks > 0) {
+            uint8_t* ring = p.ring + (size_t)ld_cluster_u32(c_misc + M_SMID) * ((size_t)kRing * kSlotBytes);
+            uint32_t ph_gfree = 0;
+            for (int task = 0; task < ntasks; ++task) {
+                const int n = chunk_of(task);
+                const int rs = n % kRing;
+                uint8_t* slot = ring + (size_t)rs * kSlotBytes;
+                if (!wait_one(bar_at(misc, M_LKQ_READY), task & 1, p)) break;
+                if (n >= kRing) {
+                    const bool ok = wait_one(bar_at(misc, M_GFREE + 8u * rs), (ph_gfree >> rs) & 1u, p, true);
+                    ph_gfree ^= 1u << rs;
+                    if (!ok) break;
+                }
+                bulk_store(slot + S_LKQ, sb + P_LKQ, kAPart);
+                bulk_commit();
+                bulk_wait_read0();
+                mbar_arrive(bar_at(misc, M_LKQ_FREE));
+                if (!wait_one(bar_at(misc, M_ST_READY), task & 1, p)) break;
+                bulk_store(slot + S_YW, sb + P_ST, kBPart);
+                bulk_commit();
+                bulk_wait_read0();
+                mbar_arrive(bar_at(misc, M_ST_FREE));
+                bulk_wait0();
+                fence_proxy_async_global();
+                mbar_arrive_remote(c_misc + M_GFULL + 8u * (uint32_t)rs);
+            }
+            bulk_wait0();
         }
-    };
-    auto issue_g = [&](int64_t c0) {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar_g, 32768u);
-            tma_load_3d(sb + P_RT, &p.tg, 0, h, (int)c0, bar_g);
-        }
-    };
-
-    int n = prank - 1;
-    float beta_nx = 0.f;                    // beta of the next task, loaded a task ahead
-    if (n < nchunks) {
-        const int64_t c0 = bos + (int64_t)n * kC;
-        issue_qk(c0);
-        issue_g(c0);
-        if (tid < kC && c0 + tid < eos) beta_nx = p.beta[(c0 + tid) * H + h];
+        __syncwarp();
+        return;
     }
-    for (int task = 0; n < nchunks && !aborted; n += kProducers, ++task) {
+
+    // ---------------- compute warps ----------------
+    float* s_beta = reinterpret_cast<float*>(misc + M_BETA);
+    float* s_ga = reinterpret_cast<float*>(misc + M_GA);
+    float* s_gc = reinterpret_cast<float*>(misc + M_GC);
+    float* s_rhf = reinterpret_cast<float*>(misc + M_RHF);
+    float* s_wsum = reinterpret_cast<float*>(misc + M_WSUM);
+    float* facs = reinterpret_cast<float*>(sm + P_LKQ + S_FAC);
+    const int cg = lane & 15, tp = lane >> 4;           // fold: channel group of 8, token pair
+    const int t0 = 4 * warp + 2 * tp;                   // fold: tokens t0, t0 + 1
+    const int q4 = warp & 3, cb = warp >> 2;            // TMEM lane quarter, 16-column block
+    const uint32_t lane_sel = (uint32_t)(32 * q4) << 16;
+    int ap_issued = 0, ap_waited = 0, yw_issued = 0, yw_waited = 0;   // warp 0's products
+    auto beta_at = [&](int64_t t) {
+        if constexpr (kG) return sigmoid_f(__bfloat162float(p.beta_raw[t * H + h]));
+        else return p.beta[t * H + h];
+    };
+    float cneg = 0.f;                                   // kGate: -exp(A_log[h]) log2(e)
+    if constexpr (kG) {
+        cneg = -expf(p.A_log[h]) * kLog2e;
+        if (tid < kD) reinterpret_cast<float*>(misc + M_DT)[tid] = p.dt_bias[h * kD + tid];
+        bar_sync(kBarCompute, kCompute);
+    }
+    float beta_nx = 0.f;                                // beta of the next task (threads < 64)
+    if (ntasks > 0 && tid < kC) {
+        const int64_t c0 = bos + (int64_t)chunk_of(0) * kC;
+        if (c0 + tid < eos) beta_nx = beta_at(c0 + tid);
+    }
+    int fail = aborted ? 1 : 0;
+    for (int task = 0; task < ntasks && !aborted; ++task) {
+        const int n = chunk_of(task);
         const int64_t c0 = bos + (int64_t)n * kC;
         const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
-        const bool has_next = n + kProducers < nchunks;
-        const int64_t c_next = c0 + (int64_t)kProducers * kC;
-        trace_mark(prank, n, 14);
-        if (tid < kC) s_beta[tid] = beta_nx;    // (zero past the sequence)
+        const uint32_t ph = (uint32_t)task & 1u;
+        if (tid < kC) s_beta[tid] = beta_nx;
         beta_nx = 0.f;
-        if (has_next && tid < kC && c_next + tid < eos) beta_nx = p.beta[(c_next + tid) * H + h];
-        if (!wait_local(bar_qk, ph_qk) || !wait_local(bar_g, ph_g)) { aborted = true; break; }
-        // ring slot n % kRing must have been read by the consumer (chunk n - kRing)
-        if (n >= kRing) {
-            const int rs = n % kRing;
-            const bool ok = block_wait(bar_gfree + rs, (ph_gfree >> rs) & 1u, true, p.err);
-            ph_gfree ^= 1u << rs;
-            if (!ok) { aborted = true; break; }
+        if (task + 1 < ntasks && tid < kC) {
+            const int64_t c1 = bos + (int64_t)chunk_of(task + 1) * kC;
+            if (c1 + tid < eos) beta_nx = beta_at(c1 + tid);
         }
-        uint8_t* slot = ring + (size_t)(n % kRing) * kSlotBytes;
-        // the previous task's [Lk | Lq] store must have read the operand tiles before the folds
-        // below overwrite them (its second group may still be in flight)
-        if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-        trace_mark(prank, n, 0);
-
-        // ---- cumulative decay (thread: channel c = row, tokens [16*qt, 16*qt + 16)) ----
-        // kept in log2 units so that every decay factor is one ex2.approx. Lanes run over
-        // consecutive channels, so every 16-byte store below hits 8 distinct swizzled bank groups.
-        const int c = row, qt = wg;
-        const float* Xg = reinterpret_cast<const float*>(sm + P_RT);
-        const __nv_bfloat16* Xq = reinterpret_cast<const __nv_bfloat16*>(sm + P_X);
-        const __nv_bfloat16* Xk = reinterpret_cast<const __nv_bfloat16*>(sm + P_X + 16384);
-        constexpr float kLog2e = 1.4426950408889634f;
-        float gam[16];
+        bool ok = wait_warp(bar_at(misc, M_QK_FULL), ph, p) && wait_warp(bar_at(misc, M_G_FULL), ph, p) &&
+                  (task == 0 || wait_warp(bar_at(misc, M_LKQ_FREE), ph ^ 1u, p));
+        // ---- fold, part 1: decay sums (log2 units) of the token pair, then of the warp's 4 tokens ----
+        float s0[8], s1[8], xo[8];
+        if (ok) {
+            float ga[8], gb[8];                          // log-decay of tokens t0, t0 + 1 (log2)
+            if constexpr (kG) {
+                float xa[8], xb[8];
+                unpack8(ld16(sm, P_G + t0 * 256 + cg * 16), xa);
+                unpack8(ld16(sm, P_G + (t0 + 1) * 256 + cg * 16), xb);
+                const float* dt = reinterpret_cast<const float*>(misc + M_DT) + 8 * cg;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    ga[c] = cneg * softplus_fast(xa[c] + dt[c]);
+                    gb[c] = cneg * softplus_fast(xb[c] + dt[c]);
+                }
+            } else {
+                const float4* G = reinterpret_cast<const float4*>(sm + P_G);
+                const float4 a0 = G[t0 * 32 + 2 * cg], a1 = G[t0 * 32 + 2 * cg + 1];
+                const float4 b0 = G[(t0 + 1) * 32 + 2 * cg], b1 = G[(t0 + 1) * 32 + 2 * cg + 1];
+                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    ga[c] = av[c] * kLog2e;
+                    gb[c] = bv[c] * kLog2e;
+                }
+            }
+            const float m0 = t0 < L ? 1.f : 0.f, m1 = t0 + 1 < L ? 1.f : 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                s0[c] = ga[c] * m0;
+                s1[c] = fmaf(gb[c], m1, s0[c]);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) s0[c] = s1[c] = 0.f;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xo[c] = __shfl_xor_sync(0xffffffffu, s1[c], 16);
+        if (ok && tp == 0) {
+            float4* W = reinterpret_cast<float4*>(s_wsum + warp * kD + 8 * cg);
+            W[0] = make_float4(s1[0] + xo[0], s1[1] + xo[1], s1[2] + xo[2], s1[3] + xo[3]);
+            W[1] = make_float4(s1[4] + xo[4], s1[5] + xo[5], s1[6] + xo[6], s1[7] + xo[7]);
+        }
+        fail |= !ok;
+        if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+        // ---- exclusive prefix over the 16 warps, per channel; range test ----
+        int bad_c = 0;
+        if (tid < kD) {
+            float run = 0.f, ga = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < 16; ++ww) {
+                const float v = s_wsum[ww * kD + tid];
+                s_wsum[ww * kD + tid] = run;
+                run += v;
+                if (ww == 7) ga = run;
+            }
+            s_ga[tid] = ga;
+            s_gc[tid] = run;
+            const float kHalf2 = kHalfRange * kLog2e;
+            bad_c = (ga < -kHalf2) || (run - ga < -kHalf2);
+        }
+        const bool bad = bar_sync_or(kBarCompute, kCompute, bad_c) != 0;
+        // ---- fold, part 2: folded operands Lk, Lq (A of A|P and of the consumer's X | O), R ----
         {
-            float a0 = 0.f;
+            const int ac = cg >> 3, ch = cg & 7;
+            float gam0[8], gam1[8], gr[8], gs[8];
+            {
+                const float4* W = reinterpret_cast<const float4*>(s_wsum + warp * kD + 8 * cg);
+                const float4 w0 = W[0], w1 = W[1];
+                const float off[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const int r = 16 * qt + t;
-                a0 = fmaf(r < L ? Xg[r * kD + c] : 0.f, kLog2e, a0);
-                gam[t] = a0;
+                for (int c = 0; c < 8; ++c) {
+                    const float base = off[c] + (tp ? xo[c] : 0.f);
+                    gam0[c] = base + s0[c];
+                    gam1[c] = base + s1[c];
+                }
+                const float4* GA = reinterpret_cast<const float4*>(s_ga + 8 * cg);
+                const float4* GC = reinterpret_cast<const float4*>(s_gc + 8 * cg);
+                const float4 ga0 = GA[0], ga1 = GA[1], gc0 = GC[0], gc1 = GC[1];
+                const float gav[8] = {ga0.x, ga0.y, ga0.z, ga0.w, ga1.x, ga1.y, ga1.z, ga1.w};
+                const float gcv[8] = {gc0.x, gc0.y, gc0.z, gc0.w, gc1.x, gc1.y, gc1.z, gc1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    gr[c] = bad ? 0.f : gav[c];
+                    gs[c] = bad ? gcv[c] : gav[c];
+                }
             }
-            s_gsum[qt * 128 + c] = a0;
-        }
-        __syncthreads();                        // the g tile is dead from here on
-        const float q0s = s_gsum[c], q1s = s_gsum[128 + c], q2s = s_gsum[256 + c], q3s = s_gsum[384 + c];
-        const float off = qt == 0 ? 0.f : (qt == 1 ? q0s : (qt == 2 ? q0s + q1s : q0s + q1s + q2s));
 #pragma unroll
-        for (int t = 0; t < 16; ++t) gam[t] += off;
-        const float gA = q0s + q1s, gB = q2s + q3s;           // half-chunk decays (log2)
-        const float kHalf2 = kHalfRange * kLog2e;
-        const int bad = __syncthreads_or((gA < -kHalf2) || (gB < -kHalf2));
-        const float gC = gA + gB;
-        const float gr = bad ? 0.f : gA;        // reference for Lk, Lq, R (token 31, or 0)
-        const float gs = bad ? gC : gA;         // R's reference (the exact path does not use R)
-        const float rhf = ex2_approx(gC - gs);  // Rh = R * rhf
-        const float fac_r = ex2_approx(gr), fac_c = ex2_approx(gC);   // staged with Yh, Wh
-        if (bad) {                              // exact path: natural-log gamma
-            float* Gx = reinterpret_cast<float*>(sm + P_GX);
+            for (int u = 0; u < 2; ++u) {
+                const int t = t0 + u;
+                const bool valid = t < L;
+                float qv[8], kv[8];
+                unpack8(ld16(sm, P_Q + t * 256 + cg * 16), qv);
+                unpack8(ld16(sm, P_K + t * 256 + cg * 16), kv);
+                uint32_t lk[4], lq[4], rr[4];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) Gx[(16 * qt + t) * kD + c] = gam[t] * (1.f / kLog2e);
-        }
-        // ---- folded operands Lk, Lq (A of A|P, and the consumer's B of Sm [Lk^T | Lq^T]),
-        // R (B of A|P), Rh: 8 tokens per 16-byte store ----
-#pragma unroll
-        for (int q8 = 0; q8 < 2; ++q8) {
-            float lk[8], lq[8], rr[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int t = 8 * q8 + u;
-                const int r = 16 * qt + t;
-                const bool ok = r < L;
-                const float kv = ok ? __bfloat162float(Xk[r * kD + c]) : 0.f;
-                const float qv = ok ? __bfloat162float(Xq[r * kD + c]) : 0.f;
-                const float a = ex2_approx(gam[t] - gr), b = ex2_approx(gs - gam[t]);
-                lk[u] = kv * a; lq[u] = qv * a; rr[u] = kv * b;
+                for (int c = 0; c < 8; c += 2) {
+                    const float gm0 = u ? gam1[c] : gam0[c], gm1 = u ? gam1[c + 1] : gam0[c + 1];
+                    const float a0 = ex2_approx(gm0 - gr[c]), a1 = ex2_approx(gm1 - gr[c + 1]);
+                    const float b0 = ex2_approx(gs[c] - gm0), b1 = ex2_approx(gs[c + 1] - gm1);
+                    const float k0 = valid ? kv[c] : 0.f, k1 = valid ? kv[c + 1] : 0.f;
+                    const float q0 = valid ? qv[c] : 0.f, q1 = valid ? qv[c + 1] : 0.f;
+                    lk[c / 2] = pack_bf16(k0 * a0, k1 * a1);
+                    lq[c / 2] = pack_bf16(q0 * a0, q1 * a1);
+                    rr[c / 2] = pack_bf16(k0 * b0, k1 * b1);
+                }
+                st16(sm, P_LKQ + sw128(t, ch, ac, 128), make_uint4(lk[0], lk[1], lk[2], lk[3]));
+                st16(sm, P_LKQ + sw128(64 + t, ch, ac, 128), make_uint4(lq[0], lq[1], lq[2], lq[3]));
+                st16(sm, P_R + sw128(t, ch, ac, 64), make_uint4(rr[0], rr[1], rr[2], rr[3]));
             }
-            const int ch = 2 * qt + q8;         // 8-token chunk index within the 64 tokens
-            const uint32_t o16 = mnmaj_chunk(c, ch, 0, 16);
-            st16(sm, P_LK + o16, pack8(lk));
-            st16(sm, P_LQ + o16, pack8(lq));
-            st16(sm, P_RT + o16, pack8(rr));
-#pragma unroll
-            for (int u = 0; u < 8; ++u) rr[u] *= rhf;
-            st16(sm, P_RH + o16, pack8(rr));
+            if (tid < kD) {
+                const float ga = s_ga[tid], gc = s_gc[tid];
+                const float gra = bad ? 0.f : ga, gsa = bad ? gc : ga;
+                facs[tid] = ex2_approx(gra);
+                facs[kD + tid] = ex2_approx(gc);
+                s_rhf[tid] = ex2_approx(gc - gsa);
+            }
         }
         fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {                         // first group: [Lk | Lq]
-            bulk_store(slot + S_LK, sb + P_LK, S_YW - S_LK);
-            bulk_commit();
+        tc_fence_before();
+        bar_sync(kBarCompute, kCompute);
+        if (tid == 0) {
+            mbar_arrive(bar_at(misc, M_RAW_FREE));     // the raw tiles are dead
+            mbar_arrive(bar_at(misc, M_LKQ_READY));    // [Lk ; Lq | factors] may leave
         }
-        trace_mark(prank, n, 1);
-
-        float* Nm = reinterpret_cast<float*>(sm + P_X);
-        if (!bad) {
-            if (warp == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 64, true, true);
-                const uint64_t a0 = make_desc(sb + P_LK, P_LQ - P_LK, 1024);
-                const uint64_t b0 = make_desc(sb + P_RT, 16384, 1024);
-                if (elect_one()) {
-#pragma unroll
-                    for (int s = 0; s < 8; ++s)
-                        mma_bf16(tm + TP_AP, desc_add(a0, s * 2048), desc_add(b0, s * 2048), id, s > 0);
-                    mma_commit(bar_mma);
-                }
-                __syncwarp();
-            }
-            if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
-            trace_mark(prank, n, 2);
+        if (warp == 0) {                               // [A ; P] = [Lk ; Lq] R^T
             tc_fence_after();
+            if (elect_one()) {
+                const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tm + TP_AP, make_desc(sb + P_LKQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                             make_desc(sb + P_R + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), id, s > 0);
+                mma_commit(bar_at(misc, M_AP));
+            }
+            __syncwarp();
+            ++ap_issued;
+        }
+        // ---- extraction: N = diag(beta) A (strictly lower, fp32), P' (inclusive, bf16) ----
+        ok = wait_warp(bar_at(misc, M_AP), ph, p);
+        if (warp == 0 && ok) ++ap_waited;
+        tc_fence_after();
+        if (ok && !bad) {
             float val[16];
-            tmem_ld16(tm + lane_sel + TP_AP + 16 * wg, val);
-            const int i0 = 16 * wg;
-            if (row < 64) {
-                const int r = row;
+            tmem_ld16(tm + lane_sel + TP_AP + 16 * cb, val);
+            const int i0 = 16 * cb;
+            if (q4 < 2) {
+                const int r = 32 * q4 + lane;
                 const float br = s_beta[r];
+                float* Nr = reinterpret_cast<float*>(sm + P_NM) + r * kLd + i0;
 #pragma unroll
                 for (int i4 = 0; i4 < 4; ++i4) {
                     float4 w;
@@ -462,471 +699,428 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                     w.y = (i0 + 4 * i4 + 1 < r) ? br * val[4 * i4 + 1] : 0.f;
                     w.z = (i0 + 4 * i4 + 2 < r) ? br * val[4 * i4 + 2] : 0.f;
                     w.w = (i0 + 4 * i4 + 3 < r) ? br * val[4 * i4 + 3] : 0.f;
-                    *reinterpret_cast<float4*>(Nm + r * kLd + i0 + 4 * i4) = w;
+                    reinterpret_cast<float4*>(Nr)[i4] = w;
                 }
             } else {
-                const int r = row - 64;
+                const int r = 32 * (q4 - 2) + lane;
 #pragma unroll
-                for (int qq = 0; qq < 2; ++qq) {
+                for (int k8 = 0; k8 < 2; ++k8) {
                     float pv[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) pv[u] = (i0 + 8 * qq + u <= r) ? val[8 * qq + u] : 0.f;
-                    st16(sm, P_PO + kmaj_chunk(r, (i0 >> 3) + qq, 0, 64), pack8(pv));
+                    for (int u = 0; u < 8; ++u) pv[u] = (i0 + 8 * k8 + u <= r) ? val[8 * k8 + u] : 0.f;
+                    st16(sm, P_PO + sw128(r, 2 * cb + k8, 0, 0), pack8(pv));
                 }
             }
-        } else {
-            exact_ap(sm, s_beta, L);
-            const float* Aex = reinterpret_cast<const float*>(sm + P_AEX);
-            // the raw tiles are dead: move diag(beta) A into the inverse's scratch
-            for (int e = tid; e < kC * kC; e += kThreads) Nm[(e >> 6) * kLd + (e & 63)] = Aex[e];
         }
-        __syncthreads();
-        trace_mark(prank, n, 3);
-
-        // ---- T' = (I + N)^-1 diag(beta) in fp32, N = diag(beta) A ----
-        // Block recursion on the unit lower triangular matrix: the inverse of [[A, 0], [B, C]]
-        // is [[A^-1, 0], [-C^-1 B A^-1, C^-1]]. 8x8 diagonal blocks by column substitution,
-        // then 8 -> 16 on CUDA cores (fp32), 16 -> 32 -> 64 as warp-level tensor-core products
-        // (TF32 inputs, fp32 sums). T' is rounded to bf16 afterwards.
-        {
-            float* Tm = Nm + kC * kLd;
-            float* Y = Tm + kC * kLd;                     // [4][16][kLdY] products / [4][8][8]
-            if (tid < 64) {                               // level 0: block b, column i
-                const int b = tid >> 3, i = tid & 7;
-                const float* Nb = Nm + (8 * b) * kLd + 8 * b;
-                float x[8];
-#pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    float s0 = 0.f;
-#pragma unroll
-                    for (int m = 0; m < r; ++m) s0 = fmaf(Nb[r * kLd + m], x[m], s0);
-                    x[r] = (r < i) ? 0.f : (r == i ? 1.f : -s0);
-                    Tm[(8 * b + r) * kLd + 8 * b + i] = x[r];
-                }
-            }
-            __syncthreads();
-            trace_mark(prank, n, 4);
-            if (tid < 256) {                              // level 1: 16-block blk, element (r, j)
-                const int blk = tid >> 6, r = (tid >> 3) & 7, j = tid & 7, o = 16 * blk;
-                float y = 0.f;
-#pragma unroll
-                for (int m = 0; m < 8; ++m) y = fmaf(Nm[(o + 8 + r) * kLd + o + m], Tm[(o + m) * kLd + o + j], y);
-                Y[blk * 64 + r * 8 + j] = y;
-                Tm[(o + r) * kLd + o + 8 + j] = 0.f;      // upper-right 8x8 of the 16-block
-            }
-            __syncthreads();
-            if (tid < 256) {
-                const int blk = tid >> 6, r = (tid >> 3) & 7, j = tid & 7, o = 16 * blk;
-                float t = 0.f;
-#pragma unroll
-                for (int m = 0; m < 8; ++m) t = fmaf(Tm[(o + 8 + r) * kLd + o + 8 + m], Y[blk * 64 + m * 8 + j], t);
-                Tm[(o + 8 + r) * kLd + o + j] = -t;
-            }
-            __syncthreads();
-            // level 2: 32-blocks g = 0, 1 on warps 0, 1; the other warps zero their upper-right 16x16
-            if (warp < 2) {
-                const int o = 32 * warp;
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                warp_block_mma16(acc, Nm + (o + 16) * kLd + o, kLd, Tm + o * kLd + o, kLd);
-                warp_block_store16(Y + warp * 16 * kLdY, kLdY, acc, 1.f);
-            } else {
-                for (int e = tid - 64; e < 512; e += kThreads - 64) {
-                    const int g2 = e >> 8, r = (e >> 4) & 15, j = e & 15;
-                    Tm[(32 * g2 + r) * kLd + 32 * g2 + 16 + j] = 0.f;
-                }
-            }
-            __syncthreads();
-            if (warp < 2) {
-                const int o = 32 * warp;
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                warp_block_mma16(acc, Tm + (o + 16) * kLd + o + 16, kLd, Y + warp * 16 * kLdY, kLdY);
-                warp_block_store16(Tm + (o + 16) * kLd + o, kLd, acc, -1.f);
-            }
-            __syncthreads();
-            // level 3: the lower-left 32x32 as 2x2 blocks of 16, warp w = (a, b)
-            if (warp < 4) {
-                const int a = warp >> 1, b = warp & 1;
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                for (int k2 = b; k2 < 2; ++k2)            // Y_ab = sum_k N21_ak T11_kb
-                    warp_block_mma16(acc, Nm + (32 + 16 * a) * kLd + 16 * k2, kLd, Tm + (16 * k2) * kLd + 16 * b, kLd);
-                warp_block_store16(Y + warp * 16 * kLdY, kLdY, acc, 1.f);
-            }
-            __syncthreads();
-            if (warp < 4) {
-                const int a = warp >> 1, b = warp & 1;
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                for (int k2 = 0; k2 <= a; ++k2)           // T21_ab = -sum_k T22_ak Y_kb
-                    warp_block_mma16(acc, Tm + (32 + 16 * a) * kLd + 32 + 16 * k2, kLd, Y + (2 * k2 + b) * 16 * kLdY, kLdY);
-                warp_block_store16(Tm + (32 + 16 * a) * kLd + 16 * b, kLd, acc, -1.f);
-            }
-            __syncthreads();
-            trace_mark(prank, n, 5);
-            // T' = T diag(beta): 8 consecutive columns per item from two 16-byte reads
-            for (int e = tid; e < kC * 8; e += kThreads) {
-                const int r = e >> 3, q8 = e & 7;
-                const float4 t0 = *reinterpret_cast<const float4*>(Tm + r * kLd + 8 * q8);
-                const float4 t1 = *reinterpret_cast<const float4*>(Tm + r * kLd + 8 * q8 + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(s_beta + 8 * q8);
-                const float4 b1 = *reinterpret_cast<const float4*>(s_beta + 8 * q8 + 4);
-                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                float w8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = 8 * q8 + u;
-                    w8[u] = (i < r) ? tv[u] * bv[u] : (i == r ? bv[u] : 0.f);
-                }
-                st16(sm, P_TP + kmaj_chunk(r, q8, 0, 64), pack8(w8));
-            }
+        fail |= !ok;
+        if (bad) {
+            // the exact path uses the staging as scratch: the previous chunk must have left it
+            ok = task == 0 || wait_warp(bar_at(misc, M_ST_FREE), ph ^ 1u, p);
+            fail |= !ok;
+            if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+            exact_ap<MODE>(p, sm, s_beta, h, c0, L);
         }
         fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (has_next) issue_qk(c_next);         // the inverse's scratch is dead
-        announce(false);                        // the previous chunk, stored a task ago
-        trace_mark(prank, n, 6);
-
-        // ---- Yh^T = Rh^T T' (M = key ch) and Wh^T = P' T' (M = token, 64 rows of 128) ----
+        if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+        // ---- T' = (I + N)^-1 diag(beta) on warps 0..3 ----
+        if (warp < 4) inverse(sm, s_beta);
+        fence_async_smem();
+        bar_sync(kBarCompute, kCompute);
+        // ---- Yh^T = R^T T' (M = key ch) and Wh^T = P' T' (M = token) ----
         if (warp == 0) {
             tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, false, true);
-            const uint64_t aY = make_desc(sb + P_RH, 16, 1024);
-            const uint64_t aW = make_desc(sb + P_PO, 16, 1024);
-            const uint64_t bT = make_desc(sb + P_TP, 8192, 1024);
             if (elect_one()) {
+                const uint32_t idY = idesc_bf16(128, 64, true, true);
+                const uint32_t idW = idesc_bf16(128, 64, false, true);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tm + TP_Y, desc_add(aY, s * 32), desc_add(bT, s * 2048), id, s > 0);
+                    mma_bf16(tm + TP_Y, make_desc(sb + P_R + s * 2048, 8192, 1024),
+                             make_desc(sb + P_TP + s * 2048, 8192, 1024), idY, s > 0);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tm + TP_W, desc_add(aW, s * 32), desc_add(bT, s * 2048), id, s > 0);
-                mma_commit(bar_mma);
+                    mma_bf16(tm + TP_W, make_desc(sb + P_PO + s * 32, 16, 1024),
+                             make_desc(sb + P_TP + s * 2048, 8192, 1024), idW, s > 0);
+                mma_commit(bar_at(misc, M_YW));
             }
             __syncwarp();
+            ++yw_issued;
         }
-        // the staging is free once the previous chunk's second group has read it
-        if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-        if (!wait_local(bar_mma, ph_mma)) { aborted = true; break; }
-        trace_mark(prank, n, 7);
-        if (has_next) issue_g(c_next);          // R and Rh are dead
+        ok = wait_warp(bar_at(misc, M_YW), ph, p);
+        if (warp == 0 && ok) ++yw_waited;
+        if (ok && !bad && task > 0) ok = wait_warp(bar_at(misc, M_ST_FREE), ph ^ 1u, p);
         tc_fence_after();
-        {
+        // ---- staging: Yh^T rows scaled by e^{gamma_C - gamma_s}, then Wh^T, as bf16 ----
+        if (ok) {
             float val[16];
-            tmem_ld16(tm + lane_sel + TP_Y + 16 * wg, val);
+            const int c = 32 * q4 + lane;
+            tmem_ld16(tm + lane_sel + TP_Y + 16 * cb, val);
+            const float f = s_rhf[c];
 #pragma unroll
-            for (int qq = 0; qq < 2; ++qq)
-                st16(sm, P_ST + kmaj_chunk(row, 2 * wg + qq, 0, 0), pack8(val + 8 * qq));
-            if ((warp & 3) < 2) {               // lanes 0..63 hold Wh^T
-                tmem_ld16(tm + lane_sel + TP_W + 16 * wg, val);
-#pragma unroll
-                for (int qq = 0; qq < 2; ++qq)
-                    st16(sm, P_ST + kmaj_chunk(128 + row, 2 * wg + qq, 0, 0), pack8(val + 8 * qq));
-            }
-            if (qt == 0) {
-                float* fs = reinterpret_cast<float*>(sm + P_ST + (S_FAC - S_YW));
-                fs[c] = fac_r;
-                fs[128 + c] = fac_c;
+            for (int u = 0; u < 16; ++u) val[u] *= f;
+            st16(sm, P_ST + sw128(c, 2 * cb, 0, 0), pack8(val));
+            st16(sm, P_ST + sw128(c, 2 * cb + 1, 0, 0), pack8(val + 8));
+            if (q4 < 2) {
+                tmem_ld16(tm + lane_sel + TP_W + 16 * cb, val);
+                st16(sm, P_ST + sw128(128 + c, 2 * cb, 0, 0), pack8(val));
+                st16(sm, P_ST + sw128(128 + c, 2 * cb + 1, 0, 0), pack8(val + 8));
             }
         }
+        fail |= !ok;
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {                         // second group: [Yh^T | Wh^T | factors]
-            bulk_store(slot + S_YW, sb + P_ST, kSlotBytes - S_YW);
-            bulk_commit();
-        }
-        pending = n;
-        trace_mark(prank, n, 8);
+        if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+        if (tid == 0) mbar_arrive(bar_at(misc, M_ST_READY));
     }
-    if (!aborted) announce(true);
-    if (tid == 0) bulk_wait0();
+    // products still in flight must finish before the tensor memory is freed (the last commit
+    // on each barrier covers every earlier product)
+    if (warp == 0) {
+        if (ap_issued > ap_waited)
+            mbar_wait(bar_at(misc, M_AP), (uint32_t)(ap_issued - 1) & 1u, kDefaultWaitCycles);
+        if (yw_issued > yw_waited)
+            mbar_wait(bar_at(misc, M_YW), (uint32_t)(yw_issued - 1) & 1u, kDefaultWaitCycles);
+    }
 }
 
 // ============================== consumer ==============================
+
+template <int MODE>
 __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, int h,
-                         int64_t bos, int64_t eos, bool& aborted) {
-    const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, j = tid & 127;
-    const uint32_t lane_sel = (uint32_t)(32 * (warp & 3)) << 16;
+                         int64_t bos, int64_t eos, bool aborted) {
+    constexpr bool kN = (MODE & kNorm) != 0;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* misc = sm + C_MISC;
-    uint64_t* bar_x = reinterpret_cast<uint64_t*>(misc + M_BAR_X);
-    uint64_t* bar_s = reinterpret_cast<uint64_t*>(misc + M_BAR_S);
-    uint64_t* bar_o = reinterpret_cast<uint64_t*>(misc + M_BAR_O);
-    uint64_t* bar_lfull = reinterpret_cast<uint64_t*>(misc + M_LFULL);
-    uint64_t* bar_gfull = reinterpret_cast<uint64_t*>(misc + M_GFULL);
-    uint64_t* bar_v = reinterpret_cast<uint64_t*>(misc + M_BAR_V);
     const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
     const int H = p.H;
     const int nchunks = (int)((eos - bos + kC - 1) / kC);
-    uint32_t ph_x = 0, ph_s = 0, ph_lfull = 0, ph_gfull = 0, ph_v = 0;   // bit i: barrier i
-    const uint8_t* ring = p.ring + (size_t)smid() * (kRing * kSlotBytes);
-    const int64_t sbase = ((int64_t)n_seq * H + h) * kD * kD;
 
-    float sreg[32];                     // S[32*wg + cc][j]
-#pragma unroll
-    for (int cc = 0; cc < 32; ++cc)
-        sreg[cc] = p.h0 ? p.h0[sbase + (int64_t)(32 * wg + cc) * kD + j] : 0.f;
-
-    // V tile of chunk nn into ring entry nn % 3 by TMA: two (64 channels x 64 tokens) boxes,
-    // 128B-swizzled. Rows past the sequence do not matter (the matching rows of Lk, Yh and Wh
-    // are zero). Thread kLoader (warp 2) issues every V and ring load, beside warp 0's MMA issue.
-    constexpr int kLoader = 64;
-    auto issue_v = [&](int nn) {
-        if (tid == kLoader) {
-            const int e = nn % 3;
-            const uint32_t base = sb + C_V + (uint32_t)e * 16384;
-            const int c0 = (int)(bos + (int64_t)nn * kC);
-            mbar_arrive_expect_tx(bar_v + e, 16384u);
-            tma_load_3d(base, &p.tv, 0, h, c0, bar_v + e);
-            tma_load_3d(base + 8192, &p.tv, 64, h, c0, bar_v + e);
-        }
-    };
-    // Factors of chunk nn from its global ring slot into shared slot nn % 2 (the shared slot
-    // must be free): waits for the producer's announcement, then one bulk load.
-    auto issue_load = [&](int nn) -> bool {
-        bool ok = true;
-        if (tid == kLoader) {
-            const int rs = nn % kRing;
-            ok = mbar_wait_cluster_bounded(bar_gfull + rs, (ph_gfull >> rs) & 1u, kWaitCycles);
-            ph_gfull ^= 1u << rs;
-            if (ok) {
+    if (warp == kIoWarp) {
+        // ---------------- loader: V tiles, each chunk's factors, ring slots back ----------------
+        if (lane == 0 && !aborted && nchunks > 0) {
+            const uint8_t* ring = p.ring + (size_t)smid() * ((size_t)kRing * kSlotBytes);
+            uint32_t ph_gfull = 0;
+            int loaded = 0;          // chunks whose A and B loads were issued
+            int v_issued = 0;        // chunks whose V tiles were issued
+            bool ok = true;
+            // the ring slot of chunk mm goes back to the producer that writes chunk mm + kRing
+            // once both of its loads have landed
+            auto release = [&](int mm) -> bool {
+                const uint32_t par = (uint32_t)(mm >> 1) & 1u;
+                if (!wait_one(bar_at(misc, M_AFULL + 8 * (mm & 1)), par, p) ||
+                    !wait_one(bar_at(misc, M_BFULL + 8 * (mm & 1)), par, p))
+                    return false;
+                if (mm + kRing < nchunks)
+                    mbar_arrive_remote(map_to_rank(sb + P_MISC + M_GFREE + 8u * (uint32_t)(mm % kRing),
+                                                   1 + (mm + kRing) % kProducers));
+                return true;
+            };
+            for (int m = 0; m < nchunks && ok; ++m) {
+                const int sl = m & 1;
+                const uint32_t pfree = (uint32_t)((m - 2) >> 1) & 1u;
+                const int c0 = (int)(bos + (int64_t)m * kC);
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint64_t* vf = bar_at(misc, M_VFULL + 8 * (2 * hh + sl));
+                    if (m >= 2 && !(ok = wait_one(bar_at(misc, M_VFREE + 8 * (2 * hh + sl)), pfree, p))) break;
+                    mbar_arrive_expect_tx(vf, 8192u);
+                    tma_load_3d(sb + C_V + (uint32_t)(2 * hh + sl) * 8192, &p.tv, 64 * hh, h, c0, vf);
+                    v_issued = m + 1;
+                }
+                if (!ok) break;
+                const int rs = m % kRing;
+                ok = wait_one(bar_at(misc, M_GFULL + 8 * rs), (ph_gfull >> rs) & 1u, p, true);
+                ph_gfull ^= 1u << rs;
+                if (!ok) break;
                 fence_proxy_async_global();
-                uint64_t* bl = bar_lfull + (nn & 1);
-                const uint32_t dst = sb + C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
-                mbar_arrive_expect_tx(bl, kSlotBytes);
-                bulk_load(dst, ring + (size_t)rs * kSlotBytes, kSlotBytes, bl);
-            } else {
-                atomicOr(p.err, kErrTimeout);
+                const uint8_t* slot = ring + (size_t)rs * kSlotBytes;
+                if (m >= 2 && !(ok = wait_one(bar_at(misc, M_AFREE + 8 * sl), pfree, p))) break;
+                mbar_arrive_expect_tx(bar_at(misc, M_AFULL + 8 * sl), kAPart);
+                bulk_load(sb + C_A + (uint32_t)sl * kAPart, slot + S_LKQ, kAPart, bar_at(misc, M_AFULL + 8 * sl));
+                if (m >= 2 && !(ok = wait_one(bar_at(misc, M_BFREE + 8 * sl), pfree, p))) {
+                    // the A load of this chunk is in flight: it must land before the CTA leaves
+                    mbar_wait(bar_at(misc, M_AFULL + 8 * sl), (uint32_t)(m >> 1) & 1u, kDefaultWaitCycles);
+                    break;
+                }
+                mbar_arrive_expect_tx(bar_at(misc, M_BFULL + 8 * sl), kBPart);
+                bulk_load(sb + C_B + (uint32_t)sl * kBPart, slot + S_YW, kBPart, bar_at(misc, M_BFULL + 8 * sl));
+                loaded = m + 1;
+                if (m >= 1) ok = release(m - 1);
             }
-        }
-        return ok;
-    };
-    // Factors and V tile of chunk nn both in (one polling thread, one block barrier); then
-    // its ring slot may take chunk nn + kRing.
-    auto wait_next = [&](int nn) -> bool {
-        const int sl = nn & 1, e = nn % 3;
-        int fail = 0;
-        if (tid == kPoller) {
-            const bool ok = mbar_wait_bounded(bar_lfull + sl, (ph_lfull >> sl) & 1u, kWaitCycles) &&
-                            mbar_wait_bounded(bar_v + e, (ph_v >> e) & 1u, kWaitCycles);
-            if (!ok) {
-                atomicOr(p.err, kErrTimeout);
-                fail = 1;
+            if (ok && loaded == nchunks) release(nchunks - 1);
+            // every copy issued into this CTA's shared memory must land before it leaves
+            for (int mm = (loaded > 2 ? loaded - 2 : 0); mm < loaded; ++mm) {
+                const uint32_t par = (uint32_t)(mm >> 1) & 1u;
+                mbar_wait(bar_at(misc, M_AFULL + 8 * (mm & 1)), par, kDefaultWaitCycles);
+                mbar_wait(bar_at(misc, M_BFULL + 8 * (mm & 1)), par, kDefaultWaitCycles);
             }
+            for (int mm = (v_issued > 2 ? v_issued - 2 : 0); mm < v_issued; ++mm)
+                for (int hh = 0; hh < 2; ++hh)
+                    mbar_wait(bar_at(misc, M_VFULL + 8 * (2 * hh + (mm & 1))), (uint32_t)(mm >> 1) & 1u,
+                              kDefaultWaitCycles);
         }
-        ph_lfull ^= 1u << sl;
-        ph_v ^= 1u << e;
-        if (__syncthreads_or(fail)) return false;
-        if (tid == 0 && nn + kRing < nchunks)
-            mbar_arrive_remote_relaxed(map_to_rank(sb + P_MISC + M_GFREE + 8u * (uint32_t)(nn % kRing),
-                                                   1 + (nn + kRing) % kProducers));
-        return true;
+        __syncwarp();
+        return;
+    }
+
+    // ---------------- the two halves of the value columns ----------------
+    const int half = warp >> 3, lw = warp & 7, q = lw & 3, cp = lw >> 2;
+    const int tid_h = tid & 255;
+    const uint32_t lane_sel = (uint32_t)(32 * q) << 16;
+    const int bar_half = 1 + half, bar_out = 3 + half;
+    const uint32_t t_xo = tm + 128 * half, t_ds = tm + 256 + 64 * half;
+    uint64_t* bar_xo = bar_at(misc, M_XO + 8 * half);
+    uint64_t* bar_ds = bar_at(misc, M_DS + 8 * half);
+    const uint32_t sm_h = C_SM + 16384u * half, u_h = C_U + 8192u * half, ost_h = C_OST + 8192u * half;
+    const int i_row = 32 * q + lane;                 // state row (key channel) of this thread
+    const int jg0 = 64 * half + 32 * cp;             // its first value column
+    const int64_t sbase = ((int64_t)n_seq * H + h) * kD * kD;
+    const bool issuer = (lw == 0);
+    int xo_issued = 0, xo_waited = 0, ds_issued = 0, ds_waited = 0;   // issuer's bookkeeping
+
+    float S[32];
+#pragma unroll
+    for (int c4 = 0; c4 < 8; ++c4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p.h0) v = reinterpret_cast<const float4*>(p.h0 + sbase + (int64_t)i_row * kD + jg0)[c4];
+        S[4 * c4] = v.x; S[4 * c4 + 1] = v.y; S[4 * c4 + 2] = v.z; S[4 * c4 + 3] = v.w;
+    }
+    auto fac = [&](int nn) {
+        return reinterpret_cast<const float*>(sm + C_A + (uint32_t)(nn & 1) * kAPart + S_FAC);
     };
-    // [X | O](nn) = Sm(nn) [Lk^T | Lq^T] (one converged warp; A operand Sm in tensor memory)
+    // Sm(nn) = diag(e^{gamma_ref(nn)}) S as bf16, MN-major (K = key channel, N = value column)
+    auto write_sm = [&](int nn) {
+        const float e = fac(nn)[i_row];
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+            float w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) w[u] = S[8 * k8 + u] * e;
+            st16(sm, sm_h + sw128(i_row, 4 * cp + k8, 0, 0), pack8(w));
+        }
+    };
     auto issue_xo = [&](int nn) {
-        const uint32_t so = C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
         tc_fence_after();
-        const uint32_t id = idesc_bf16(128, 128, false, true);
-        const uint64_t b0 = make_desc(sb + so + S_LK, S_LQ - S_LK, 1024);
-        const uint32_t d = tm + ((nn & 1) ? TXO1 : TXO0);
         if (elect_one()) {
+            const uint32_t id = idesc_bf16(128, 64, false, true);
+            const uint32_t a = sb + C_A + (uint32_t)(nn & 1) * kAPart + S_LKQ;
 #pragma unroll
-            for (int s = 0; s < 8; ++s) mma_bf16_ts(d, tm + TC_SM + 8 * s, desc_add(b0, s * 2048), id, s > 0);
-            mma_commit(bar_x);
+            for (int s = 0; s < 8; ++s)
+                mma_bf16(t_xo + 64 * (nn & 1), make_desc(a + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                         make_desc(sb + sm_h + s * 2048, 8192, 1024), id, s > 0);
+            mma_commit(bar_xo);
         }
         __syncwarp();
+        ++xo_issued;
     };
-    // state delta U Yh (commit S), then O(nn) += U Wh (commit O); A operand U in tensor memory
-    auto issue_u = [&](int nn) {
-        const uint32_t so = C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes;
+    // O of chunk nn (rows 64..127 of its [X ; O] accumulator) by the output warps: bf16 through
+    // the swizzled staging and one TMA store, or straight to global for a ragged last chunk
+    // (rows past the sequence belong to the next one). The named barriers run whether or not
+    // `ok` holds, so the four warps always meet.
+    auto epilogue_o = [&](int nn, bool ok) {
+        const int64_t c0 = bos + (int64_t)nn * kC;
+        const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
+        const int t = 32 * (q - 2) + lane;
+        const uint32_t src = t_xo + 64 * (nn & 1) + lane_sel + 32 * cp;
+        float inv = 0.f;                            // kNorm: 1 / rms of token t over 128 columns
+        uint4 zr[4];
+        if constexpr (kN) {
+            // the output's gate for this thread's 32 columns (loads in flight during the sums)
+            const uint4* zsrc = reinterpret_cast<const uint4*>(
+                p.z + ((c0 + (t < L ? t : 0)) * H + h) * kD + jg0);
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) zr[k8] = ok ? zsrc[k8] : make_uint4(0, 0, 0, 0);
+            float ss = 0.f;
+            if (ok) {
+#pragma unroll
+                for (int hx = 0; hx < 2; ++hx) {
+                    float ov[16];
+                    tmem_ld16(src + 16 * hx, ov);
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) ss = fmaf(ov[u], ov[u], ss);
+                }
+            }
+            float* s_ss = reinterpret_cast<float*>(misc + M_SS) + (nn & 1) * 256;
+            s_ss[(2 * half + cp) * 64 + t] = ss * p.scale * p.scale;
+            bar_sync(bar_out, 128);
+            if (ok && lw == 2 && lane == 0) mbar_arrive(bar_at(misc, M_NRM + 8 * (nn & 1)));
+            ok = ok && wait_warp(bar_at(misc, M_NRM + 8 * (nn & 1)), (uint32_t)(nn >> 1) & 1u, p);
+            if (ok) {
+                const float tot = s_ss[t] + s_ss[64 + t] + s_ss[128 + t] + s_ss[192 + t];
+                inv = rsqrtf(tot * (1.f / kD) + p.norm_eps);
+            }
+        }
+        // this thread's 16 output values hx (scaled, and normed with kNorm), as bf16
+        auto finish = [&](int hx, float* ov) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) ov[u] *= p.scale;
+            if constexpr (kN) {
+                const float* wn = reinterpret_cast<const float*>(misc + M_WN) + jg0 + 16 * hx;
+                float zv[16];
+                unpack8(zr[2 * hx], zv);
+                unpack8(zr[2 * hx + 1], zv + 8);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) ov[u] = ov[u] * inv * wn[u] * sigmoid_f(zv[u]);
+            }
+        };
+        if (L == kC) {
+            const bool storer = (lw == 2 && lane == 0);
+            if (storer) bulk_wait_read0();          // the previous tile has left the staging
+            bar_sync(bar_out, 128);
+            if (ok) {
+#pragma unroll
+                for (int hx = 0; hx < 2; ++hx) {
+                    float ov[16];
+                    tmem_ld16(src + 16 * hx, ov);
+                    finish(hx, ov);
+                    st16(sm, ost_h + sw128(t, 4 * cp + 2 * hx, 0, 0), pack8(ov));
+                    st16(sm, ost_h + sw128(t, 4 * cp + 2 * hx + 1, 0, 0), pack8(ov + 8));
+                }
+            }
+            fence_async_smem();
+            bar_sync(bar_out, 128);
+            if (storer && ok) {
+                tma_store_3d(&p.to, 64 * half, h, (int)c0, sb + ost_h);
+                bulk_commit();
+            }
+        } else if (ok) {
+            uint4* dst = reinterpret_cast<uint4*>(p.o + ((c0 + t) * H + h) * kD + jg0);
+#pragma unroll
+            for (int hx = 0; hx < 2; ++hx) {
+                float ov[16];
+                tmem_ld16(src + 16 * hx, ov);       // (warp-collective: every lane loads)
+                finish(hx, ov);
+                if (t < L) {
+                    dst[2 * hx] = pack8(ov);
+                    dst[2 * hx + 1] = pack8(ov + 8);
+                }
+            }
+        }
+    };
+
+    bool stop = aborted;
+    int fail = aborted ? 1 : 0;
+    // prologue: Sm(0), then [X ; O](0)
+    if (!stop && nchunks > 0) {
+        const bool ok = wait_warp(bar_at(misc, M_AFULL), 0, p);
+        if (ok) write_sm(0);
+        fail |= !ok;
+        fence_async_smem();
+        stop = bar_sync_or(bar_half, 256, fail) != 0;
+        if (!stop && issuer) issue_xo(0);
+    }
+    for (int n = 0; n < nchunks && !stop; ++n) {
+        const int b = n & 1;
+        // (1) [X ; O](n) is in tensor memory: U(n) = V(n) - X(n) from rows 0..63, and the output
+        //     of chunk n - 1 from rows 64..127 of the other accumulator
+        bool ok = wait_warp(bar_xo, (uint32_t)b, p);
+        if (issuer && ok) ++xo_waited;
         tc_fence_after();
-        const uint32_t idS = idesc_bf16(128, 128, false, false);
-        const uint32_t idO = idesc_bf16(128, 64, false, false);
-        const uint64_t bY = make_desc(sb + so + S_YW, 16, 1024);
-        const uint64_t bW = make_desc(sb + so + S_YW + 128 * 128, 16, 1024);
-        const uint32_t dO = tm + ((nn & 1) ? TXO1 : TXO0) + 64;
-        if (elect_one()) {
+        if (ok && n > 0 && tid_h == 0) mbar_arrive(bar_at(misc, M_BFREE + 8 * ((n - 1) & 1)));
+        if (q < 2) {
+            if (ok) ok = wait_warp(bar_at(misc, M_VFULL + 8 * (2 * half + b)), (uint32_t)(n >> 1) & 1u, p);
+            if (ok) {
+                const int t = 32 * q + lane;
+                const uint8_t* vt = sm + C_V + (uint32_t)(2 * half + b) * 8192;
 #pragma unroll
-            for (int s = 0; s < 4; ++s) mma_bf16_ts(tm + TC_DS, tm + TC_U + 8 * s, desc_add(bY, s * 32), idS, s > 0);
-            mma_commit(bar_s);
+                for (int hx = 0; hx < 2; ++hx) {
+                    float xv[16];
+                    tmem_ld16(t_xo + 64 * b + lane_sel + 32 * cp + 16 * hx, xv);
 #pragma unroll
-            for (int s = 0; s < 4; ++s) mma_bf16_ts(dO, tm + TC_U + 8 * s, desc_add(bW, s * 32), idO, 1);
-            mma_commit(bar_o);
+                    for (int k2 = 0; k2 < 2; ++k2) {
+                        const int ck = 4 * cp + 2 * hx + k2;
+                        float vv[8];
+                        unpack8(ld16(vt, t * 128 + ((ck ^ (t & 7)) << 4)), vv);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) vv[u] -= xv[8 * k2 + u];
+                        st16(sm, u_h + sw128(t, ck, 0, 0), pack8(vv));
+                    }
+                }
+            }
+        } else if (n > 0) {
+            epilogue_o(n - 1, ok);
         }
-        __syncwarp();
-    };
-    // Sm(nn) = (S^T diag(e^{gamma_ref(nn)})) as bf16 pairs along the key channel
-    auto pack_sm = [&](int nn, uint32_t* w) {
-        const float* fac = reinterpret_cast<const float*>(sm + C_SLOT0 + (uint32_t)(nn & 1) * kSlotBytes + S_FAC);
-        const float4* e4 = reinterpret_cast<const float4*>(fac + 32 * wg);
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 e = e4[q4];
-            w[2 * q4] = pack_bf16(sreg[4 * q4] * e.x, sreg[4 * q4 + 1] * e.y);
-            w[2 * q4 + 1] = pack_bf16(sreg[4 * q4 + 2] * e.z, sreg[4 * q4 + 3] * e.w);
-        }
-    };
-    // U(nn) = V(nn)^T - X(nn) for value channel j and tokens [16 wg, 16 wg + 16), as bf16
-    // pairs along the token into tensor memory. V[t][j] sits in box j / 64, row t, 16-byte
-    // chunk ((j % 64) / 8) ^ (t % 8) of the 128B-swizzled tile.
-    auto make_u = [&](int nn) {
-        tc_fence_after();
-        float xv[16];
-        tmem_ld16(tm + lane_sel + ((nn & 1) ? TXO1 : TXO0) + 16 * wg, xv);
-        const uint8_t* vt = sm + C_V + (uint32_t)(nn % 3) * 16384 + 8192 * (j >> 6) + (j & 7) * 2;
-        const int jc = (j & 63) >> 3;
-        uint32_t w[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t0 = 16 * wg + 2 * u;
-            const float v0 = bf(reinterpret_cast<const __nv_bfloat16*>(vt + t0 * 128 + ((jc ^ (t0 & 7)) << 4)));
-            const float v1 = bf(reinterpret_cast<const __nv_bfloat16*>(vt + (t0 + 1) * 128 + ((jc ^ ((t0 + 1) & 7)) << 4)));
-            w[u] = pack_bf16(v0 - xv[2 * u], v1 - xv[2 * u + 1]);
-        }
-        tmem_st8(tm + lane_sel + TC_U + 8 * wg, w);
-        tmem_wait_st();
-    };
-    // O of chunk nn, by warps 1..15 (warp 4 also takes warp 0's share): TMEM -> bf16
-    // [token][channel] staging -> one TMA tile store (a ragged last chunk: one bulk copy per
-    // valid token, so rows of the next sequence are never touched)
-    auto epilogue_o = [&](int nn) -> bool {
-        if (warp == 1) bulk_wait_read0();       // the previous O tile has left the staging
-        const bool ok = group_wait(bar_o, (uint32_t)(nn & 1), nullptr, 0, p.err);   // once per chunk
-        tc_fence_after();
-        const uint32_t to = tm + lane_sel + ((nn & 1) ? TXO1 : TXO0) + 64;
-        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
-        for (int part = (warp == 4 ? 0 : 1); part < 2; ++part) {
-            const int t0 = part ? 16 * wg : 0;
-            float ov[16];
-            tmem_ld16(to + t0, ov);
-#pragma unroll
-            for (int t = 0; t < 16; ++t) st[(t0 + t) * kD + j] = __float2bfloat16_rn(p.scale * ov[t]);
-        }
+        fail |= !ok;
         fence_async_smem();
         tc_fence_before();
-        group_sync();
-        if (warp == 1) {
-            const int64_t c0 = bos + (int64_t)nn * kC;
-            const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
-            const int lane = tid & 31;
-            if (L == kC) {
-                if (lane == 0) tma_store_3d(&p.to, 0, h, (int)c0, sb + C_OST);
+        if (bar_sync_or(bar_half, 256, fail)) { stop = true; break; }
+        if (tid_h == 0) mbar_arrive(bar_at(misc, M_VFREE + 8 * (2 * half + b)));
+        // (2) state delta Yh^T U (commit), then O(n) += Wh^T U
+        if (issuer) {
+            if (wait_warp(bar_at(misc, M_BFULL + 8 * b), (uint32_t)(n >> 1) & 1u, p)) {
+                tc_fence_after();
+                if (elect_one()) {
+                    const uint32_t id = idesc_bf16(128, 64, false, true);
+                    const uint32_t bp = sb + C_B + (uint32_t)b * kBPart;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(t_ds, make_desc(bp + s * 32, 16, 1024), make_desc(sb + u_h + s * 2048, 8192, 1024),
+                                 id, s > 0);
+                    mma_commit(bar_ds);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(t_xo + 64 * b, make_desc(bp + 8192 + s * 32, 16, 1024),
+                                 make_desc(sb + u_h + s * 2048, 8192, 1024), id, 1);
+                }
+                __syncwarp();
+                ++ds_issued;
             } else {
-                for (int r = lane; r < L; r += 32)
-                    bulk_store(p.o + ((c0 + r) * H + h) * kD, sb + C_OST + r * 256, 256);
-            }
-            bulk_commit();
-        }
-        return ok;
-    };
-
-    // prologue: V tiles of chunks 0..2, factors of chunks 0 and 1, Sm(0), then [X | O](0)
-    if (nchunks > 0) {
-        issue_v(0);
-        if (nchunks > 1) issue_v(1);
-        if (nchunks > 2) issue_v(2);
-        // chunk 0 must have arrived (which frees ring slot 0 for chunk kRing) before the loader
-        // waits for chunk 1: a producer announces a chunk only during its next task
-        if (__syncthreads_or(!issue_load(0))) aborted = true;   // (seen by every thread)
-        if (!aborted && !wait_next(0)) aborted = true;
-        if (!aborted && nchunks > 1 && __syncthreads_or(!issue_load(1))) aborted = true;
-        if (!aborted) {
-            uint32_t w[16];
-            pack_sm(0, w);
-            tmem_st16(tm + lane_sel + TC_SM + 16 * wg, w);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncthreads();
-            if (warp == 0) issue_xo(0);
-        }
-    }
-
-    // Warp 0 issues the MMAs and blocks for about their execution time, so after each issue
-    // warps 1..15 go on alone (named barrier 1) and warp 0 catches up at the next block-wide
-    // barrier. A failed wait only raises `fail`; the block leaves the loop together at the
-    // next block-wide barrier.
-    int fail = 0;
-    for (int n = 0; n < nchunks && !aborted; ++n) {
-        const float* fac = reinterpret_cast<const float*>(sm + C_SLOT0 + (uint32_t)(n & 1) * kSlotBytes + S_FAC);
-        const bool more = n + 1 < nchunks;
-        const int n1 = n + 1, sl1 = n1 & 1, e1 = n1 % 3;
-        trace_mark(0, n, 0);
-        // (1) U(n) = V(n)^T - X(n), then U [Yh | Wh]
-        if (!block_wait_or(bar_x, ph_x & 1u, fail, p.err)) { aborted = true; break; }
-        ph_x ^= 1u;
-        trace_mark(0, n, 1);
-        make_u(n);
-        tc_fence_before();
-        __syncthreads();
-        trace_mark(0, n, 2);
-        // (2) the next chunk's operands and this chunk's state delta
-        if (warp == 0) {
-            issue_u(n);
-            trace_mark(0, n, 3);
-            if (more && !warp_wait(bar_lfull + sl1, (ph_lfull >> sl1) & 1u, p.err)) fail = 1;
-            if (!warp_wait(bar_s, ph_s & 1u, p.err)) fail = 1;
-        } else {
-            if (more && !group_wait(bar_lfull + sl1, (ph_lfull >> sl1) & 1u, bar_v + e1, (ph_v >> e1) & 1u, p.err))
                 fail = 1;
-            if (more && tid == 32 && n1 + kRing < nchunks)    // ring slot of n + 1 may take n + 1 + kRing
-                mbar_arrive_remote_relaxed(map_to_rank(sb + P_MISC + M_GFREE + 8u * (uint32_t)(n1 % kRing),
-                                                       1 + (n1 + kRing) % kProducers));
-            if (!group_wait(bar_s, ph_s & 1u, nullptr, 0, p.err)) fail = 1;
-        }
-        if (more) {
-            ph_lfull ^= 1u << sl1;
-            ph_v ^= 1u << e1;
-        }
-        ph_s ^= 1u;
-        trace_mark(0, n, 4);
-        // (3) state update S' = e^{gamma_C} S + U Yh, then Sm(n + 1)
-        tc_fence_after();
-        {
-            float v32[32];
-            tmem_ld32(tm + lane_sel + TC_DS + 32 * wg, v32);
-            const float4* eC4 = reinterpret_cast<const float4*>(fac + 128 + 32 * wg);
-#pragma unroll
-            for (int t4 = 0; t4 < 8; ++t4) {
-                const float4 ec = eC4[t4];
-                const float* v = v32 + 4 * t4;
-                const int cc = 4 * t4;
-                sreg[cc] = fmaf(ec.x, sreg[cc], v[0]);
-                sreg[cc + 1] = fmaf(ec.y, sreg[cc + 1], v[1]);
-                sreg[cc + 2] = fmaf(ec.z, sreg[cc + 2], v[2]);
-                sreg[cc + 3] = fmaf(ec.w, sreg[cc + 3], v[3]);
             }
         }
-        if (more) {
-            uint32_t w[16];
-            pack_sm(n1, w);
-            tmem_st16(tm + lane_sel + TC_SM + 16 * wg, w);
-            tmem_wait_st();
+        // (3) S' = e^{gamma_C} S + delta, then Sm(n + 1)
+        ok = wait_warp(bar_ds, (uint32_t)b, p);
+        if (issuer && ok) ++ds_waited;
+        tc_fence_after();
+        if (ok) {
+            const float eC = fac(n)[kD + i_row];
+#pragma unroll
+            for (int hx = 0; hx < 2; ++hx) {
+                float dv[16];
+                tmem_ld16(t_ds + lane_sel + 32 * cp + 16 * hx, dv);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) S[16 * hx + u] = fmaf(eC, S[16 * hx + u], dv[u]);
+            }
+            if (n + 1 < nchunks) {
+                ok = wait_warp(bar_at(misc, M_AFULL + 8 * ((n + 1) & 1)), (uint32_t)((n + 1) >> 1) & 1u, p);
+                if (ok) write_sm(n + 1);
+            }
         }
-        trace_mark(0, n, 5);
+        fail |= !ok;
+        fence_async_smem();
         tc_fence_before();
-        if (__syncthreads_or(fail)) { aborted = true; break; }
-        trace_mark(0, n, 6);
-        if (warp == 0) {
-            // (4) the next chunk's [X | O]
-            if (more) issue_xo(n1);
-            trace_mark(0, n, 7);
-        } else {
-            // (4') output of chunk n, then the loads that the completed chunk n made possible:
-            // shared slot n % 2 takes chunk n + 2, V ring entry n % 3 takes V(n + 3)
-            if (!epilogue_o(n)) fail = 1;
-            trace_mark(0, n, 8, 32);
-            if (n + 2 < nchunks) issue_load(n + 2);   // a failed wait flags the error word; the
-                                                      // consumer then gives up at the next wait
-            if (n + 3 < nchunks) issue_v(n + 3);
-            trace_mark(0, n, 9, 32);
+        if (bar_sync_or(bar_half, 256, fail)) { stop = true; break; }
+        if (tid_h == 0) mbar_arrive(bar_at(misc, M_AFREE + 8 * b));
+        // (4) the next chunk's [X ; O], or a commit that covers O(n) after the last chunk
+        if (issuer) {
+            if (n + 1 < nchunks) {
+                issue_xo(n + 1);
+            } else {
+                tc_fence_after();
+                if (elect_one()) mma_commit(bar_xo);
+                __syncwarp();
+                ++xo_issued;
+            }
         }
     }
-    if (warp == 1) bulk_wait0();
-    if (p.ht && !aborted) {
+    if (!stop && nchunks > 0) {
+        const bool ok = wait_warp(bar_xo, (uint32_t)(nchunks & 1), p);
+        if (issuer && ok) ++xo_waited;
+        tc_fence_after();
+        if (q >= 2) epilogue_o(nchunks - 1, ok);
+        stop = bar_sync_or(bar_half, 256, !ok) != 0;
+    }
+    if (!stop && p.ht) {
+        float4* dst = reinterpret_cast<float4*>(p.ht + sbase + (int64_t)i_row * kD + jg0);
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc) p.ht[sbase + (int64_t)(32 * wg + cc) * kD + j] = sreg[cc];
+        for (int c4 = 0; c4 < 8; ++c4) dst[c4] = make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
+    }
+    if (lw == 2 && lane == 0) bulk_wait0();
+    // products still in flight must finish before the tensor memory is freed
+    if (issuer) {
+        if (xo_issued > xo_waited) mbar_wait(bar_xo, (uint32_t)((xo_issued - 1) & 1), kDefaultWaitCycles);
+        if (ds_issued > ds_waited) mbar_wait(bar_ds, (uint32_t)((ds_issued - 1) & 1), kDefaultWaitCycles);
     }
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -947,22 +1141,35 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
     }
     if (threadIdx.x == 0) {
         // every barrier completes once per use: one arrival (plus transaction bytes where a TMA
-        // or bulk copy feeds it)
-        for (uint32_t b = 0; b < kBars; ++b) mbar_init(reinterpret_cast<uint64_t*>(misc + 8 * b), 1);
+        // or bulk copy feeds it), except the consumer's slot-free barriers: one per half
         if (is_consumer) {
+            for (int b = 0; b < kBarsC; ++b) {
+                const uint32_t off = 8u * b;
+                const bool two = (off >= M_AFREE && off < M_VFULL) || off >= M_NRM;
+                mbar_init(bar_at(misc, off), two ? 2 : 1);
+            }
             const uint32_t id = smid();
             *reinterpret_cast<uint32_t*>(misc + M_SMID) = id;
             if ((int)id >= p.ring_sms) atomicOr(p.err, kErrTimeout);
+        } else {
+            for (int b = 0; b < kBarsP; ++b) mbar_init(bar_at(misc, 8u * b), 1);
         }
+        fence_mbar_init();
+    }
+    if (is_consumer && (MODE & kNorm) != 0)          // the output norm's weight
+        for (int i = threadIdx.x; i < kD; i += kThreads) reinterpret_cast<float*>(misc + M_WN)[i] = p.w_norm[i];
+    if (!is_consumer) {     // T' blocks above the diagonal are never written: zero them once
+        for (int e = threadIdx.x; e < 8192 / 16; e += kThreads) st16(sm, P_TP + 16 * e, make_uint4(0, 0, 0, 0));
+        fence_async_smem();
     }
     tc_fence_before();
     cluster_sync();                     // barriers of every CTA exist before any remote arrive
     tc_fence_after();
 
     // a consumer SM outside the workspace's ring table (flagged above): nobody touches the ring
-    bool aborted = (int)ld_cluster_u32(map_to_rank(sb + C_MISC + M_SMID, 0)) >= p.ring_sms;
-    if (is_consumer) consumer(p, sm, sb, n_seq, h, bos, eos, aborted);
-    else producer(p, sm, sb, (int)crank, h, bos, eos, aborted);
+    const bool aborted = (int)ld_cluster_u32(map_to_rank(sb + C_MISC + M_SMID, 0)) >= p.ring_sms;
+    if (is_consumer) consumer<MODE>(p, sm, sb, n_seq, h, bos, eos, aborted);
+    else producer<MODE>(p, sm, sb, (int)crank, h, bos, eos, aborted);
 
     tc_fence_before();
     __syncthreads();
@@ -975,25 +1182,32 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
 
 }  // namespace
 
-// Ring tables for SM ids 0 .. kRingSms - 1 (a B200 has 148 SMs).
-constexpr int kRingSms = 160;
-size_t chunk_tcx_workspace_bytes() { return (size_t)kRingSms * kRing * kSlotBytes; }
+size_t chunk_tcx_workspace_bytes() { return kTcxWorkspaceBytes; }
 
 cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspace_bytes,
                              unsigned int* err, cudaStream_t stream) {
     const int64_t units = (int64_t)a.N * a.H;
     if (units == 0) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(chunk_tcx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const int mode = (a.g_raw != nullptr ? kGate : 0) | (a.z != nullptr ? kNorm : 0);
+    if (mode == kNorm) return cudaErrorInvalidValue;          // the norm comes with the gate
+    void (*kernel)(Params) = mode == 0 ? chunk_tcx_kernel<0>
+                           : mode == kGate ? chunk_tcx_kernel<kGate> : chunk_tcx_kernel<kGate | kNorm>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     Params p;
+    const bool gate = (mode & kGate) != 0;
     const bool maps_ok =
         make_tmap_thd(&p.tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false) &&
         make_tmap_thd(&p.tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false) &&
-        make_tmap_thd(&p.tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.T_tot, a.H, kD, kD, kC, false) &&
+        (gate ? make_tmap_thd(&p.tg, a.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false)
+              : make_tmap_thd(&p.tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.T_tot, a.H, kD, kD, kC, false)) &&
         make_tmap_thd(&p.tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, 64, kC, true) &&
-        make_tmap_thd(&p.to, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false);
+        make_tmap_thd(&p.to, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, 64, kC, true);
     if (!maps_ok) return cudaErrorInvalidValue;
+    p.q = static_cast<const __nv_bfloat16*>(a.q);
+    p.k = static_cast<const __nv_bfloat16*>(a.k);
+    p.g = a.g;
     p.beta = a.beta;
     p.scale = a.scale;
     p.h0 = a.h0;
@@ -1004,8 +1218,16 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
     p.N = a.N;
     p.H = a.H;
     p.err = err;
+    p.wait_cycles = g_chunk_wait_cycles > 0 ? g_chunk_wait_cycles : kDefaultWaitCycles;
     p.ring = static_cast<uint8_t*>(workspace);
     p.ring_sms = (int)(workspace_bytes / ((size_t)kRing * kSlotBytes));
+    p.g_raw = static_cast<const __nv_bfloat16*>(a.g_raw);
+    p.beta_raw = static_cast<const __nv_bfloat16*>(a.beta_raw);
+    p.A_log = a.A_log;
+    p.dt_bias = a.dt_bias;
+    p.z = static_cast<const __nv_bfloat16*>(a.z);
+    p.w_norm = a.w_norm;
+    p.norm_eps = a.norm_eps;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units * kCluster), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1018,16 +1240,9 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, chunk_tcx_kernel, p);
+    e = cudaLaunchKernelEx(&cfg, kernel, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 }  // namespace kda
-
-#ifdef KDA_TRACE
-// Copies the prefill phase timestamps (see trace_mark) to `host` (4 * 512 * 16 uint64).
-extern "C" __attribute__((visibility("default"))) int kda_trace_dump(unsigned long long* host) {
-    return (int)cudaMemcpyFromSymbol(host, kda::g_trace, sizeof(kda::g_trace));
-}
-#endif

@@ -24,13 +24,28 @@ struct ConvArgs {
 cudaError_t launch_conv(const ConvArgs& a, cudaStream_t stream);
 
 struct StepArgs {
-    const void *q, *k, *v;
+    const void *q, *k, *v;           // formed q, k, v, or the raw inputs when conv_state is set
     const float *g, *beta;
     float scale;
     float* state;
     void* o;
     int N, H, dk, dv;
     Io io;
+    // conv prologue fused into the step (conv_state non-null): weights [H*d, 4], the width-3
+    // history [N, H*(2dk+dv), 3] advanced in place, and the L2-norm epsilon of q and k
+    const float* w[3] = {nullptr, nullptr, nullptr};
+    void* conv_state = nullptr;
+    float eps = 0.f;
+    // gate from raw logits (A_log non-null): g_raw [N,H,dk] and beta_raw [N,H] in the io
+    // dtype, A_log [H], dt_bias [H*dk]; then g and beta above are unused. Optional output
+    // gated RMSNorm: z [N,H,dv] io dtype (null: none), w_norm [dv], norm_eps.
+    const void* g_raw = nullptr;
+    const void* beta_raw = nullptr;
+    const float* A_log = nullptr;
+    const float* dt_bias = nullptr;
+    const void* z = nullptr;
+    const float* w_norm = nullptr;
+    float norm_eps = 0.f;
 };
 cudaError_t launch_recurrent_step(const StepArgs& a, cudaStream_t stream);
 
@@ -47,15 +62,35 @@ struct ChunkArgs {
     int T_pad;
     int N, H, dk, dv, chunk;
     Io io;
+    // tensor-core path only: gate and beta from raw logits (g_raw non-null: bf16 g_raw
+    // [T_tot,H,dk] and beta_raw [T_tot,H], A_log [H], dt_bias [H*dk]; g and beta unused), and
+    // the output's gated RMSNorm (z non-null: bf16 z [T_tot,H,dv], w_norm [dv], norm_eps)
+    const void* g_raw = nullptr;
+    const void* beta_raw = nullptr;
+    const float* A_log = nullptr;
+    const float* dt_bias = nullptr;
+    const void* z = nullptr;
+    const float* w_norm = nullptr;
+    float norm_eps = 0.f;
 };
 cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 
-// Tensor-core (tcgen05) prefill: bf16 I/O, dk = dv = 128, chunk 64.
-bool chunk_tc_supported(const ChunkArgs& a);
-cudaError_t launch_chunk_tc(const ChunkArgs& a, unsigned int* err, cudaStream_t stream);
-// Same math as a producer/consumer pipeline in one 4-CTA cluster per (sequence, head). Needs a
-// device workspace of chunk_tcx_workspace_bytes() (16-byte aligned): the per-SM hand-off rings.
+// Hand-off rings of the cluster prefill (bf16 I/O, dk = dv = 128, chunk 64): one ring of
+// kTcxRingSlots slots per SM id below kTcxRingSms, each slot one chunk's factors.
+constexpr int kTcxRingSms = 160;                 // a B200 has 148 SMs
+constexpr int kTcxRingSlots = 6;
+constexpr size_t kTcxSlotBytes = 58368;
+constexpr size_t kTcxWorkspaceBytes = (size_t)kTcxRingSms * kTcxRingSlots * kTcxSlotBytes;
+
+// Tensor-core (tcgen05) prefill for bf16 I/O, dk = dv = 128, chunk 64: a producer/consumer
+// pipeline in one 4-CTA cluster per (sequence, head). Needs a device workspace of
+// chunk_tcx_workspace_bytes() (16-byte aligned): the per-SM hand-off rings.
+inline bool chunk_tc_supported(const ChunkArgs& a) {
+    return a.io == Io::BF16 && a.dk == 128 && a.dv == 128 && a.chunk == 64;
+}
 size_t chunk_tcx_workspace_bytes();
+// Bound (SM cycles) of every device-side wait of later prefill launches; 0 restores the default.
+extern long long g_chunk_wait_cycles;
 cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspace_bytes,
                              unsigned int* err, cudaStream_t stream);
 

@@ -1,17 +1,19 @@
-// tc.cuh -- thin wrappers over the sm_100a tensor-core (tcgen05 / TMEM), mbarrier and
-// proxy-fence PTX used by the prefill kernel, plus the shared-memory operand layouts.
+// tc.cuh -- thin wrappers over the sm_100a PTX that the prefill kernel uses: tensor cores
+// (tcgen05 / TMEM), mbarriers, TMA and bulk copies, clusters, and named barriers; plus the
+// shared-memory operand layouts.
 //
-// Operand layouts (bf16, 128-byte swizzle, "canonical" tcgen05 shared-memory forms):
-//  K-major   : rows of the M (or N) index, 64 K-elements (128 B) per row inside one
-//              swizzle atom of 8 rows (1024 B); 16-byte chunk c of row r is stored at
-//              chunk position c ^ (r % 8). K > 64 uses further atom columns of
-//              rows_total * 128 bytes each. Descriptor: SBO = 1024 B (8-row groups);
-//              a K step of 16 elements advances the start address by 32 B.
-//  MN-major  : rows of the K index, 64 M/N-elements (128 B) per row inside one atom of
-//              8 K-rows (1024 B), same chunk swizzle with the K-row index. K-groups of
-//              8 rows follow each other at 1024 B (SBO); a second 64-wide M/N block
-//              starts after all K-groups of the first (LBO). A K step of 16 elements
-//              advances the start address by 2048 B.
+// Operand layouts (bf16, 128-byte swizzle, the canonical tcgen05 shared-memory forms):
+//  K-major  : rows of the M (or N) index, 64 K-elements (128 B) per row inside one swizzle
+//             atom of 8 rows (1024 B); 16-byte chunk c of row r is stored at chunk position
+//             c ^ (r % 8). K > 64 uses further atom columns (rows_total * 128 bytes each).
+//             Descriptor: SBO = 1024 B (8-row groups); a K step of 16 elements advances the
+//             start address by 32 B inside an atom column.
+//  MN-major : rows of the K index, 64 M/N-elements (128 B) per row inside one atom of 8 K-rows
+//             (1024 B), with the same chunk swizzle by the K-row index. K-groups of 8 rows
+//             follow each other at 1024 B (SBO); a second 64-wide M/N block starts LBO bytes
+//             later. A K step of 16 elements advances the start address by 2048 B.
+// The two forms are the same bytes: a tile written K-major with rows r and 16-byte chunks c is
+// also the MN-major operand whose K index is r and whose M/N index runs along the chunks.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -25,7 +27,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// ---- shared-memory descriptor (tcgen05 matrix descriptor) ----
+// ---------------------------------------------------------------------------------------------
+// Operand descriptors and layouts
+// ---------------------------------------------------------------------------------------------
+
+// Shared-memory matrix descriptor (128-byte swizzle, sm_100 descriptor version).
 __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
@@ -36,13 +42,11 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo_bytes
     return d;
 }
 
-// ---- instruction descriptor: kind::f16 with bf16 A/B and fp32 accumulation ----
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major,
-                                                  bool negate_a = false) {
+// Instruction descriptor of kind::f16 with bf16 A and B and fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                         // D format: f32
          | (1u << 7)                         // A format: bf16
          | (1u << 10)                        // B format: bf16
-         | ((negate_a ? 1u : 0u) << 13)
          | ((a_mn_major ? 1u : 0u) << 15)
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)
@@ -50,21 +54,35 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
 }
 
 // Byte offset of the 16-byte chunk `chunk` (0..7 inside a 64-element atom row) of row `row`
-// of a K-major operand whose atom column `acol` holds `rows_total` rows.
-__device__ __forceinline__ uint32_t kmaj_chunk(int row, int chunk, int acol, int rows_total) {
+// of a 128B-swizzled operand whose atom column `acol` holds `rows_total` rows.
+__host__ __device__ __forceinline__ uint32_t sw128(int row, int chunk, int acol, int rows_total) {
     return (uint32_t)(acol * rows_total * 128 + (row >> 3) * 1024 + (row & 7) * 128 +
                       ((chunk ^ (row & 7)) << 4));
 }
-// Byte offset of the 16-byte chunk `chunk` (0..7) of K-row `k` in M/N block `mnb` of an
-// MN-major operand with `kgroups` groups of 8 K-rows.
-__device__ __forceinline__ uint32_t mnmaj_chunk(int k, int chunk, int mnb, int kgroups) {
-    return (uint32_t)(mnb * kgroups * 1024 + (k >> 3) * 1024 + (k & 7) * 128 +
-                      ((chunk ^ (k & 7)) << 4));
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
-// ---- mbarrier ----
+// 2^x by the SFU (approximate; inputs here stay within +-116).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ---------------------------------------------------------------------------------------------
+// mbarriers (every wait is bounded by a cycle count and reports whether the phase completed)
+// ---------------------------------------------------------------------------------------------
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
@@ -78,20 +96,62 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: gives up after ~`limit_cycles` SM cycles and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  long long limit_cycles) {
+// Wait with cluster-scope acquire (pairs with a remote release arrive).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase with the given parity: false after ~limit_cycles SM cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_cycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait(bar, parity))
         if (clock64() - t0 > limit_cycles) return false;
-    }
     return true;
 }
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, long long limit_cycles) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity))
+        if (clock64() - t0 > limit_cycles) return false;
+    return true;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// Arrive on a barrier of another CTA of the cluster (address from map_to_rank).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                 ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
 
-// ---- proxy / tcgen05 ordering fences ----
+// ---------------------------------------------------------------------------------------------
+// Fences, named barriers, clusters
+// ---------------------------------------------------------------------------------------------
+
+// Makes this thread's generic-proxy shared-memory writes visible to the async proxy (tensor
+// cores, bulk copies).
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Orders this thread's async-proxy global accesses with its generic ones.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -99,8 +159,94 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+// Named barrier `id` over `nthreads` threads (whole warps) with an OR-reduction of `pred`.
+__device__ __forceinline__ int bar_sync_or(int id, int nthreads, int pred) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.s32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r;
+}
+__device__ __forceinline__ void bar_sync(int id, int nthreads) {
+    asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+__device__ __forceinline__ uint32_t smid() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
+// One lane of a converged warp returns true.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(pred));
+    return pred != 0;
+}
 
-// ---- TMEM allocation (whole warp) ----
+// ---------------------------------------------------------------------------------------------
+// TMA and bulk copies
+// ---------------------------------------------------------------------------------------------
+
+// 3-D tiled load of the box at (c0, c1, c2) into this CTA's shared memory; completes on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)) : "memory");
+}
+// 3-D tiled store of a shared-memory box to (c0, c1, c2); tracked by the thread's bulk groups.
+__device__ __forceinline__ void tma_store_3d(const void* tmap, int c0, int c1, int c2, uint32_t src) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+                 ::"l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(src) : "memory");
+}
+// Bulk copy global -> this CTA's shared memory, completing on a local mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+// Bulk copy shared -> global, tracked by bulk groups of the issuing thread.
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(gdst), "r"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until the thread's bulk groups have finished reading their shared-memory sources.
+__device__ __forceinline__ void bulk_wait_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until the thread's bulk groups are complete (their writes performed).
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------------
+// Tensor memory and tensor-core MMA (kind::f16, bf16 inputs, fp32 accumulation)
+// ---------------------------------------------------------------------------------------------
+
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
@@ -112,8 +258,7 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                  : "memory");
 }
-
-// ---- MMA (single thread) and commit ----
+// D (tensor memory) (+)= A (shared) * B (shared); issued by one thread.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -123,12 +268,28 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Arrives on `bar` once every tcgen05 operation this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(smem_u32(bar)) : "memory");
 }
+// Descriptor advanced by a byte offset (the start address field is in 16-byte units).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
-// ---- TMEM -> registers: 32 lanes x 32 consecutive 32-bit columns per warp ----
+// TMEM -> registers: 32 lanes x 16 (or 32) consecutive 32-bit columns per warp.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     uint32_t r[32];
     asm volatile(
@@ -147,131 +308,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-    __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&p);
-}
+// ---------------------------------------------------------------------------------------------
+// Warp-level 16x16 fp32 block products on the tensor cores (TF32 inputs, fp32 sums)
+// ---------------------------------------------------------------------------------------------
 
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-
-// ---- thread-block clusters and distributed shared memory ----
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Address of the same shared-memory location in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void st_cluster16(uint32_t addr, uint4 v) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};"
-                 ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
-                 ::"r"(cluster_addr) : "memory");
-}
-// Wait with cluster-scope acquire (pairs with mbar_arrive_remote), bounded.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity,
-                                                          long long limit_cycles) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait_cluster(bar, parity)) {
-        if (clock64() - t0 > limit_cycles) return false;
-    }
-    return true;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
-                 ::: "memory");
-}
-__device__ __forceinline__ void fence_async_cluster() {
-    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_acq_rel_cluster() {
-    asm volatile("fence.acq_rel.cluster;" ::: "memory");
-}
-
-// ---- 16-byte asynchronous global -> shared copy (zero-fills when src_bytes == 0) ----
-__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* gptr, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                 ::"r"(saddr), "l"(gptr), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-
-// One lane of a converged warp returns true (tcgen05.mma / commit issue).
-__device__ __forceinline__ bool elect_one() {
-    uint32_t pred = 0;
-    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(pred));
-    return pred != 0;
-}
-// Issued by every lane of one converged warp: one lane issues the MMA.
-__device__ __forceinline__ void warp_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate) {
-    if (elect_one()) mma_bf16(d_tmem, adesc, bdesc, idesc, accumulate);
-    __syncwarp();
-}
-__device__ __forceinline__ void warp_commit(uint64_t* bar) {
-    if (elect_one()) mma_commit(bar);
-    __syncwarp();
-}
-// Descriptor advanced by a byte offset (the start address field is in 16-byte units).
-__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
-
-// Remote arrive that also announces `bytes` of incoming transactions on a peer's mbarrier.
-__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_addr, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
-                 ::"r"(cluster_addr), "r"(bytes) : "memory");
-}
-// Bulk copy from this CTA's shared memory into a peer's, completing on the peer's mbarrier.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                                  uint32_t mbar_cluster) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst_cluster), "r"(src_cta), "r"(bytes), "r"(mbar_cluster) : "memory");
-}
-
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
-}
-
-// ---- warp-level 16x16 fp32 block products on the tensor cores (TF32 inputs, fp32 sums) ----
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -305,224 +345,8 @@ __device__ __forceinline__ void warp_block_mma16(float (*acc)[4], const float* A
         }
     }
 }
-// Writes scale * acc (two 16x8 fragments) to a 16x16 fp32 block with row stride ld.
-__device__ __forceinline__ void warp_block_store16(float* C, int ld, const float (*acc)[4], float scale) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        C[g * ld + 8 * nt + 2 * t] = scale * acc[nt][0];
-        C[g * ld + 8 * nt + 2 * t + 1] = scale * acc[nt][1];
-        C[(g + 8) * ld + 8 * nt + 2 * t] = scale * acc[nt][2];
-        C[(g + 8) * ld + 8 * nt + 2 * t + 1] = scale * acc[nt][3];
-    }
-}
+// Element (row, col) of the 16x16 accumulator held by this lane as acc[nt][e]:
+// row = g + 8 * (e >> 1), col = 8 * nt + 2 * t + (e & 1), with g = lane / 4, t = lane % 4.
 
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-
-// ---- TMA (tensor memory accelerator) ----
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-// 3-D tiled load of the box at (c0, c1, c2) into this CTA's shared memory; completes on `bar`.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int c0, int c1, int c2,
-                                            uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(dst), "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)) : "memory");
-}
-// Bulk copy shared -> global (async proxy), tracked by bulk groups of the issuing thread.
-__device__ __forceinline__ void bulk_store(void* gdst, uint32_t src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-                 ::"l"(gdst), "r"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-// 3-D tiled store of a shared-memory box to (c0, c1, c2); tracked by the thread's bulk groups.
-__device__ __forceinline__ void tma_store_3d(const void* tmap, int c0, int c1, int c2, uint32_t src) {
-    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
-                 ::"l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(src) : "memory");
-}
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-// 2^x by the SFU (approximate; inputs here stay within +-116).
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-// Relaxed remote arrive announcing `bytes` of bulk transfers that carry the data themselves.
-__device__ __forceinline__ void mbar_arrive_expect_tx_remote_relaxed(uint32_t cluster_addr, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;"
-                 ::"r"(cluster_addr), "r"(bytes) : "memory");
-}
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-// MMA with the A operand in tensor memory (K-major, two 16-bit elements per 32-bit column,
-// row m in lane m); B from shared memory.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void warp_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    if (elect_one()) mma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, accumulate);
-    __syncwarp();
-}
-// ---- registers -> TMEM: 32 lanes x 32 consecutive 32-bit columns per warp ----
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
-          "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]),
-          "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-          "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() {
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-// 32-bit load from a peer CTA's shared memory (cluster address from map_to_rank).
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
-    return v;
-}
-// Orders this thread's async-proxy global accesses with its generic ones.
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-// Bulk copy global -> this CTA's shared memory, completing on a local mbarrier.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ uint32_t smid() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
-    return r;
-}
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-// 2^x on the FMA pipe, leaving the SFU to other work: x = n + f with n = round(x) (by the
-// 1.5 * 2^23 shifter, exact for |x| < 2^22) and |f| <= 1/2; 2^f by a degree-4 polynomial
-// fitted in relative least squares on [-1/2, 1/2] (max relative error 2.7e-6); 2^n is added
-// to the exponent field. x is clamped to [-125, 125], where the result stays a normal float.
-__device__ __forceinline__ float exp2_fma(float x) {
-    x = fminf(fmaxf(x, -125.f), 125.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    float p = fmaf(f, 0.009560510516166687f, 0.05591703951358795f);
-    p = fmaf(p, f, 0.24024981260299683f);
-    p = fmaf(p, f, 0.6931219696998596f);
-    p = fmaf(p, f, 0.9999991655349731f);
-    const int ni = __float_as_int(t) - 0x4B400000;
-    return __int_as_float(__float_as_int(p) + (ni << 23));
-}
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-// Two 32-column TMEM loads in flight before one wait.
-__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float* va, float* vb) {
-    uint32_t r[64];
-#define KDA_LD32(base, addr)                                                                     \
-    asm volatile(                                                                                \
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                                \
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"                                \
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"               \
-        : "=r"(r[base + 0]), "=r"(r[base + 1]), "=r"(r[base + 2]), "=r"(r[base + 3]),            \
-          "=r"(r[base + 4]), "=r"(r[base + 5]), "=r"(r[base + 6]), "=r"(r[base + 7]),            \
-          "=r"(r[base + 8]), "=r"(r[base + 9]), "=r"(r[base + 10]), "=r"(r[base + 11]),          \
-          "=r"(r[base + 12]), "=r"(r[base + 13]), "=r"(r[base + 14]), "=r"(r[base + 15]),        \
-          "=r"(r[base + 16]), "=r"(r[base + 17]), "=r"(r[base + 18]), "=r"(r[base + 19]),        \
-          "=r"(r[base + 20]), "=r"(r[base + 21]), "=r"(r[base + 22]), "=r"(r[base + 23]),        \
-          "=r"(r[base + 24]), "=r"(r[base + 25]), "=r"(r[base + 26]), "=r"(r[base + 27]),        \
-          "=r"(r[base + 28]), "=r"(r[base + 29]), "=r"(r[base + 30]), "=r"(r[base + 31])         \
-        : "r"(addr))
-    KDA_LD32(0, ta);
-    KDA_LD32(32, tb);
-#undef KDA_LD32
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) { va[i] = __uint_as_float(r[i]); vb[i] = __uint_as_float(r[32 + i]); }
-}
-}  // namespace tc
-}  // namespace kda
-
-namespace kda {
-namespace tc {
-// TMEM <-> registers, 32 lanes x 16 (or 8) consecutive 32-bit columns per warp.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-          "r"(r[7])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
-          "r"(r[14]), "r"(r[15])
-        : "memory");
-}
 }  // namespace tc
 }  // namespace kda

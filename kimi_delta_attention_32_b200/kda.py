@@ -21,7 +21,9 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUD
 KDA_IO_F32, KDA_IO_BF16 = 0, 1
 
 EXPORTED = ("kda_status_string", "kda_version", "kda_conv_fwd", "kda_chunk_fwd_workspace_size",
-            "kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_recurrent_step", "kda_last_device_error")
+            "kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_chunk_fwd_noalloc", "kda_recurrent_step",
+            "kda_conv_recurrent_step", "kda_fused_recurrent_step", "kda_set_wait_limit",
+            "kda_last_device_error")
 
 _lock = threading.Lock()
 _lib = None
@@ -60,12 +62,24 @@ def load_library(path: str = LIB_PATH):
                                       ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci, ci,
                                       ci, vp, cs, vp]
         lib.kda_chunk_fwd.restype = ci
+        lib.kda_chunk_fwd_gated.argtypes = [vp, vp, vp, vp, vp, fp, fp, vp, fp, cf, cf, fp, fp, vp,
+                                            i32p, ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci,
+                                            ci, ci, ci, ci, vp, cs, vp]
+        lib.kda_chunk_fwd_gated.restype = ci
         lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, cf, fp, fp, vp, i32p,
                                               ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci,
                                               ci, ci, vp]
         lib.kda_chunk_fwd_noalloc.restype = ci
         lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, cf, fp, vp, ci, ci, ci, ci, ci, vp]
         lib.kda_recurrent_step.restype = ci
+        lib.kda_conv_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, cf, fp, vp, ci,
+                                                ci, ci, ci, ci, cf, ci, vp]
+        lib.kda_conv_recurrent_step.restype = ci
+        lib.kda_fused_recurrent_step.argtypes = [vp, vp, vp, vp, vp, fp, fp, fp, vp, fp, fp, vp, fp,
+                                                 cf, cf, fp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
+        lib.kda_fused_recurrent_step.restype = ci
+        lib.kda_set_wait_limit.argtypes = [ctypes.c_int64]
+        lib.kda_set_wait_limit.restype = ci
         lib.kda_last_device_error.argtypes = [vp]
         lib.kda_last_device_error.restype = ci
         if path == LIB_PATH:
@@ -168,6 +182,39 @@ def chunk_fwd(q, k, v, g, beta, scale=1.0, h0=None, ht=None, o=None, cu_seqlens=
     return o, ht
 
 
+def chunk_fwd_gated(q, k, v, g_raw, beta_raw, A_log, dt_bias, z=None, w_norm=None, norm_eps=1e-6,
+                    scale=1.0, h0=None, ht=None, o=None, cu_seqlens=None, cu_host=None, chunk=64,
+                    workspace=None, stream=None):
+    """Chunked prefill with g and beta from raw logits (g = -exp(A_log) softplus(g_raw +
+    dt_bias), beta = sigmoid(beta_raw)) and, when z is given, the gated RMSNorm of the output.
+    Layouts as chunk_fwd; g_raw [.., H, dk] and beta_raw [.., H] bf16. Returns (o, ht)."""
+    lib = load_library()
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape if q.dim() == 4 else (1, *q.shape)
+        N, T_tot = B, B * T
+    else:
+        B, T = 1, 0
+        T_tot, H, dk = q.shape
+        N = len(cu_host) - 1
+    dv = v.shape[-1]
+    o = torch.empty_like(v) if o is None else o
+    if ht is None:
+        ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = chunk_fwd_workspace_size(N, T_tot, H, dk, dv, chunk, _io(q))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    keep, cuh = _host_cu(cu_host)
+    st = lib.kda_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(g_raw), _ptr(beta_raw),
+                                 _ptr(A_log), _ptr(dt_bias), _ptr(z), _ptr(w_norm),
+                                 float(norm_eps), float(scale), _ptr(h0), _ptr(ht), _ptr(o),
+                                 _ptr(cu_seqlens), cuh, B, T, N, H, dk, dv, chunk, _io(q),
+                                 _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                 _stream(stream))
+    del keep
+    _check("kda_chunk_fwd_gated", st)
+    return o, ht
+
+
 def chunk_fwd_noalloc(q, k, v, g, beta, scale=1.0, h0=None, ht=None, o=None, cu_seqlens=None,
                       cu_host=None, chunk=64, stream=None):
     """chunk_fwd through kda_chunk_fwd_noalloc: no workspace is allocated for the call (o and
@@ -204,6 +251,49 @@ def recurrent_step(q, k, v, g, beta, state, scale=1.0, o=None, stream=None):
                                 _ptr(state), _ptr(o), N, H, dk, dv, _io(q), _stream(stream))
     _check("kda_recurrent_step", st)
     return o
+
+
+def conv_recurrent_step(q_raw, k_raw, v_raw, w_q, w_k, w_v, conv_state, g, beta, state,
+                        scale=1.0, o=None, l2_eps=1e-6, K=4, stream=None):
+    """One decode token from raw q, k, v: conv (cache advanced in place) + SiLU + L2 norm and
+    the state update in one kernel. Shapes: raw q, k, g [N,H,dk], v [N,H,dv], beta [N,H],
+    conv_state [N, H*(2dk+dv), K-1], state [N,H,dk,dv] fp32 (in place). Returns o [N,H,dv]."""
+    lib = load_library()
+    N, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    o = torch.empty_like(v_raw) if o is None else o
+    st = lib.kda_conv_recurrent_step(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(w_q), _ptr(w_k),
+                                     _ptr(w_v), _ptr(conv_state), _ptr(g), _ptr(beta),
+                                     float(scale), _ptr(state), _ptr(o), N, H, dk, dv, K,
+                                     float(l2_eps), _io(q_raw), _stream(stream))
+    _check("kda_conv_recurrent_step", st)
+    return o
+
+
+def fused_recurrent_step(q_raw, k_raw, v_raw, g_raw, beta_raw, w_q, w_k, w_v, conv_state, A_log,
+                         dt_bias, state, z=None, w_norm=None, norm_eps=1e-6, scale=1.0, o=None,
+                         l2_eps=1e-6, K=4, stream=None):
+    """The whole decode step from raw projections: conv (cache in place), gate and beta from raw
+    logits, state update, and the gated RMSNorm of the output when z is given. Shapes: raw q, k,
+    g [N,H,dk], v, z [N,H,dv], beta_raw [N,H]; A_log [H], dt_bias [H*dk], w_norm [dv].
+    Returns o [N,H,dv]."""
+    lib = load_library()
+    N, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    o = torch.empty_like(v_raw) if o is None else o
+    st = lib.kda_fused_recurrent_step(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(g_raw),
+                                      _ptr(beta_raw), _ptr(w_q), _ptr(w_k), _ptr(w_v),
+                                      _ptr(conv_state), _ptr(A_log), _ptr(dt_bias), _ptr(z),
+                                      _ptr(w_norm), float(norm_eps), float(scale), _ptr(state),
+                                      _ptr(o), N, H, dk, dv, K, float(l2_eps), _io(q_raw),
+                                      _stream(stream))
+    _check("kda_fused_recurrent_step", st)
+    return o
+
+
+def set_wait_limit(cycles: int) -> None:
+    """Bound (SM cycles) of every device-side wait of later prefill launches; 0 = default."""
+    _check("kda_set_wait_limit", load_library().kda_set_wait_limit(int(cycles)))
 
 
 def last_device_error(stream=None) -> int:

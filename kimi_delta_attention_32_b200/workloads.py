@@ -16,6 +16,11 @@ Distributions (one reading of each workload, see the design notes):
            (exp(g) < 0.5);
   h0     = 0, or N(0, 0.02) fp32 where the workload says so;
   conv weights ~ N(0, 0.5) fp32, shape [H*d, 4].
+Raw projections for the fully fused entry points (their own generator, seed + 100, so the
+fields above keep their values): gate logits g_raw = -u, u ~ N(4, 1), with A_log ~ N(0, 0.1)
+per head and dt_bias ~ N(0, 0.1) per key channel (so -exp(A_log) softplus(g_raw + dt_bias)
+follows the g recipe above); beta logits ~ N(0, 1); output-norm gate z ~ N(0, 1) and weight
+w_norm ~ N(1, 0.1) [dv].
 N(m, s) means mean m and standard deviation s.
 """
 from __future__ import annotations
@@ -125,12 +130,14 @@ def _log_decay(shape, gen, device, skew_channels=0, head_axis=-2):
     return -F.softplus(-u)
 
 
-def make_prefill(wl: Workload, device="cpu", T: int | None = None, lengths=None) -> dict:
+def make_prefill(wl: Workload, device="cpu", T: int | None = None, lengths=None,
+                 raw: bool = False) -> dict:
     """Inputs of one prefill call (padded as one packed batch when varlen is empty).
 
     Returns a dict with q, k, v (io dtype), g, beta (fp32), h0 (fp32 or None),
     cu_seqlens (int32 tensor on device), cu_host (list), and for prologue workloads
-    q_raw/k_raw/v_raw and w_q/w_k/w_v instead of q/k/v being normalised.
+    q_raw/k_raw/v_raw and w_q/w_k/w_v instead of q/k/v being normalised. raw=True adds the raw
+    projections of the fused entry points (g_raw, beta_raw, A_log, dt_bias, z, w_norm).
     """
     gen = _gen(device, wl.seed)
     dt = io_dtype(wl.io)
@@ -160,6 +167,8 @@ def make_prefill(wl: Workload, device="cpu", T: int | None = None, lengths=None)
     d["g"] = _log_decay((T_tot, H, dk), gen, device, wl.skew_channels)
     d["h0"] = (_randn((len(lengths), H, dk, dv), gen, device, std=wl.h0_std)
                if wl.h0_std > 0 else None)
+    if raw:
+        d.update(_raw_projections((T_tot, H), H, dk, dv, dt, device, wl.seed))
     return d
 
 
@@ -181,4 +190,16 @@ def make_decode(wl: Workload, device="cpu", N: int | None = None, steps: int | N
     d["v_raw"] = _randn((steps, N, H, dv), gen, device, dtype=dt)
     d["beta"] = torch.sigmoid(_randn((steps, N, H), gen, device))
     d["g"] = _log_decay((steps, N, H, dk), gen, device)
+    d.update(_raw_projections((steps, N, H), H, dk, dv, dt, device, wl.seed))
     return d
+
+
+def _raw_projections(lead, H, dk, dv, dt, device, seed) -> dict:
+    """Raw gate and beta logits, A_log, dt_bias, and the output norm's gate and weight."""
+    gen = _gen(device, seed + 100)
+    return {"g_raw": _randn((*lead, dk), gen, device, mean=-4.0, dtype=dt),
+            "beta_raw": _randn(lead, gen, device, dtype=dt),
+            "A_log": _randn((H,), gen, device, std=0.1),
+            "dt_bias": _randn((H * dk,), gen, device, std=0.1),
+            "z": _randn((*lead, dv), gen, device, dtype=dt),
+            "w_norm": _randn((dv,), gen, device, mean=1.0, std=0.1)}

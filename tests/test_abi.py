@@ -149,11 +149,79 @@ def test_workspace_query(lib):
         kda.KDA_ERR_INVALID_ARG
 
 
-def test_chunk_fwd_checks_workspace(lib, monkeypatch):
-    monkeypatch.delenv("KDA_CHUNK_KERNEL", raising=False)
+def test_wait_limit_checks_its_argument(lib):
+    assert lib.kda_set_wait_limit(-1) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_set_wait_limit(123456) == kda.KDA_OK
+    assert lib.kda_set_wait_limit(0) == kda.KDA_OK
+
+
+def test_chunk_fwd_checks_workspace(lib):
     out = ctypes.c_size_t(0)
     assert lib.kda_chunk_fwd_workspace_size(1, 64, 2, 128, 128, 64, 1, ctypes.byref(out)) == 0
     need = out.value
     assert _chunk(lib) == kda.KDA_ERR_WORKSPACE                          # missing
     assert _chunk(lib, ws=MIS, wsb=need) == kda.KDA_ERR_WORKSPACE         # misaligned
     assert _chunk(lib, ws=FAKE, wsb=need - 16) == kda.KDA_ERR_WORKSPACE   # too small
+
+
+def _fused_step(lib, **kw):
+    a = dict(qr=FAKE, kr=FAKE, vr=FAKE, gr=FAKE, br=FAKE, wq=FAKE, wk=FAKE, wv=FAKE, cs=FAKE,
+             A=FAKE, dt=FAKE, z=None, wn=None, neps=1e-6, scale=1.0, state=FAKE, o=FAKE, N=2,
+             H=2, dk=128, dv=128, K=4, eps=1e-6, io=1, stream=None)
+    a.update(kw)
+    return lib.kda_fused_recurrent_step(a["qr"], a["kr"], a["vr"], a["gr"], a["br"], a["wq"],
+                                        a["wk"], a["wv"], a["cs"], a["A"], a["dt"], a["z"],
+                                        a["wn"], a["neps"], a["scale"], a["state"], a["o"], a["N"],
+                                        a["H"], a["dk"], a["dv"], a["K"], a["eps"], a["io"],
+                                        a["stream"])
+
+
+def _conv_step(lib, **kw):
+    a = dict(qr=FAKE, kr=FAKE, vr=FAKE, wq=FAKE, wk=FAKE, wv=FAKE, cs=FAKE, g=FAKE, b=FAKE,
+             scale=1.0, state=FAKE, o=FAKE, N=2, H=2, dk=128, dv=128, K=4, eps=1e-6, io=1,
+             stream=None)
+    a.update(kw)
+    return lib.kda_conv_recurrent_step(a["qr"], a["kr"], a["vr"], a["wq"], a["wk"], a["wv"],
+                                       a["cs"], a["g"], a["b"], a["scale"], a["state"], a["o"],
+                                       a["N"], a["H"], a["dk"], a["dv"], a["K"], a["eps"],
+                                       a["io"], a["stream"])
+
+
+def test_fused_decode_entry_points_check_arguments(lib):
+    for fn in (_fused_step, _conv_step):
+        assert fn(lib, cs=None) == kda.KDA_ERR_INVALID_ARG          # the conv history is required
+        assert fn(lib, qr=MIS) == kda.KDA_ERR_INVALID_ARG
+        assert fn(lib, K=1) == kda.KDA_ERR_INVALID_ARG
+        assert fn(lib, K=3) == kda.KDA_ERR_UNSUPPORTED
+        assert fn(lib, dk=96) == kda.KDA_ERR_UNSUPPORTED
+        assert fn(lib, eps=-1.0) == kda.KDA_ERR_INVALID_ARG
+        assert fn(lib, H=0) == kda.KDA_ERR_INVALID_ARG
+        assert fn(lib, io=7) == kda.KDA_ERR_INVALID_ARG
+    assert _fused_step(lib, A=None) == kda.KDA_ERR_INVALID_ARG
+    assert _fused_step(lib, dt=None) == kda.KDA_ERR_INVALID_ARG
+    assert _fused_step(lib, z=FAKE) == kda.KDA_ERR_INVALID_ARG       # a norm gate without weight
+    assert _fused_step(lib, br=ctypes.c_void_p(0x10001)) == kda.KDA_ERR_INVALID_ARG
+
+
+def _gated(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, gr=FAKE, br=FAKE, A=FAKE, dt=FAKE, z=None, wn=None,
+             neps=1e-6, scale=1.0, h0=None, ht=None, o=FAKE, cu=None, cuh=None, B=1, T=64, N=1,
+             H=2, dk=128, dv=128, chunk=64, io=1, ws=FAKE, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return lib.kda_chunk_fwd_gated(a["q"], a["k"], a["v"], a["gr"], a["br"], a["A"], a["dt"],
+                                   a["z"], a["wn"], a["neps"], a["scale"], a["h0"], a["ht"],
+                                   a["o"], a["cu"], a["cuh"], a["B"], a["T"], a["N"], a["H"],
+                                   a["dk"], a["dv"], a["chunk"], a["io"], a["ws"], a["wsb"],
+                                   a["stream"])
+
+
+def test_gated_prefill_checks_arguments(lib):
+    assert _gated(lib, gr=None) == kda.KDA_ERR_INVALID_ARG
+    assert _gated(lib, A=None) == kda.KDA_ERR_INVALID_ARG
+    assert _gated(lib, dt=None) == kda.KDA_ERR_INVALID_ARG
+    assert _gated(lib, br=ctypes.c_void_p(0x10001)) == kda.KDA_ERR_INVALID_ARG
+    assert _gated(lib, z=FAKE) == kda.KDA_ERR_INVALID_ARG           # a norm gate without weight
+    assert _gated(lib, chunk=0) == kda.KDA_ERR_INVALID_ARG
+    assert _gated(lib, io=0) == kda.KDA_ERR_UNSUPPORTED              # tensor-core path only
+    assert _gated(lib, dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
+    assert _gated(lib, ws=None) == kda.KDA_ERR_WORKSPACE
