@@ -464,12 +464,43 @@ def _prefill_row(torch, kda, dev, flush, hbm_peak, stream, name, with_prologue=F
             conv()
             chunk()
         ms2 = statistics.mean(_events_time(torch, both, steps, 2, flush=flush, stream=stream))
-        # the config's own bytes: raw q/k/v in instead of the normalised ones (same size)
-        row.update({"conv_plus_chunk_ms": ms2, "tokens/s": T_tot / ms2 * 1e3,
-                    "frac_hbm": algo / ms2 / 1e6 / hbm_peak})
+
+        def fused():
+            kda.chunk_fwd_fused(d["q_raw"], d["k_raw"], d["v_raw"], d["g"], d["beta"], w_q=d["w_q"],
+                                w_k=d["w_k"], w_v=d["w_v"], h0=d["h0"], ht=ht, o=o,
+                                cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], workspace=ws,
+                                stream=stream)
+        ms3 = statistics.mean(_events_time(torch, fused, steps, 2, flush=flush, stream=stream))
+        # the config's own bytes: raw q/k/v in instead of the normalised ones (same size); the
+        # headline of the row is the prefill with the prologue fused in, as the config states
+        row.update({"conv_then_chunk_ms": ms2, "fused_ms": ms3, "tokens/s": T_tot / ms3 * 1e3,
+                    "frac_hbm": algo / ms3 / 1e6 / hbm_peak,
+                    "conv_then_chunk_frac_hbm": algo / ms2 / 1e6 / hbm_peak})
     else:
         row.update({"tokens/s": T_tot / ms * 1e3, "frac_hbm": algo / ms / 1e6 / hbm_peak})
     return row
+
+
+def _gated_row(torch, kda, dev, flush, hbm_peak, stream, steps=5):
+    """prefill_8k's shape with the gate and beta from raw bf16 logits and the gated RMSNorm of
+    the output fused in: bytes per token*head are q, k, v, o (4 * 256) + raw gate logits (256) +
+    raw beta (2) + the norm's gate z (256)."""
+    from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_prefill
+    d = make_prefill(WORKLOADS["prefill_8k"], dev, raw=True)
+    T_tot, N, H, dk, dv = d["T_tot"], d["N"], d["H"], d["dk"], d["dv"]
+    o = torch.empty_like(d["v"])
+    ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(kda.chunk_fwd_workspace_size(N, T_tot, H, dk, dv), dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.chunk_fwd_fused(d["q"], d["k"], d["v"], g_raw=d["g_raw"], beta_raw=d["beta_raw"],
+                            A_log=d["A_log"], dt_bias=d["dt_bias"], z=d["z"], w_norm=d["w_norm"],
+                            ht=ht, o=o, workspace=ws, stream=stream)
+    ms = statistics.mean(_events_time(torch, step, steps, 2, flush=flush, stream=stream))
+    algo = T_tot * H * (4 * 256 + 256 + 2 + 256) + N * H * dk * dv * 4
+    return {"workload": "prefill_8k shape, gate and beta from raw bf16 logits, gated RMSNorm output",
+            "ms": ms, "tokens/s": T_tot / ms * 1e3, "algorithmic_bytes": algo,
+            "frac_hbm": algo / ms / 1e6 / hbm_peak}
 
 
 def measure_rows(torch, kda, dev, flush, hbm_peak, stream):
@@ -499,6 +530,8 @@ def measure_rows(torch, kda, dev, flush, hbm_peak, stream):
                                           "varlen_prologue", with_prologue=True, steps=3)
     torch.cuda.empty_cache()
     out["long_256k"] = _prefill_row(torch, kda, dev, flush, hbm_peak, stream, "long_256k", steps=3)
+    torch.cuda.empty_cache()
+    out["prefill_8k_gated_norm"] = _gated_row(torch, kda, dev, flush, hbm_peak, stream)
     torch.cuda.empty_cache()
 
     wl = WORKLOADS["decode_256x32"]

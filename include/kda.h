@@ -107,7 +107,7 @@ kda_status kda_conv_fwd(const void* q_raw, const void* k_raw, const void* v_raw,
  * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd needs
  * for these sizes (written to *bytes, host). Zero means none; the call then
  * accepts workspace == NULL. The bf16, dk = dv = 128, chunk-64 prefill needs a
- * fixed ~56.0 MB whatever the batch: per-SM hand-off rings through which the
+ * fixed ~71.8 MB whatever the batch: per-SM hand-off rings through which the
  * kernel's producer CTAs pass each chunk's operands to its consumer CTA via L2.
  * The contents need no initialisation and are dead after the call; one
  * workspace may serve consecutive calls on one stream, not concurrent ones.
@@ -134,7 +134,8 @@ kda_status kda_chunk_fwd_workspace_size(int N, int64_t T_tot, int H, int dk, int
  *  workspace: device memory of at least kda_chunk_fwd_workspace_size() bytes,
  *         16-byte aligned, owned by the caller (KDA_ERR_WORKSPACE otherwise);
  *         may be NULL when that size is 0.
- *  Supported: dk == dv in {64, 128} for io F32; dk == dv == 128 or 64 for BF16.
+ *  Supported: dk, dv each in {64, 128}, chunk 64 (bf16 with dk = dv = 128 runs on the tensor
+ *  cores, every other combination on CUDA cores in fp32).
  *  Empty sequences are allowed (their final state is the initial state).
  */
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
@@ -145,28 +146,39 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          void* stream);
 
 /*
- * kda_chunk_fwd_gated -- kda_chunk_fwd with the gate and beta formed from raw logits inside the
- * kernel, and optionally the gated RMSNorm of the output before it is stored.
- * (m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...": the gate is computed from
- *  a_log_bias and dt_bias, delta is the residual times sigmoid(beta); sarnas.ru, section
- *  "Отвергнутые решения": every norm except the QK norms is a gated RMSNorm.)
+ * kda_chunk_fwd_fused -- kda_chunk_fwd with the surrounding steps of the KDA layer fused into the
+ * prefill kernel, each optional:
+ *  - conv prologue (w_q, w_k, w_v given): q, k, v are the RAW projections; each is passed
+ *    through the kernel-4 causal depthwise conv and SiLU, and q, k through the L2 norm, exactly
+ *    as kda_conv_fwd computes them, in the producers' load stage (no HBM round trip). The history
+ *    before each sequence is conv_state (or zero when NULL); when conv_state is given it is
+ *    overwritten with the new history afterwards (the last K-1 raw inputs, as kda_conv_fwd does).
+ *  - gate from raw logits (g_raw given): g = -exp(A_log[h]) * softplus(g_raw + dt_bias[h, c]) and
+ *    beta = sigmoid(beta_raw), in the producers' fold; otherwise g and beta are taken as given.
+ *  - gated RMSNorm of the output (z given): o' = o / sqrt(mean_j o_j^2 + norm_eps) * w_norm *
+ *    sigmoid(z), before the store.
+ * (m.lqnn.cn/news/205170, section "KDA 与 Gated Attention ...": kernel-4 causal conv with a
+ *  cache, the gate from a_log_bias and dt_bias, delta = residual * sigmoid(beta); sarnas.ru,
+ *  section "Отвергнутые решения": every norm except the QK norms is a gated RMSNorm.)
  *
- *     g[t, h, c]  = -exp(A_log[h]) * softplus(g_raw[t, h, c] + dt_bias[h * dk + c])
- *     beta[t, h]  = sigmoid(beta_raw[t, h])
- *     o'[t, h, :] = o / sqrt(mean_j o_j^2 + norm_eps) * w_norm * sigmoid(z[t, h, :])   (z != NULL)
- *
- *  g_raw : [T_tot, H, dk] bf16      beta_raw : [T_tot, H] bf16 (2-byte aligned)
- *  A_log : [H] fp32                 dt_bias  : [H*dk] fp32
- *  z     : [T_tot, H, dv] bf16 or NULL (no output norm)    w_norm : [dv] fp32 (with z)
+ *  q, k, v     : as kda_chunk_fwd (raw projections with the conv)
+ *  w_q, w_k, w_v: [H*d, K] fp32 conv weights, all NULL or all given; conv_state: [N, H*(2dk+dv),
+ *                K-1] bf16 or NULL (only with the conv); l2_eps: the q, k L2-norm epsilon
+ *  g, beta     : as kda_chunk_fwd, used when g_raw is NULL
+ *  g_raw       : [T_tot, H, dk] bf16   beta_raw : [T_tot, H] bf16 (2-byte aligned)
+ *  A_log       : [H] fp32              dt_bias  : [H*dk] fp32 (with g_raw)
+ *  z           : [T_tot, H, dv] bf16 or NULL        w_norm : [dv] fp32 (with z)
  *  other arguments, the workspace and the errors as for kda_chunk_fwd.
- *  Supported: bf16 I/O, dk == dv == 128, chunk 64 (KDA_ERR_UNSUPPORTED otherwise).
+ *  Supported: bf16 I/O, dk == dv == 128, chunk 64, K == 4 (KDA_ERR_UNSUPPORTED otherwise).
  */
-kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v, const void* g_raw,
+kda_status kda_chunk_fwd_fused(const void* q, const void* k, const void* v, const float* w_q,
+                               const float* w_k, const float* w_v, const void* conv_state,
+                               float l2_eps, const float* g, const float* beta, const void* g_raw,
                                const void* beta_raw, const float* A_log, const float* dt_bias,
                                const void* z, const float* w_norm, float norm_eps, float scale,
                                const float* h0, float* ht, void* o, const int32_t* cu_seqlens,
-                               const int32_t* cu_seqlens_host, int B, int T, int N, int H,
-                               int dk, int dv, int chunk, kda_io_dtype io, void* workspace,
+                               const int32_t* cu_seqlens_host, int B, int T, int N, int H, int dk,
+                               int dv, int K, int chunk, kda_io_dtype io, void* workspace,
                                size_t workspace_bytes, void* stream);
 
 /*

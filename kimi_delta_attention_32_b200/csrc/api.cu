@@ -129,7 +129,7 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
         if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
     if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
     if (!ok_opt(h0) || !ok_opt(ht) || !ok_opt(cu_seqlens)) return KDA_ERR_INVALID_ARG;
-    if (chunk != 64 || dk != dv || !head_dim_ok(dk)) return KDA_ERR_UNSUPPORTED;
+    if (chunk != 64 || !head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
     kda::ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.scale = scale;
     a.h0 = h0; a.ht = ht; a.o = o;
@@ -150,47 +150,75 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
     return from_cuda(kda::launch_chunk_simt(a, static_cast<cudaStream_t>(stream)));
 }
 
-KDA_API kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v,
-                                       const void* g_raw, const void* beta_raw, const float* A_log,
-                                       const float* dt_bias, const void* z, const float* w_norm,
-                                       float norm_eps, float scale, const float* h0, float* ht,
-                                       void* o, const int32_t* cu_seqlens,
-                                       const int32_t* cu_seqlens_host, int B, int T, int N, int H,
-                                       int dk, int dv, int chunk, kda_io_dtype io, void* workspace,
-                                       size_t workspace_bytes, void* stream) {
+KDA_API kda_status kda_chunk_fwd_fused(
+    const void* q, const void* k, const void* v, const float* w_q, const float* w_k,
+    const float* w_v, const void* conv_state, float l2_eps, const float* g, const float* beta,
+    const void* g_raw, const void* beta_raw, const float* A_log, const float* dt_bias,
+    const void* z, const float* w_norm, float norm_eps, float scale, const float* h0, float* ht,
+    void* o, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int B, int T, int N,
+    int H, int dk, int dv, int K, int chunk, kda_io_dtype io, void* workspace,
+    size_t workspace_bytes, void* stream) {
     if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
-    if (H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0) return KDA_ERR_INVALID_ARG;
+    if (H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0 || K < 2) return KDA_ERR_INVALID_ARG;
     int64_t T_tot = 0;
     int Nn = 0;
     if (!batch_geometry(cu_seqlens, cu_seqlens_host, B, T, N, &T_tot, &Nn)) return KDA_ERR_INVALID_ARG;
-    const void* req[] = {q, k, v, g_raw, o};
+    const void* req[] = {q, k, v, o};
     for (const void* p : req)
         if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
-    if (A_log == nullptr || !aligned4(A_log) || dt_bias == nullptr || !aligned4(dt_bias))
+    if (!ok_opt(h0) || !ok_opt(ht) || !ok_opt(cu_seqlens) || !ok_opt(z) || !ok_opt(conv_state))
         return KDA_ERR_INVALID_ARG;
-    if (beta_raw == nullptr || (reinterpret_cast<uintptr_t>(beta_raw) & 1u) != 0)   // bf16 elements
+    const bool conv = (w_q != nullptr || w_k != nullptr || w_v != nullptr);
+    if (conv && (!ok_req(w_q) || !ok_req(w_k) || !ok_req(w_v) || !(l2_eps >= 0.f)))
         return KDA_ERR_INVALID_ARG;
-    if (!ok_opt(h0) || !ok_opt(ht) || !ok_opt(cu_seqlens) || !ok_opt(z)) return KDA_ERR_INVALID_ARG;
+    if (!conv && conv_state != nullptr) return KDA_ERR_INVALID_ARG;
+    const bool gate = (g_raw != nullptr);
+    if (gate) {
+        if (!ok_req(g_raw) || A_log == nullptr || !aligned4(A_log) || dt_bias == nullptr ||
+            !aligned4(dt_bias) || beta_raw == nullptr || (reinterpret_cast<uintptr_t>(beta_raw) & 1u) != 0)
+            return KDA_ERR_INVALID_ARG;
+    } else if (!ok_req(g) || beta == nullptr || !aligned4(beta)) {
+        return KDA_ERR_INVALID_ARG;
+    }
     if (z != nullptr && (w_norm == nullptr || !aligned4(w_norm) || !(norm_eps >= 0.f)))
         return KDA_ERR_INVALID_ARG;
     kda::ChunkArgs a;
-    a.q = q; a.k = k; a.v = v; a.g = nullptr; a.beta = nullptr; a.scale = scale;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.scale = scale;
     a.h0 = h0; a.ht = ht; a.o = o;
     a.cu = cu_seqlens; a.cu_host = cu_seqlens_host;
     a.T_tot = T_tot;
     a.T_pad = cu_seqlens ? 0 : T;
     a.N = Nn; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk;
     a.io = io == KDA_IO_BF16 ? kda::Io::BF16 : kda::Io::F32;
-    a.g_raw = g_raw; a.beta_raw = beta_raw; a.A_log = A_log; a.dt_bias = dt_bias;
+    if (gate) { a.g_raw = g_raw; a.beta_raw = beta_raw; a.A_log = A_log; a.dt_bias = dt_bias; }
     a.z = z; a.w_norm = w_norm; a.norm_eps = norm_eps;
-    if (!kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
+    if (conv) {
+        a.wconv[0] = w_q; a.wconv[1] = w_k; a.wconv[2] = w_v;
+        a.conv_state = conv_state;
+        a.l2_eps = l2_eps;
+    }
+    if (!kda::chunk_tc_supported(a) || K != 4) return KDA_ERR_UNSUPPORTED;
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0 ||
         workspace_bytes < kda::chunk_tcx_workspace_bytes())
         return KDA_ERR_WORKSPACE;
     unsigned int* err = device_error_word();
     if (err == nullptr) return KDA_ERR_CUDA;
-    return from_cuda(kda::launch_chunk_tcx(a, workspace, workspace_bytes, err,
-                                           static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = kda::launch_chunk_tcx(a, workspace, workspace_bytes, err, st);
+    if (e != cudaSuccess || !conv || conv_state == nullptr) return from_cuda(e);
+    // the new conv cache: the last three raw inputs of each sequence's history
+    kda::ConvArgs c;
+    c.x[0] = q; c.x[1] = k; c.x[2] = v;
+    c.w[0] = w_q; c.w[1] = w_k; c.w[2] = w_v;
+    c.y[0] = c.y[1] = c.y[2] = nullptr;
+    c.conv_state = const_cast<void*>(conv_state);
+    c.cu = cu_seqlens;
+    c.T_tot = T_tot;
+    c.T_pad = cu_seqlens ? 0 : T;
+    c.N = Nn; c.H = H; c.dk = dk; c.dv = dv;
+    c.eps = l2_eps;
+    c.io = a.io;
+    return from_cuda(kda::launch_conv_cache(c, st));
 }
 
 KDA_API kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,

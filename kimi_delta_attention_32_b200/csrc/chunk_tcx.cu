@@ -32,12 +32,15 @@
 // Sm (M = 128 token rows, N = 64), U = V - X, then the state delta Yh^T U and the output term
 // Wh^T U; the fp32 state stays in registers (thread = key channel x 32 value columns).
 //
-// Two compile-time variants serve kda_chunk_fwd_gated. kGate: the producers form g from raw
+// Compile-time variants serve kda_chunk_fwd_fused. kGate: the producers form g from raw
 // gate logits, g = -exp(A_log[h]) softplus(x + dt_bias) (m.lqnn.cn/news/205170: the gate comes
 // from a_log_bias and dt_bias), in the fold, and beta = sigmoid(b) from raw logits. kNorm: the
 // consumer's output warps apply the gated RMSNorm o / sqrt(mean(o^2) + eps) * w * sigmoid(z)
 // (sarnas.ru, section "Отвергнутые решения") before the store, the two value halves exchanging
-// their per-token sums of squares through shared memory.
+// their per-token sums of squares through shared memory. kConv: q, k, v arrive raw; the
+// producers load them with a 3-token halo and apply the causal depthwise conv (kernel 4), SiLU
+// and the L2 norm of q, k in shared memory before the fold (m.lqnn.cn/news/205170: q/k/v pass a
+// kernel-4 causal conv), and send v after the conv with the chunk's factors.
 //
 // Every wait is bounded (a launch parameter); a wait that gives up sets the error word, and the
 // CTA leaves its loop, waits for its own copies and products in flight, and frees its tensor
@@ -66,7 +69,8 @@ constexpr int kCluster = 1 + kProducers;
 constexpr float kHalfRange = 80.f;       // largest natural-log decay allowed per half chunk
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr long long kDefaultWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
-constexpr int kGate = 1, kNorm = 2;      // variant bits
+constexpr int kGate = 1, kNorm = 2, kConv = 4;   // variant bits
+constexpr int kHalo = 3;                 // kConv: the conv's three earlier tokens
 constexpr float kLn2 = 0.6931471805599453f;
 
 // ---- one chunk's hand-off (identical image in a global ring slot and the consumer's slots) ----
@@ -75,31 +79,40 @@ constexpr uint32_t S_FAC = 32768;        // e^{gamma_ref}[128], e^{gamma_C}[128]
 constexpr uint32_t kAPart = 33792;       // [Lk ; Lq | factors]
 constexpr uint32_t S_YW = kAPart;        // [Yh^T (rows key ch 0..127) ; Wh^T (rows token)]: K-major
 constexpr uint32_t kBPart = 24576;
-constexpr uint32_t kSlotBytes = kAPart + kBPart;
+constexpr uint32_t S_V = kAPart + kBPart;   // kConv: V after the conv, [half][token][64 ch] SW128
+constexpr uint32_t kVPart = 16384;
+constexpr uint32_t kSlotBytes = kAPart + kBPart + kVPart;
 constexpr int kRing = kTcxRingSlots;
 static_assert(kSlotBytes == kTcxSlotBytes, "slot size");
 static_assert(kAPart % 1024 == 0 && kBPart % 1024 == 0, "slot parts stay swizzle-atom aligned");
 
 // ---- producer shared memory ----
-constexpr uint32_t P_Q = 0;              // raw q tile [64][128] bf16 (TMA, unswizzled)
-constexpr uint32_t P_K = 16384;          // raw k tile
-constexpr uint32_t P_G = 32768;          // raw g tile [64][128] fp32
-constexpr uint32_t P_LKQ = 65536;        // [Lk ; Lq | factors]: the slot's A part image
+constexpr uint32_t kRawTile = 17408;     // 68 token rows of 256 B: 64, after 3 halo rows with kConv
+constexpr uint32_t P_Q = 0;              // q tile [rows][128] bf16 (TMA, unswizzled); with kConv
+                                         //   raw, then overwritten by the conv's output
+constexpr uint32_t P_K = kRawTile;       // k tile, the same
+constexpr uint32_t P_V = 2 * kRawTile;   // kConv: raw v tile
+constexpr uint32_t P_G = 3 * kRawTile;   // g tile [64][128] fp32 (kGate: bf16 logits); with kConv
+                                         //   v after the conv (the slot's V part) once g is read
+constexpr uint32_t P_LKQ = P_G + 32768;  // [Lk ; Lq | factors]: the slot's A part image
 constexpr uint32_t P_R = P_LKQ + kAPart; // R: K-major, 2 atom columns x 64 token rows
 constexpr uint32_t P_PO = P_R + 16384;   // P': K-major, 64 token rows x 64 (A of Wh^T; its M = 128
                                          //     padding rows read T' and give unused rows)
 constexpr uint32_t P_TP = P_PO + 8192;   // T': rows r (K), 64 columns i (N): MN-major B
 constexpr int kLd = 68;                  // fp32 row stride of the 64 x 64 inverse scratch
 constexpr int kLdY = 24;                 // row stride of the per-warp 16 x 16 products
-constexpr uint32_t P_NM = P_TP + 8192;   // N = diag(beta) A (fp32 [64][kLd])
+constexpr uint32_t P_NM = P_TP + 8192;   // N = diag(beta) A (fp32 [64][kLd]); during the fold the
+                                         //   per-warp decay sums [16][128]
 constexpr uint32_t P_TM = P_NM + 64 * kLd * 4;   // T (fp32 [64][kLd])
 constexpr uint32_t P_Y = P_TM + 64 * kLd * 4;    // [4][16][kLdY] fp32
 constexpr uint32_t P_ST = ((P_Y + 4 * 16 * kLdY * 4 + 1023) / 1024) * 1024;   // [Yh^T ; Wh^T] staging
 constexpr uint32_t P_GX = P_TM;          // exact path: natural-log gamma fp32 [64][128] (32 KB over
                                          //   T, Y and the staging, all idle at that point)
 constexpr uint32_t P_MISC = P_ST + kBPart;
-static_assert(P_R % 1024 == 0 && P_PO % 1024 == 0 && P_TP % 1024 == 0 && P_ST % 1024 == 0,
-              "operand tiles are swizzle-atom aligned");
+static_assert(P_LKQ % 1024 == 0 && P_R % 1024 == 0 && P_PO % 1024 == 0 && P_TP % 1024 == 0 &&
+              P_ST % 1024 == 0, "operand tiles are swizzle-atom aligned");
+static_assert((kC + kHalo) * 256 <= kRawTile && 2 * kVPart / 2 <= 32768 && 16 * 128 * 4 <= 64 * kLd * 4,
+              "tile and scratch sizes");
 static_assert(P_GX + 64 * 128 * 4 <= P_MISC, "exact-path scratch");
 
 // ---- consumer shared memory ----
@@ -125,8 +138,7 @@ constexpr uint32_t M_BETA = 512;      // beta[64]
 constexpr uint32_t M_GA = 768;        // gamma at token 31, per channel (log2 units)
 constexpr uint32_t M_GC = 1280;       // gamma at token 63 (log2 units)
 constexpr uint32_t M_RHF = 1792;      // e^{gamma_C - gamma_s} per channel
-constexpr uint32_t M_WSUM = 2304;     // [16 warps][128] decay sums, then their exclusive prefix
-constexpr uint32_t M_DT = M_WSUM + 16 * 128 * 4;   // kGate: dt_bias of this head [128]
+constexpr uint32_t M_DT = 2304;       // kGate: dt_bias of this head [128]
 constexpr uint32_t kMiscP = M_DT + 512;
 // consumer barriers ([X ; O] and delta per half; A, B parts per slot; V per half and slot)
 constexpr uint32_t M_XO = 0, M_DS = 16, M_AFULL = 32, M_BFULL = 48, M_AFREE = 64, M_BFREE = 80,
@@ -180,6 +192,11 @@ struct Params {
     const __nv_bfloat16* z;
     const float* w_norm;
     float norm_eps;
+    // kConv: q, k, v are raw (tq, tk, tv map them in 67-token boxes from 3 tokens back); conv
+    // weights [H*128, 4] of q, k, v; the conv history [N, H*384, 3] (or null: zero); L2 epsilon
+    const float* wconv[3];
+    const __nv_bfloat16* conv_state;
+    float l2_eps;
 };
 
 // softplus(x) = log(1 + e^x) = max(x, 0) + log(1 + e^-|x|), one ex2 and one lg2 on the SFU
@@ -192,6 +209,14 @@ __device__ __forceinline__ float softplus_fast(float x) {
     return fmaxf(x, 0.f) + l * kLn2;
 }
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+// silu(z) = z sigmoid(z) = h + h tanh(h), h = z / 2: one tanh.approx (relative error below 2^-10,
+// under the bf16 rounding of its result).
+__device__ __forceinline__ float silu_fast(float z) {
+    const float hz = 0.5f * z;
+    float th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hz));
+    return fmaf(hz, th, hz);
+}
 
 __device__ __forceinline__ void st16(uint8_t* base, uint32_t off, uint4 v) {
     *reinterpret_cast<uint4*>(base + off) = v;
@@ -265,7 +290,7 @@ __device__ void unit_of(const Params& p, int unit, int* s_tmp, int& n, int& h, i
 
 // Exact A and P on CUDA cores for a chunk whose decay fails the range test: natural-log gamma
 // from the global g (thread = channel), then one warp per (r, i) pair with lanes over channels,
-// reading q and k from global memory. Writes N = diag(beta) A into the inverse's scratch and P
+// reading q and k from the chunk's shared tiles (kept until the exact path is done). Writes N = diag(beta) A into the inverse's scratch and P
 // into its operand. Rare, so kept out of line. Every compute thread calls it.
 template <int MODE>
 __device__ __noinline__ void exact_ap(const Params& p, uint8_t* sm, const float* s_beta, int h,
@@ -298,9 +323,10 @@ __device__ __noinline__ void exact_ap(const Params& p, uint8_t* sm, const float*
         const int i = pidx - r * (r + 1) / 2;
         float a = 0.f, pp = 0.f;
         if (r < L) {
-            const __nv_bfloat16* kr = p.k + (c0 + r) * rs + (int64_t)h * kD;
-            const __nv_bfloat16* qr = p.q + (c0 + r) * rs + (int64_t)h * kD;
-            const __nv_bfloat16* ki = p.k + (c0 + i) * rs + (int64_t)h * kD;
+            constexpr int halo = (MODE & kConv) != 0 ? kHalo : 0;
+            const __nv_bfloat16* kr = reinterpret_cast<const __nv_bfloat16*>(sm + P_K) + (r + halo) * kD;
+            const __nv_bfloat16* qr = reinterpret_cast<const __nv_bfloat16*>(sm + P_Q) + (r + halo) * kD;
+            const __nv_bfloat16* ki = reinterpret_cast<const __nv_bfloat16*>(sm + P_K) + (i + halo) * kD;
             for (int cc = lane; cc < kD; cc += 32) {
                 const float kd = __bfloat162float(ki[cc]) * expf(Gx[r * kD + cc] - Gx[i * kD + cc]);
                 a = fmaf(__bfloat162float(kr[cc]), kd, a);
@@ -435,10 +461,13 @@ __device__ void inverse(uint8_t* sm, const float* s_beta) {
 }
 
 template <int MODE>
-__device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, int h,
+__device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, int n_seq, int h,
                          int64_t bos, int64_t eos, bool aborted) {
     constexpr bool kG = (MODE & kGate) != 0;
+    constexpr bool kCv = (MODE & kConv) != 0;
     constexpr uint32_t kGBytes = kG ? 16384u : 32768u;   // raw logits bf16, or g fp32
+    constexpr int halo = kCv ? kHalo : 0;
+    constexpr uint32_t kTileBytes = (kC + halo) * 256;   // one q / k / v tile
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* misc = sm + P_MISC;
     const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
@@ -451,24 +480,33 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
     if (warp == kIoWarp) {
         // ---------------- I/O warp: lane 0 loads tiles, lane 1 stores and announces ----------
         if (lane == 0 && !aborted && ntasks > 0) {
-            auto issue = [&](int task) {
-                const int c0 = (int)(bos + (int64_t)chunk_of(task) * kC);
-                mbar_arrive_expect_tx(bar_at(misc, M_QK_FULL), 32768u);
+            auto issue_qkv = [&](int task) {
+                const int c0 = (int)(bos + (int64_t)chunk_of(task) * kC) - halo;
+                mbar_arrive_expect_tx(bar_at(misc, M_QK_FULL), (kCv ? 3u : 2u) * kTileBytes);
                 tma_load_3d(sb + P_Q, &p.tq, 0, h, c0, bar_at(misc, M_QK_FULL));
                 tma_load_3d(sb + P_K, &p.tk, 0, h, c0, bar_at(misc, M_QK_FULL));
+                if constexpr (kCv) tma_load_3d(sb + P_V, &p.tv, 0, h, c0, bar_at(misc, M_QK_FULL));
+            };
+            auto issue_g = [&](int task) {
+                const int c0 = (int)(bos + (int64_t)chunk_of(task) * kC);
                 mbar_arrive_expect_tx(bar_at(misc, M_G_FULL), kGBytes);
                 tma_load_3d(sb + P_G, &p.tg, 0, h, c0, bar_at(misc, M_G_FULL));
             };
-            issue(0);
-            int last = 0;
+            issue_qkv(0);
+            issue_g(0);
+            int last_qkv = 0, last_g = 0;
             for (int task = 0; task + 1 < ntasks; ++task) {
                 if (!wait_one(bar_at(misc, M_RAW_FREE), task & 1, p)) break;
-                issue(task + 1);
-                last = task + 1;
+                issue_qkv(task + 1);
+                last_qkv = task + 1;
+                // with kConv the g tile holds the conv's v until that leaves with the A part
+                if (kCv && !wait_one(bar_at(misc, M_LKQ_FREE), task & 1, p)) break;
+                issue_g(task + 1);
+                last_g = task + 1;
             }
-            // the tiles of the last load must land before the CTA may leave
-            mbar_wait(bar_at(misc, M_QK_FULL), last & 1, kDefaultWaitCycles);
-            mbar_wait(bar_at(misc, M_G_FULL), last & 1, kDefaultWaitCycles);
+            // the tiles of the last loads must land before the CTA may leave
+            mbar_wait(bar_at(misc, M_QK_FULL), last_qkv & 1, kDefaultWaitCycles);
+            mbar_wait(bar_at(misc, M_G_FULL), last_g & 1, kDefaultWaitCycles);
         } else if (lane == 1 && !aborted && ntasks > 0) {
             uint8_t* ring = p.ring + (size_t)ld_cluster_u32(c_misc + M_SMID) * ((size_t)kRing * kSlotBytes);
             uint32_t ph_gfree = 0;
@@ -483,6 +521,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                     if (!ok) break;
                 }
                 bulk_store(slot + S_LKQ, sb + P_LKQ, kAPart);
+                if constexpr (kCv) bulk_store(slot + S_V, sb + P_G, kVPart);
                 bulk_commit();
                 bulk_wait_read0();
                 mbar_arrive(bar_at(misc, M_LKQ_FREE));
@@ -506,7 +545,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
     float* s_ga = reinterpret_cast<float*>(misc + M_GA);
     float* s_gc = reinterpret_cast<float*>(misc + M_GC);
     float* s_rhf = reinterpret_cast<float*>(misc + M_RHF);
-    float* s_wsum = reinterpret_cast<float*>(misc + M_WSUM);
+    float* s_wsum = reinterpret_cast<float*>(sm + P_NM);   // (the inverse's scratch is idle)
     float* facs = reinterpret_cast<float*>(sm + P_LKQ + S_FAC);
     const int cg = lane & 15, tp = lane >> 4;           // fold: channel group of 8, token pair
     const int t0 = 4 * warp + 2 * tp;                   // fold: tokens t0, t0 + 1
@@ -540,8 +579,10 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             const int64_t c1 = bos + (int64_t)chunk_of(task + 1) * kC;
             if (c1 + tid < eos) beta_nx = beta_at(c1 + tid);
         }
+        trace_mark(prank, n, 0);
         bool ok = wait_warp(bar_at(misc, M_QK_FULL), ph, p) && wait_warp(bar_at(misc, M_G_FULL), ph, p) &&
                   (task == 0 || wait_warp(bar_at(misc, M_LKQ_FREE), ph ^ 1u, p));
+        trace_mark(prank, n, 1);
         // ---- fold, part 1: decay sums (log2 units) of the token pair, then of the warp's 4 tokens ----
         float s0[8], s1[8], xo[8];
         if (ok) {
@@ -604,6 +645,81 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             bad_c = (ga < -kHalf2) || (run - ga < -kHalf2);
         }
         const bool bad = bar_sync_or(kBarCompute, kCompute, bad_c) != 0;
+        if constexpr (kCv) {
+            // ---- conv prologue: q, k, v of tokens t0, t0 + 1 (8 channels each) from raw rows
+            //      t0 - 3 .. t0 + 1 (history before the sequence: the conv cache or zero), SiLU,
+            //      and the L2 norm of q and k over the 16 lanes that hold a token's 128 channels
+            uint4 outv[2][2];                            // q, k after the conv (v is stored at once)
+#pragma unroll
+            for (int z = 2; z >= 0; --z) {
+                const uint32_t tile = z == 0 ? P_Q : (z == 1 ? P_K : P_V);
+                float y0[8], y1[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) y0[c] = y1[c] = 0.f;
+                const float4* wz = reinterpret_cast<const float4*>(p.wconv[z]) + (size_t)h * kD + 8 * cg;
+#pragma unroll
+                for (int j = 0; j < 5; ++j) {
+                    const int r = t0 - kHalo + j;                 // token row relative to c0
+                    float x[8];
+                    unpack8(ld16(sm, tile + (r + kHalo) * 256 + cg * 16), x);
+                    if (c0 + r < bos) {                           // before the sequence
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            float hv = 0.f;
+                            if (p.conv_state != nullptr) {
+                                const int64_t ch = (int64_t)z * H * kD + (int64_t)h * kD + 8 * cg + c;
+                                hv = __bfloat162float(p.conv_state[((int64_t)n_seq * H * 3 * kD + ch) * 3 +
+                                                                   (kHalo - (int)(bos - (c0 + r)))]);
+                            }
+                            x[c] = hv;
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 w = __ldg(wz + c);
+                        const float wa[4] = {w.x, w.y, w.z, w.w};
+                        if (j <= 3) y0[c] = fmaf(wa[j], x[c], y0[c]);
+                        if (j >= 1) y1[c] = fmaf(wa[j - 1], x[c], y1[c]);
+                    }
+                }
+                float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    y0[c] = silu_fast(y0[c]);
+                    y1[c] = silu_fast(y1[c]);
+                    ss0 = fmaf(y0[c], y0[c], ss0);
+                    ss1 = fmaf(y1[c], y1[c], ss1);
+                }
+                if (z < 2) {
+#pragma unroll
+                    for (int o = 1; o < 16; o <<= 1) {
+                        ss0 += __shfl_xor_sync(0xffffffffu, ss0, o);
+                        ss1 += __shfl_xor_sync(0xffffffffu, ss1, o);
+                    }
+                    const float i0 = rsqrtf(ss0 + p.l2_eps), i1 = rsqrtf(ss1 + p.l2_eps);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        y0[c] *= i0;
+                        y1[c] *= i1;
+                    }
+                }
+                if (z == 2) {                            // the g tile is dead: v goes there now
+                    st16(sm, P_G + (uint32_t)(cg >> 3) * 8192 + sw128(t0, cg & 7, 0, 0), pack8(y0));
+                    st16(sm, P_G + (uint32_t)(cg >> 3) * 8192 + sw128(t0 + 1, cg & 7, 0, 0), pack8(y1));
+                } else {
+                    outv[z][0] = pack8(y0);
+                    outv[z][1] = pack8(y1);
+                }
+            }
+            bar_sync(kBarCompute, kCompute);             // every raw row has been read
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int t = t0 + u;
+                st16(sm, P_Q + (t + kHalo) * 256 + cg * 16, outv[0][u]);
+                st16(sm, P_K + (t + kHalo) * 256 + cg * 16, outv[1][u]);
+            }
+            bar_sync(kBarCompute, kCompute);
+        }
         // ---- fold, part 2: folded operands Lk, Lq (A of A|P and of the consumer's X | O), R ----
         {
             const int ac = cg >> 3, ch = cg & 7;
@@ -634,8 +750,8 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                 const int t = t0 + u;
                 const bool valid = t < L;
                 float qv[8], kv[8];
-                unpack8(ld16(sm, P_Q + t * 256 + cg * 16), qv);
-                unpack8(ld16(sm, P_K + t * 256 + cg * 16), kv);
+                unpack8(ld16(sm, P_Q + (t + halo) * 256 + cg * 16), qv);
+                unpack8(ld16(sm, P_K + (t + halo) * 256 + cg * 16), kv);
                 uint32_t lk[4], lq[4], rr[4];
 #pragma unroll
                 for (int c = 0; c < 8; c += 2) {
@@ -663,9 +779,10 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         fence_async_smem();
         tc_fence_before();
         bar_sync(kBarCompute, kCompute);
+        trace_mark(prank, n, 2);
         if (tid == 0) {
-            mbar_arrive(bar_at(misc, M_RAW_FREE));     // the raw tiles are dead
-            mbar_arrive(bar_at(misc, M_LKQ_READY));    // [Lk ; Lq | factors] may leave
+            if (!bad) mbar_arrive(bar_at(misc, M_RAW_FREE));   // the q, k (v) tiles are dead
+            mbar_arrive(bar_at(misc, M_LKQ_READY));            // [Lk ; Lq | factors] may leave
         }
         if (warp == 0) {                               // [A ; P] = [Lk ; Lq] R^T
             tc_fence_after();
@@ -682,6 +799,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         }
         // ---- extraction: N = diag(beta) A (strictly lower, fp32), P' (inclusive, bf16) ----
         ok = wait_warp(bar_at(misc, M_AP), ph, p);
+        trace_mark(prank, n, 3);
         if (warp == 0 && ok) ++ap_waited;
         tc_fence_after();
         if (ok && !bad) {
@@ -722,10 +840,13 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         }
         fence_async_smem();
         if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+        if (bad && tid == 0) mbar_arrive(bar_at(misc, M_RAW_FREE));   // the exact path is done
+        trace_mark(prank, n, 4);
         // ---- T' = (I + N)^-1 diag(beta) on warps 0..3 ----
         if (warp < 4) inverse(sm, s_beta);
         fence_async_smem();
         bar_sync(kBarCompute, kCompute);
+        trace_mark(prank, n, 5);
         // ---- Yh^T = R^T T' (M = key ch) and Wh^T = P' T' (M = token) ----
         if (warp == 0) {
             tc_fence_after();
@@ -746,6 +867,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             ++yw_issued;
         }
         ok = wait_warp(bar_at(misc, M_YW), ph, p);
+        trace_mark(prank, n, 6);
         if (warp == 0 && ok) ++yw_waited;
         if (ok && !bad && task > 0) ok = wait_warp(bar_at(misc, M_ST_FREE), ph ^ 1u, p);
         tc_fence_after();
@@ -770,6 +892,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
         tc_fence_before();
         if (bar_sync_or(kBarCompute, kCompute, fail)) break;
         if (tid == 0) mbar_arrive(bar_at(misc, M_ST_READY));
+        trace_mark(prank, n, 7);
     }
     // products still in flight must finish before the tensor memory is freed (the last commit
     // on each barrier covers every earlier product)
@@ -787,6 +910,7 @@ template <int MODE>
 __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, int h,
                          int64_t bos, int64_t eos, bool aborted) {
     constexpr bool kN = (MODE & kNorm) != 0;
+    constexpr bool kCv = (MODE & kConv) != 0;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* misc = sm + C_MISC;
     const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
@@ -808,6 +932,11 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 if (!wait_one(bar_at(misc, M_AFULL + 8 * (mm & 1)), par, p) ||
                     !wait_one(bar_at(misc, M_BFULL + 8 * (mm & 1)), par, p))
                     return false;
+                if constexpr (kCv) {        // the V tiles were read from the slot too
+                    if (!wait_one(bar_at(misc, M_VFULL + 8 * (mm & 1)), par, p) ||
+                        !wait_one(bar_at(misc, M_VFULL + 8 * (2 + (mm & 1))), par, p))
+                        return false;
+                }
                 if (mm + kRing < nchunks)
                     mbar_arrive_remote(map_to_rank(sb + P_MISC + M_GFREE + 8u * (uint32_t)(mm % kRing),
                                                    1 + (mm + kRing) % kProducers));
@@ -817,20 +946,33 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 const int sl = m & 1;
                 const uint32_t pfree = (uint32_t)((m - 2) >> 1) & 1u;
                 const int c0 = (int)(bos + (int64_t)m * kC);
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint64_t* vf = bar_at(misc, M_VFULL + 8 * (2 * hh + sl));
-                    if (m >= 2 && !(ok = wait_one(bar_at(misc, M_VFREE + 8 * (2 * hh + sl)), pfree, p))) break;
-                    mbar_arrive_expect_tx(vf, 8192u);
-                    tma_load_3d(sb + C_V + (uint32_t)(2 * hh + sl) * 8192, &p.tv, 64 * hh, h, c0, vf);
-                    v_issued = m + 1;
-                }
-                if (!ok) break;
                 const int rs = m % kRing;
+                const uint8_t* slot = ring + (size_t)rs * kSlotBytes;
+                // V tiles: by TMA from v, or (kConv) the conv's output from the ring slot
+                if constexpr (!kCv) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint64_t* vf = bar_at(misc, M_VFULL + 8 * (2 * hh + sl));
+                        if (m >= 2 && !(ok = wait_one(bar_at(misc, M_VFREE + 8 * (2 * hh + sl)), pfree, p))) break;
+                        mbar_arrive_expect_tx(vf, 8192u);
+                        tma_load_3d(sb + C_V + (uint32_t)(2 * hh + sl) * 8192, &p.tv, 64 * hh, h, c0, vf);
+                        v_issued = m + 1;
+                    }
+                    if (!ok) break;
+                }
                 ok = wait_one(bar_at(misc, M_GFULL + 8 * rs), (ph_gfull >> rs) & 1u, p, true);
                 ph_gfull ^= 1u << rs;
                 if (!ok) break;
                 fence_proxy_async_global();
-                const uint8_t* slot = ring + (size_t)rs * kSlotBytes;
+                if constexpr (kCv) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint64_t* vf = bar_at(misc, M_VFULL + 8 * (2 * hh + sl));
+                        if (m >= 2 && !(ok = wait_one(bar_at(misc, M_VFREE + 8 * (2 * hh + sl)), pfree, p))) break;
+                        mbar_arrive_expect_tx(vf, 8192u);
+                        bulk_load(sb + C_V + (uint32_t)(2 * hh + sl) * 8192, slot + S_V + hh * 8192, 8192u, vf);
+                        v_issued = m + 1;
+                    }
+                    if (!ok) break;
+                }
                 if (m >= 2 && !(ok = wait_one(bar_at(misc, M_AFREE + 8 * sl), pfree, p))) break;
                 mbar_arrive_expect_tx(bar_at(misc, M_AFULL + 8 * sl), kAPart);
                 bulk_load(sb + C_A + (uint32_t)sl * kAPart, slot + S_LKQ, kAPart, bar_at(misc, M_AFULL + 8 * sl));
@@ -1011,6 +1153,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         // (1) [X ; O](n) is in tensor memory: U(n) = V(n) - X(n) from rows 0..63, and the output
         //     of chunk n - 1 from rows 64..127 of the other accumulator
         bool ok = wait_warp(bar_xo, (uint32_t)b, p);
+        trace_mark(0, n, 8 * half + 0, 256 * half);
         if (issuer && ok) ++xo_waited;
         tc_fence_after();
         if (ok && n > 0 && tid_h == 0) mbar_arrive(bar_at(misc, M_BFREE + 8 * ((n - 1) & 1)));
@@ -1041,6 +1184,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         fence_async_smem();
         tc_fence_before();
         if (bar_sync_or(bar_half, 256, fail)) { stop = true; break; }
+        trace_mark(0, n, 8 * half + 1, 256 * half);
         if (tid_h == 0) mbar_arrive(bar_at(misc, M_VFREE + 8 * (2 * half + b)));
         // (2) state delta Yh^T U (commit), then O(n) += Wh^T U
         if (issuer) {
@@ -1067,6 +1211,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         }
         // (3) S' = e^{gamma_C} S + delta, then Sm(n + 1)
         ok = wait_warp(bar_ds, (uint32_t)b, p);
+        trace_mark(0, n, 8 * half + 2, 256 * half);
         if (issuer && ok) ++ds_waited;
         tc_fence_after();
         if (ok) {
@@ -1087,6 +1232,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         fence_async_smem();
         tc_fence_before();
         if (bar_sync_or(bar_half, 256, fail)) { stop = true; break; }
+        trace_mark(0, n, 8 * half + 3, 256 * half);
         if (tid_h == 0) mbar_arrive(bar_at(misc, M_AFREE + 8 * b));
         // (4) the next chunk's [X ; O], or a commit that covers O(n) after the last chunk
         if (issuer) {
@@ -1169,7 +1315,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
     // a consumer SM outside the workspace's ring table (flagged above): nobody touches the ring
     const bool aborted = (int)ld_cluster_u32(map_to_rank(sb + C_MISC + M_SMID, 0)) >= p.ring_sms;
     if (is_consumer) consumer<MODE>(p, sm, sb, n_seq, h, bos, eos, aborted);
-    else producer<MODE>(p, sm, sb, (int)crank, h, bos, eos, aborted);
+    else producer<MODE>(p, sm, sb, (int)crank, n_seq, h, bos, eos, aborted);
 
     tc_fence_before();
     __syncthreads();
@@ -1188,22 +1334,28 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
                              unsigned int* err, cudaStream_t stream) {
     const int64_t units = (int64_t)a.N * a.H;
     if (units == 0) return cudaSuccess;
-    const int mode = (a.g_raw != nullptr ? kGate : 0) | (a.z != nullptr ? kNorm : 0);
-    if (mode == kNorm) return cudaErrorInvalidValue;          // the norm comes with the gate
-    void (*kernel)(Params) = mode == 0 ? chunk_tcx_kernel<0>
-                           : mode == kGate ? chunk_tcx_kernel<kGate> : chunk_tcx_kernel<kGate | kNorm>;
+    const int mode = (a.g_raw != nullptr ? kGate : 0) | (a.z != nullptr ? kNorm : 0) |
+                     (a.wconv[0] != nullptr ? kConv : 0);
+    using KernelFn = void (*)(Params);
+    static const KernelFn kernels[8] = {
+        chunk_tcx_kernel<0>, chunk_tcx_kernel<1>, chunk_tcx_kernel<2>, chunk_tcx_kernel<3>,
+        chunk_tcx_kernel<4>, chunk_tcx_kernel<5>, chunk_tcx_kernel<6>, chunk_tcx_kernel<7>};
+    const KernelFn kernel = kernels[mode];
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     Params p;
-    const bool gate = (mode & kGate) != 0;
+    const bool gate = (mode & kGate) != 0, conv = (mode & kConv) != 0;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int tile_rows = conv ? kC + kHalo : kC;
     const bool maps_ok =
-        make_tmap_thd(&p.tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false) &&
-        make_tmap_thd(&p.tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false) &&
-        (gate ? make_tmap_thd(&p.tg, a.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, kD, kC, false)
+        make_tmap_thd(&p.tq, a.q, BF, 2, a.T_tot, a.H, kD, kD, tile_rows, false) &&
+        make_tmap_thd(&p.tk, a.k, BF, 2, a.T_tot, a.H, kD, kD, tile_rows, false) &&
+        (gate ? make_tmap_thd(&p.tg, a.g_raw, BF, 2, a.T_tot, a.H, kD, kD, kC, false)
               : make_tmap_thd(&p.tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.T_tot, a.H, kD, kD, kC, false)) &&
-        make_tmap_thd(&p.tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, 64, kC, true) &&
-        make_tmap_thd(&p.to, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T_tot, a.H, kD, 64, kC, true);
+        (conv ? make_tmap_thd(&p.tv, a.v, BF, 2, a.T_tot, a.H, kD, kD, tile_rows, false)
+              : make_tmap_thd(&p.tv, a.v, BF, 2, a.T_tot, a.H, kD, 64, kC, true)) &&
+        make_tmap_thd(&p.to, a.o, BF, 2, a.T_tot, a.H, kD, 64, kC, true);
     if (!maps_ok) return cudaErrorInvalidValue;
     p.q = static_cast<const __nv_bfloat16*>(a.q);
     p.k = static_cast<const __nv_bfloat16*>(a.k);
@@ -1228,6 +1380,9 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
     p.z = static_cast<const __nv_bfloat16*>(a.z);
     p.w_norm = a.w_norm;
     p.norm_eps = a.norm_eps;
+    for (int i = 0; i < 3; ++i) p.wconv[i] = a.wconv[i];
+    p.conv_state = static_cast<const __nv_bfloat16*>(a.conv_state);
+    p.l2_eps = a.l2_eps;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units * kCluster), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1246,3 +1401,10 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
 }
 
 }  // namespace kda
+
+#ifdef KDA_TRACE
+// Copies the prefill phase timestamps (see trace_mark) to `host` (4 * 512 * 16 uint64).
+extern "C" __attribute__((visibility("default"))) int kda_trace_dump(unsigned long long* host) {
+    return (int)cudaMemcpyFromSymbol(host, kda::g_trace, sizeof(kda::g_trace));
+}
+#endif

@@ -271,6 +271,26 @@ cudaError_t launch_conv_t(const ConvParams& p, cudaStream_t stream) {
 
 }  // namespace
 
+cudaError_t launch_conv_cache(const ConvArgs& a, cudaStream_t stream) {
+    ConvParams p;
+    for (int i = 0; i < 3; ++i) { p.x[i] = a.x[i]; p.w[i] = a.w[i]; p.y[i] = a.y[i]; }
+    p.conv_state = a.conv_state;
+    p.cu = a.cu;
+    p.T_tot = a.T_tot;
+    p.T_pad = a.T_pad;
+    p.N = a.N; p.H = a.H; p.dk = a.dk; p.dv = a.dv;
+    p.Ctot = a.H * (2 * a.dk + a.dv);
+    p.eps = a.eps;
+    p.step_mode = 0;
+    if (p.conv_state == nullptr || p.N == 0) return cudaSuccess;
+    const int64_t total = (int64_t)p.N * p.Ctot;
+    if (a.io == Io::BF16)
+        conv_cache_kernel<__nv_bfloat16><<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(p);
+    else
+        conv_cache_kernel<float><<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_conv(const ConvArgs& a, cudaStream_t stream) {
     ConvParams p;
     for (int i = 0; i < 3; ++i) { p.x[i] = a.x[i]; p.w[i] = a.w[i]; p.y[i] = a.y[i]; }

@@ -22,6 +22,9 @@ struct ConvArgs {
     Io io;
 };
 cudaError_t launch_conv(const ConvArgs& a, cudaStream_t stream);
+// Only the cache update of the prefill form: conv_state <- the last K-1 raw inputs of each
+// sequence's extended history (the cache followed by x).
+cudaError_t launch_conv_cache(const ConvArgs& a, cudaStream_t stream);
 
 struct StepArgs {
     const void *q, *k, *v;           // formed q, k, v, or the raw inputs when conv_state is set
@@ -72,6 +75,11 @@ struct ChunkArgs {
     const void* z = nullptr;
     const float* w_norm = nullptr;
     float norm_eps = 0.f;
+    // conv prologue in the producers' load stage (wconv[0] non-null): q, k, v are raw; conv
+    // weights [H*d, 4]; conv_state [N, H*(2dk+dv), 3] bf16 history (null: zero), read only here
+    const float* wconv[3] = {nullptr, nullptr, nullptr};
+    const void* conv_state = nullptr;
+    float l2_eps = 0.f;
 };
 cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 
@@ -79,7 +87,7 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 // kTcxRingSlots slots per SM id below kTcxRingSms, each slot one chunk's factors.
 constexpr int kTcxRingSms = 160;                 // a B200 has 148 SMs
 constexpr int kTcxRingSlots = 6;
-constexpr size_t kTcxSlotBytes = 58368;
+constexpr size_t kTcxSlotBytes = 74752;
 constexpr size_t kTcxWorkspaceBytes = (size_t)kTcxRingSms * kTcxRingSlots * kTcxSlotBytes;
 
 // Tensor-core (tcgen05) prefill for bf16 I/O, dk = dv = 128, chunk 64: a producer/consumer

@@ -21,7 +21,7 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUD
 KDA_IO_F32, KDA_IO_BF16 = 0, 1
 
 EXPORTED = ("kda_status_string", "kda_version", "kda_conv_fwd", "kda_chunk_fwd_workspace_size",
-            "kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_chunk_fwd_noalloc", "kda_recurrent_step",
+            "kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_fwd_noalloc", "kda_recurrent_step",
             "kda_conv_recurrent_step", "kda_fused_recurrent_step", "kda_set_wait_limit",
             "kda_last_device_error")
 
@@ -62,10 +62,11 @@ def load_library(path: str = LIB_PATH):
                                       ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci, ci,
                                       ci, vp, cs, vp]
         lib.kda_chunk_fwd.restype = ci
-        lib.kda_chunk_fwd_gated.argtypes = [vp, vp, vp, vp, vp, fp, fp, vp, fp, cf, cf, fp, fp, vp,
-                                            i32p, ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci,
-                                            ci, ci, ci, ci, vp, cs, vp]
-        lib.kda_chunk_fwd_gated.restype = ci
+        lib.kda_chunk_fwd_fused.argtypes = [vp, vp, vp, fp, fp, fp, vp, cf, fp, fp, vp, vp, fp, fp, vp,
+                                            fp, cf, cf, fp, fp, vp, i32p,
+                                            ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci,
+                                            ci, ci, ci, vp, cs, vp]
+        lib.kda_chunk_fwd_fused.restype = ci
         lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, cf, fp, fp, vp, i32p,
                                               ctypes.POINTER(ctypes.c_int32), ci, ci, ci, ci, ci, ci,
                                               ci, ci, vp]
@@ -182,12 +183,15 @@ def chunk_fwd(q, k, v, g, beta, scale=1.0, h0=None, ht=None, o=None, cu_seqlens=
     return o, ht
 
 
-def chunk_fwd_gated(q, k, v, g_raw, beta_raw, A_log, dt_bias, z=None, w_norm=None, norm_eps=1e-6,
-                    scale=1.0, h0=None, ht=None, o=None, cu_seqlens=None, cu_host=None, chunk=64,
-                    workspace=None, stream=None):
-    """Chunked prefill with g and beta from raw logits (g = -exp(A_log) softplus(g_raw +
-    dt_bias), beta = sigmoid(beta_raw)) and, when z is given, the gated RMSNorm of the output.
-    Layouts as chunk_fwd; g_raw [.., H, dk] and beta_raw [.., H] bf16. Returns (o, ht)."""
+def chunk_fwd_fused(q, k, v, g=None, beta=None, *, w_q=None, w_k=None, w_v=None,
+                    conv_state=None, l2_eps=1e-6, g_raw=None, beta_raw=None, A_log=None,
+                    dt_bias=None, z=None, w_norm=None, norm_eps=1e-6, scale=1.0, h0=None, ht=None,
+                    o=None, cu_seqlens=None, cu_host=None, chunk=64, K=4, workspace=None,
+                    stream=None):
+    """Chunked prefill with optional fused steps: the conv prologue (w_q, w_k, w_v given: q, k, v
+    are raw projections; conv_state is read as the history and overwritten with the new one),
+    the gate from raw logits (g_raw, beta_raw, A_log, dt_bias given; else g and beta are used),
+    and the gated RMSNorm of the output (z, w_norm given). Returns (o, ht)."""
     lib = load_library()
     if cu_seqlens is None:
         B, T, H, dk = q.shape if q.dim() == 4 else (1, *q.shape)
@@ -204,14 +208,14 @@ def chunk_fwd_gated(q, k, v, g_raw, beta_raw, A_log, dt_bias, z=None, w_norm=Non
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     keep, cuh = _host_cu(cu_host)
-    st = lib.kda_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(g_raw), _ptr(beta_raw),
-                                 _ptr(A_log), _ptr(dt_bias), _ptr(z), _ptr(w_norm),
-                                 float(norm_eps), float(scale), _ptr(h0), _ptr(ht), _ptr(o),
-                                 _ptr(cu_seqlens), cuh, B, T, N, H, dk, dv, chunk, _io(q),
-                                 _ptr(workspace), 0 if workspace is None else workspace.numel(),
-                                 _stream(stream))
+    st = lib.kda_chunk_fwd_fused(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(w_q), _ptr(w_k), _ptr(w_v), _ptr(conv_state),
+        float(l2_eps), _ptr(g), _ptr(beta), _ptr(g_raw), _ptr(beta_raw), _ptr(A_log),
+        _ptr(dt_bias), _ptr(z), _ptr(w_norm), float(norm_eps), float(scale), _ptr(h0), _ptr(ht),
+        _ptr(o), _ptr(cu_seqlens), cuh, B, T, N, H, dk, dv, K, chunk, _io(q), _ptr(workspace),
+        0 if workspace is None else workspace.numel(), _stream(stream))
     del keep
-    _check("kda_chunk_fwd_gated", st)
+    _check("kda_chunk_fwd_fused", st)
     return o, ht
 
 

@@ -75,7 +75,7 @@ def _cu_host(vals):
     (dict(io=7), kda.KDA_ERR_INVALID_ARG),
     (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
     (dict(dk=96, dv=96), kda.KDA_ERR_UNSUPPORTED),
-    (dict(dk=128, dv=64), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dk=128, dv=32), kda.KDA_ERR_UNSUPPORTED),
 ])
 def test_chunk_fwd_rejects(lib, kw, status):
     assert _chunk(lib, **kw) == status
@@ -203,25 +203,33 @@ def test_fused_decode_entry_points_check_arguments(lib):
     assert _fused_step(lib, br=ctypes.c_void_p(0x10001)) == kda.KDA_ERR_INVALID_ARG
 
 
-def _gated(lib, **kw):
-    a = dict(q=FAKE, k=FAKE, v=FAKE, gr=FAKE, br=FAKE, A=FAKE, dt=FAKE, z=None, wn=None,
-             neps=1e-6, scale=1.0, h0=None, ht=None, o=FAKE, cu=None, cuh=None, B=1, T=64, N=1,
-             H=2, dk=128, dv=128, chunk=64, io=1, ws=FAKE, wsb=1 << 30, stream=None)
+def _fused(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, wq=None, wk=None, wv=None, cs=None, l2=1e-6, g=FAKE, b=FAKE,
+             gr=None, br=None, A=None, dt=None, z=None, wn=None, neps=1e-6, scale=1.0, h0=None,
+             ht=None, o=FAKE, cu=None, cuh=None, B=1, T=64, N=1, H=2, dk=128, dv=128, K=4,
+             chunk=64, io=1, ws=FAKE, wsb=1 << 30, stream=None)
     a.update(kw)
-    return lib.kda_chunk_fwd_gated(a["q"], a["k"], a["v"], a["gr"], a["br"], a["A"], a["dt"],
+    return lib.kda_chunk_fwd_fused(a["q"], a["k"], a["v"], a["wq"], a["wk"], a["wv"], a["cs"],
+                                   a["l2"], a["g"], a["b"], a["gr"], a["br"], a["A"], a["dt"],
                                    a["z"], a["wn"], a["neps"], a["scale"], a["h0"], a["ht"],
                                    a["o"], a["cu"], a["cuh"], a["B"], a["T"], a["N"], a["H"],
-                                   a["dk"], a["dv"], a["chunk"], a["io"], a["ws"], a["wsb"],
+                                   a["dk"], a["dv"], a["K"], a["chunk"], a["io"], a["ws"], a["wsb"],
                                    a["stream"])
 
 
-def test_gated_prefill_checks_arguments(lib):
-    assert _gated(lib, gr=None) == kda.KDA_ERR_INVALID_ARG
-    assert _gated(lib, A=None) == kda.KDA_ERR_INVALID_ARG
-    assert _gated(lib, dt=None) == kda.KDA_ERR_INVALID_ARG
-    assert _gated(lib, br=ctypes.c_void_p(0x10001)) == kda.KDA_ERR_INVALID_ARG
-    assert _gated(lib, z=FAKE) == kda.KDA_ERR_INVALID_ARG           # a norm gate without weight
-    assert _gated(lib, chunk=0) == kda.KDA_ERR_INVALID_ARG
-    assert _gated(lib, io=0) == kda.KDA_ERR_UNSUPPORTED              # tensor-core path only
-    assert _gated(lib, dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
-    assert _gated(lib, ws=None) == kda.KDA_ERR_WORKSPACE
+def test_fused_prefill_checks_arguments(lib):
+    gate = dict(gr=FAKE, br=FAKE, A=FAKE, dt=FAKE, g=None, b=None)
+    conv = dict(wq=FAKE, wk=FAKE, wv=FAKE)
+    assert _fused(lib, g=None) == kda.KDA_ERR_INVALID_ARG            # neither g nor raw logits
+    assert _fused(lib, **dict(gate, A=None)) == kda.KDA_ERR_INVALID_ARG
+    assert _fused(lib, **dict(gate, dt=None)) == kda.KDA_ERR_INVALID_ARG
+    assert _fused(lib, **dict(gate, br=ctypes.c_void_p(0x10001))) == kda.KDA_ERR_INVALID_ARG
+    assert _fused(lib, wq=FAKE) == kda.KDA_ERR_INVALID_ARG           # conv weights all or none
+    assert _fused(lib, cs=FAKE) == kda.KDA_ERR_INVALID_ARG           # a history without the conv
+    assert _fused(lib, **dict(conv, l2=-1.0)) == kda.KDA_ERR_INVALID_ARG
+    assert _fused(lib, **dict(conv, K=3)) == kda.KDA_ERR_UNSUPPORTED
+    assert _fused(lib, z=FAKE) == kda.KDA_ERR_INVALID_ARG            # a norm gate without weight
+    assert _fused(lib, chunk=0) == kda.KDA_ERR_INVALID_ARG
+    assert _fused(lib, io=0) == kda.KDA_ERR_UNSUPPORTED               # tensor-core path only
+    assert _fused(lib, dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
+    assert _fused(lib, ws=None) == kda.KDA_ERR_WORKSPACE

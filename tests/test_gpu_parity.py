@@ -249,10 +249,10 @@ def test_chunk_tiny_fp32():
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
-@pytest.mark.parametrize("d_head", [64, 128])
-def test_chunk_varlen_ragged(io, d_head):
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+def test_chunk_varlen_ragged(io, dk, dv):
     lens = [1, 63, 64, 65, 0, 130, 7, 200]
-    wl = small("prefill_8k", N=len(lens), H=3, dk=d_head, dv=d_head, io=io, h0_std=0.02, seed=31)
+    wl = small("prefill_8k", N=len(lens), H=3, dk=dk, dv=dv, io=io, h0_std=0.02, seed=31)
     d = make_prefill(wl, DEV, lengths=lens)
     o, ht = run_chunk(d)
     torch.cuda.synchronize()
@@ -295,8 +295,8 @@ def _oracle_gated_prefill(d, norm, scale=1.0):
 
 
 def _run_gated(d, norm, scale=1.0):
-    return kda.chunk_fwd_gated(d["q"], d["k"], d["v"], d["g_raw"], d["beta_raw"], d["A_log"],
-                               d["dt_bias"], z=d["z"] if norm else None,
+    return kda.chunk_fwd_fused(d["q"], d["k"], d["v"], g_raw=d["g_raw"], beta_raw=d["beta_raw"],
+                               A_log=d["A_log"], dt_bias=d["dt_bias"], z=d["z"] if norm else None,
                                w_norm=d["w_norm"] if norm else None, scale=scale, h0=d["h0"],
                                cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"])
 
@@ -341,6 +341,96 @@ def test_chunk_gated_prefill_8k_full():
     record_margin("prefill_8k gated (gate, norm)", "o pooled", eo, TOL_BF16)
     record_margin("prefill_8k gated (gate, norm)", "ht pooled", eh, TOL_BF16)
     assert eo <= TOL_BF16 and eh <= TOL_BF16
+
+
+def _oracle_conv_prefill(d, conv_state=None, gate=False, norm=False, scale=1.0):
+    """fp64 oracle of the fused prefill: the prologue on the raw inputs (with the conv history),
+    the gate and beta (from raw logits when gate), the token loop, the optional gated RMSNorm."""
+    q, k, v, cache = oracle.prologue(to64(d["q_raw"]), to64(d["k_raw"]), to64(d["v_raw"]),
+                                     to64(d["w_q"]), to64(d["w_k"]), to64(d["w_v"]),
+                                     None if conv_state is None else to64(conv_state),
+                                     d["cu_host"], 1e-6)
+    if gate:
+        g = oracle.gate(to64(d["g_raw"]), to64(d["A_log"]), to64(d["dt_bias"]))
+        beta = oracle.sigmoid(to64(d["beta_raw"]))
+    else:
+        g, beta = to64(d["g"]), to64(d["beta"])
+    o, ht = oracle.kda_fwd(q, k, v, g, beta, scale, to64(d["h0"]), d["cu_host"])
+    if norm:
+        o = oracle.gated_rmsnorm(o, to64(d["z"]), to64(d["w_norm"]), 1e-6)
+    return o, ht, cache
+
+
+def _run_conv_prefill(d, conv_state=None, gate=False, norm=False, scale=1.0):
+    kw = dict(g_raw=d["g_raw"], beta_raw=d["beta_raw"], A_log=d["A_log"],
+              dt_bias=d["dt_bias"]) if gate else dict(g=d["g"], beta=d["beta"])
+    if norm:
+        kw.update(z=d["z"], w_norm=d["w_norm"])
+    return kda.chunk_fwd_fused(d["q_raw"], d["k_raw"], d["v_raw"], w_q=d["w_q"], w_k=d["w_k"],
+                               w_v=d["w_v"], conv_state=conv_state, scale=scale, h0=d["h0"],
+                               cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], **kw)
+
+
+@pytest.mark.parametrize("with_cache", [False, True])
+def test_chunk_conv_prologue_fused_matches_oracle(with_cache):
+    """Raw q, k, v through the conv prologue in the producers' load stage (3-token halo, the
+    history from the conv cache or zero), on ragged packed sequences; the cache is advanced."""
+    lens = [1, 2, 3, 63, 64, 65, 0, 130, 200, 700]
+    wl = small("varlen_prologue", N=len(lens), H=3, seed=53)
+    d = make_prefill(wl, DEV, lengths=lens)
+    cs = None
+    if with_cache:
+        cs = torch.randn((len(lens), 3 * 384, 3), device=DEV).to(torch.bfloat16)
+    cs_in = None if cs is None else cs.clone()
+    o, ht = _run_conv_prefill(d, cs, scale=0.9)
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == kda.KDA_OK
+    o_ref, h_ref, c_ref = _oracle_conv_prefill(d, cs_in, scale=0.9)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16
+    assert rel_l2(to64(ht), h_ref) <= TOL_BF16
+    if with_cache:
+        assert np.array_equal(to64(cs), c_ref)             # the cache holds raw inputs: exact
+
+
+def test_chunk_fully_fused_layer_matches_oracle():
+    """Conv prologue, gate and beta from raw logits, and the output norm, all in the prefill."""
+    lens = [5, 64, 129, 300]
+    wl = small("varlen_prologue", N=len(lens), H=2, seed=54)
+    d = make_prefill(wl, DEV, lengths=lens, raw=True)
+    o, ht = _run_conv_prefill(d, gate=True, norm=True)
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == kda.KDA_OK
+    o_ref, h_ref, _ = _oracle_conv_prefill(d, gate=True, norm=True)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16
+    assert rel_l2(to64(ht), h_ref) <= TOL_BF16
+
+
+def test_varlen_prologue_fused_full():
+    """varlen_prologue as its config states: raw q/k/v of 64 packed sequences through the prefill
+    with the conv prologue fused in. Every (sequence, head) unit against the oracle run on the
+    raw inputs; pooled and per-unit rel-L2."""
+    wl = WORKLOADS["varlen_prologue"]
+    d = make_prefill(wl, DEV)
+    o, ht = _run_conv_prefill(d)
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == kda.KDA_OK
+    cu, N, H = d["cu_host"], d["N"], d["H"]
+    po, ph = _PerUnit(N * H), _PerUnit(N * H)
+    for n in range(N):
+        sl = slice(cu[n], cu[n + 1])
+        q, k, v, _ = oracle.prologue(to64(d["q_raw"][sl]), to64(d["k_raw"][sl]), to64(d["v_raw"][sl]),
+                                     to64(d["w_q"]), to64(d["w_k"]), to64(d["w_v"]), None,
+                                     [0, cu[n + 1] - cu[n]], 1e-6)
+        o_ref, h_ref = oracle.kda_fwd(q, k, v, to64(d["g"][sl]), to64(d["beta"][sl]), 1.0,
+                                      to64(d["h0"][n:n + 1]), None)
+        units = [n * H + h for h in range(H)]
+        po.add(units, to64(o[sl]), o_ref)
+        ph.add(units, to64(ht[n]).reshape(1, H, -1), h_ref.reshape(1, H, -1))
+    name = "varlen_prologue fused (all units)"
+    for nm, acc in (("o", po), ("ht", ph)):
+        record_margin(name, f"{nm} pooled", acc.pooled(), TOL_BF16)
+        record_margin(name, f"{nm} worst unit", acc.worst(), TOL_BF16)
+        assert acc.pooled() <= TOL_BF16 and acc.worst() <= TOL_BF16
 
 
 def test_chunk_padded_equals_packed():
