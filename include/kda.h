@@ -182,10 +182,25 @@ kda_status kda_chunk_fwd_fused(const void* q, const void* k, const void* v, cons
                                size_t workspace_bytes, void* stream);
 
 /*
- * kda_chunk_fwd_noalloc -- kda_chunk_fwd without a caller workspace: the library uses a
- * device array of its own (reserved when libkda is loaded, one per device), so the call
- * allocates nothing. Arguments, layouts, results and errors are those of kda_chunk_fwd.
- * Calls on one device must not run concurrently with each other (they share that array).
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate device memory.
+ * (The pages have no counterpart: this is a library convenience, not a step of the method.)
+ *
+ * kda_chunk_fwd needs a caller-owned workspace of kda_chunk_fwd_workspace_size() bytes
+ * (~72 MB for the bf16, dk = dv = 128 prefill). Some callers cannot cudaMalloc one where they
+ * run the prefill: a runtime whose memory pool already holds all free device memory, a plug-in
+ * handed only tensor pointers, or a latency-critical path that cannot afford cudaMalloc's
+ * implicit device synchronisation. This entry point uses instead a device array owned by the
+ * library (a file-scope __device__ array of exactly that maximum size, one per device, held by
+ * every GPU that loads libkda until the process exits), so the call allocates nothing; the
+ * caller still passes every input and output.
+ *
+ * Arguments, layouts, results and errors are those of kda_chunk_fwd. A size whose workspace
+ * would exceed the array returns KDA_ERR_WORKSPACE; if the array's device address cannot be
+ * obtained the call returns KDA_ERR_CUDA (argument errors are still reported first).
+ * Set-up: the first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any stream capture.
+ * Sharing: every call on a device uses the same array, which keeps the last call's contents
+ * (no call needs it cleared); calls that overlap on the GPU race, so run them one after another.
  */
 kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
                                  const float* beta, float scale, const float* h0, float* ht,
