@@ -407,16 +407,21 @@ def test_chunk_fully_fused_layer_matches_oracle():
 
 def test_varlen_prologue_fused_full():
     """varlen_prologue as its config states: raw q/k/v of 64 packed sequences through the prefill
-    with the conv prologue fused in. Every (sequence, head) unit against the oracle run on the
-    raw inputs; pooled and per-unit rel-L2."""
+    with the conv prologue fused in, at full size. Every head of 12 sequences (the 4 shortest,
+    the 4 longest and 4 seeded others) against the oracle run on the raw inputs; pooled and
+    per-unit rel-L2. (test_varlen_prologue_full checks every unit of the unfused path.)"""
     wl = WORKLOADS["varlen_prologue"]
     d = make_prefill(wl, DEV)
     o, ht = _run_conv_prefill(d)
     torch.cuda.synchronize()
     assert kda.last_device_error() == kda.KDA_OK
     cu, N, H = d["cu_host"], d["N"], d["H"]
+    order = np.argsort(np.array(d["lengths"]))
+    rest = [int(x) for x in order[4:-4]]
+    seqs = sorted(set([int(x) for x in order[:4]] + [int(x) for x in order[-4:]] +
+                      list(np.random.default_rng(wl.seed).choice(rest, 4, replace=False))))
     po, ph = _PerUnit(N * H), _PerUnit(N * H)
-    for n in range(N):
+    for n in seqs:
         sl = slice(cu[n], cu[n + 1])
         q, k, v, _ = oracle.prologue(to64(d["q_raw"][sl]), to64(d["k_raw"][sl]), to64(d["v_raw"][sl]),
                                      to64(d["w_q"]), to64(d["w_k"]), to64(d["w_v"]), None,
@@ -426,7 +431,7 @@ def test_varlen_prologue_fused_full():
         units = [n * H + h for h in range(H)]
         po.add(units, to64(o[sl]), o_ref)
         ph.add(units, to64(ht[n]).reshape(1, H, -1), h_ref.reshape(1, H, -1))
-    name = "varlen_prologue fused (all units)"
+    name = "varlen_prologue fused (12 seq x 32 heads)"
     for nm, acc in (("o", po), ("ht", ph)):
         record_margin(name, f"{nm} pooled", acc.pooled(), TOL_BF16)
         record_margin(name, f"{nm} worst unit", acc.worst(), TOL_BF16)
@@ -504,7 +509,8 @@ class _PerUnit:
         return float(np.sqrt(self.num.sum() / self.den.sum()))
 
     def worst(self):
-        return float(np.max(np.sqrt(self.num / np.maximum(self.den, 1e-300))))
+        seen = self.den > 0
+        return float(np.max(np.sqrt(self.num[seen] / self.den[seen]))) if seen.any() else 0.0
 
 
 def test_varlen_prologue_full():
