@@ -88,16 +88,16 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
 #pragma unroll
     for (int r = 0; r < R; ++r) Vec<float, CPL>::load(S + (warp * R + r) * DV + col, s[r]);
 
-    if constexpr (GATE) {
-        const int h = (int)(pair % cv.H);
-        const float ea = expf(cv.A_log[h]);
-        const T* graw = static_cast<const T*>(g_in);
-        for (int i = threadIdx.x; i < DK; i += blockDim.x)
-            s_a[i] = expf(-ea * softplus_f(to_f32(graw[pair * DK + i]) + cv.dt_bias[h * DK + i]));
-    } else {
-        const float* g = static_cast<const float*>(g_in);
-        for (int i = threadIdx.x; i < DK; i += blockDim.x) s_a[i] = expf(g[pair * DK + i]);
-    }
+    // per-key-channel decay exp(g), with GATE from the raw logit
+    auto decay = [&](int i) -> float {
+        if constexpr (GATE) {
+            const int h = (int)(pair % cv.H);
+            const float x = to_f32(static_cast<const T*>(g_in)[pair * DK + i]) + cv.dt_bias[h * DK + i];
+            return expf(-expf(cv.A_log[h]) * softplus_f(x));
+        } else {
+            return expf(static_cast<const float*>(g_in)[pair * DK + i]);
+        }
+    };
     if constexpr (CONV) {
         // conv step of this (sequence, head)'s 2 DK + DV channels: q, then k, then v
         __shared__ float s_inv[2];
@@ -113,6 +113,7 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
             const float4 w = *reinterpret_cast<const float4*>(wz + (int64_t)(h * D + ch) * 4);
             T* cs = cache + (n * Ctot + (int64_t)z * H * DK + (int64_t)h * D + ch) * 3;
             const T x0 = cs[0], x1 = cs[1], x2 = cs[2], xt = x[pair * D + ch];
+            if (c < DK) s_a[c] = decay(c);             // (its loads overlap the conv's)
             float zc = w.x * to_f32(x0);
             zc = fmaf(w.y, to_f32(x1), zc);
             zc = fmaf(w.z, to_f32(x2), zc);
@@ -137,11 +138,18 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
             s_k[i] *= s_inv[1];
         }
     } else {
-        for (int i = threadIdx.x; i < DK; i += blockDim.x) {
-            s_k[i] = to_f32(k[pair * DK + i]);
-            s_q[i] = to_f32(q[pair * DK + i]);
+        // every per-pair input in one pass (a thread: q, k and the gate of one key channel, or
+        // one value), so that the loads' latencies overlap
+        for (int i = threadIdx.x; i < DK + DV; i += blockDim.x) {
+            if (i < DK) {
+                const float kv = to_f32(k[pair * DK + i]), qv = to_f32(q[pair * DK + i]);
+                s_a[i] = decay(i);
+                s_k[i] = kv;
+                s_q[i] = qv;
+            } else {
+                s_v[i - DK] = to_f32(v[pair * DV + (i - DK)]);
+            }
         }
-        for (int j = threadIdx.x; j < DV; j += blockDim.x) s_v[j] = to_f32(v[pair * DV + j]);
     }
     float b;
     if constexpr (GATE) b = 1.f / (1.f + expf(-to_f32(static_cast<const T*>(beta_in)[pair])));
