@@ -242,6 +242,10 @@ def _events_time(torch, fn, steps, warmup, flush=None, stream=None):
         fn()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    from kimi_delta_attention_32_b200 import kda
+    status = kda.last_device_error()
+    if status != kda.KDA_OK:         # a bounded wait gave up: the timing is not a valid number
+        raise RuntimeError(f"device error word set during the timed steps (status {status})")
     return [a.elapsed_time(b) for a, b in ev]
 
 

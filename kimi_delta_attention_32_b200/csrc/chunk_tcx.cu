@@ -21,14 +21,10 @@
 // every factor is <= 1).
 //
 // Cluster of 4 CTAs of 17 warps: rank 0 is the consumer, ranks 1..3 are producers, each
-// preparing every third chunk. Inside a producer, a front end (8 warps: the conv prologue with
-// kConv, the decay sums, the folded operands) works one chunk ahead of a back end (8 warps: the
-// tensor-core products, the triangular inverse and the staging of the second part), so that the
-// two overlap. A chunk's factors (57 KB) travel through L2, not DSMEM: the producer's I/O warp
-// bulk-stores them into a ring in global memory owned by the consumer's SM (one lane the first
-// part right after the fold, another the second part after staging, each once the consumer has
-// handed the slot back: "gfree") and announces them on a cluster barrier ("gfull") once both are
-// written; the consumer's loader warp bulk-loads them into shared memory and hands the slot back.
+// preparing every third chunk. A chunk's factors (57 KB) travel through L2, not DSMEM: the
+// producer's I/O lane bulk-stores them into a ring in global memory owned by the consumer's SM
+// and announces them on a cluster barrier ("gfull"); the consumer's loader warp bulk-loads them
+// into shared memory and hands the ring slot back ("gfree").
 //
 // The consumer runs the value columns as two independent halves of 64 (state columns do not
 // interact), each on its own 8 warps with its own MMA issuer, so that one half's tensor-core
@@ -66,6 +62,7 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr int kWarps = 17;
 constexpr int kThreads = 32 * kWarps;     // 16 compute warps + 1 I/O (producer) or loader warp
+constexpr int kCompute = 512;
 constexpr int kIoWarp = 16;
 constexpr int kProducers = 3;
 constexpr int kCluster = 1 + kProducers;
@@ -82,8 +79,7 @@ constexpr uint32_t S_FAC = 32768;        // e^{gamma_ref}[128], e^{gamma_C}[128]
 constexpr uint32_t kAPart = 33792;       // [Lk ; Lq | factors]
 constexpr uint32_t S_YW = kAPart;        // [Yh^T (rows key ch 0..127) ; Wh^T (rows token)]: K-major
 constexpr uint32_t kBPart = 24576;
-constexpr uint32_t S_V = kAPart + kBPart;   // kConv: V after the conv, [token][128 ch] bf16; the 16-byte
-                                         //   chunk c of each 128-byte half row sits at c ^ (token & 7)
+constexpr uint32_t S_V = kAPart + kBPart;   // kConv: V after the conv, [half][token][64 ch] SW128
 constexpr uint32_t kVPart = 16384;
 constexpr uint32_t kSlotBytes = kAPart + kBPart + kVPart;
 constexpr int kRing = kTcxRingSlots;
@@ -95,9 +91,9 @@ constexpr uint32_t kRawTile = 17408;     // 68 token rows of 256 B: 64, after 3 
 constexpr uint32_t P_Q = 0;              // q tile [rows][128] bf16 (TMA, unswizzled); with kConv
                                          //   raw, then overwritten by the conv's output
 constexpr uint32_t P_K = kRawTile;       // k tile, the same
-constexpr uint32_t P_V = 2 * kRawTile;   // kConv: raw v tile, overwritten in place by v after the conv
-                                         //   (the slot's V part); otherwise the second R buffer
-constexpr uint32_t P_G = 3 * kRawTile;   // g tile [64][128] fp32 (kGate: bf16 logits)
+constexpr uint32_t P_V = 2 * kRawTile;   // kConv: raw v tile
+constexpr uint32_t P_G = 3 * kRawTile;   // g tile [64][128] fp32 (kGate: bf16 logits); with kConv
+                                         //   v after the conv (the slot's V part) once g is read
 constexpr uint32_t P_LKQ = P_G + 32768;  // [Lk ; Lq | factors]: the slot's A part image
 constexpr uint32_t P_R = P_LKQ + kAPart; // R: K-major, 2 atom columns x 64 token rows
 constexpr uint32_t P_PO = P_R + 16384;   // P': K-major, 64 token rows x 64 (A of Wh^T; its M = 128
@@ -105,7 +101,8 @@ constexpr uint32_t P_PO = P_R + 16384;   // P': K-major, 64 token rows x 64 (A o
 constexpr uint32_t P_TP = P_PO + 8192;   // T': rows r (K), 64 columns i (N): MN-major B
 constexpr int kLd = 68;                  // fp32 row stride of the 64 x 64 inverse scratch
 constexpr int kLdY = 24;                 // row stride of the per-warp 16 x 16 products
-constexpr uint32_t P_NM = P_TP + 8192;   // N = diag(beta) A (fp32 [64][kLd])
+constexpr uint32_t P_NM = P_TP + 8192;   // N = diag(beta) A (fp32 [64][kLd]); during the fold the
+                                         //   per-warp decay sums [16][128]
 constexpr uint32_t P_TM = P_NM + 64 * kLd * 4;   // T (fp32 [64][kLd])
 constexpr uint32_t P_Y = P_TM + 64 * kLd * 4;    // [4][16][kLdY] fp32
 constexpr uint32_t P_ST = ((P_Y + 4 * 16 * kLdY * 4 + 1023) / 1024) * 1024;   // [Yh^T ; Wh^T] staging
@@ -114,15 +111,14 @@ constexpr uint32_t P_GX = P_TM;          // exact path: natural-log gamma fp32 [
 constexpr uint32_t P_MISC = P_ST + kBPart;
 static_assert(P_LKQ % 1024 == 0 && P_R % 1024 == 0 && P_PO % 1024 == 0 && P_TP % 1024 == 0 &&
               P_ST % 1024 == 0, "operand tiles are swizzle-atom aligned");
-static_assert((kC + kHalo) * 256 <= kRawTile && kHalo * 256 + kVPart <= kRawTile && 16384 <= kRawTile &&
-              P_V % 1024 == 0, "tile sizes; the second R buffer");
+static_assert((kC + kHalo) * 256 <= kRawTile && 2 * kVPart / 2 <= 32768 && 16 * 128 * 4 <= 64 * kLd * 4,
+              "tile and scratch sizes");
 static_assert(P_GX + 64 * 128 * 4 <= P_MISC, "exact-path scratch");
 
 // ---- consumer shared memory ----
 constexpr uint32_t C_A = 0;                        // A parts of chunks n % 2
 constexpr uint32_t C_B = 2 * kAPart;               // B parts of chunks n % 2
-constexpr uint32_t C_V = C_B + 2 * kBPart;         // V tiles [half][n % 2] (64 ch x 64 tokens, SW128);
-                                                   //   kConv: [n % 2] (the slot's V part)
+constexpr uint32_t C_V = C_B + 2 * kBPart;         // V tiles [half][n % 2] (64 ch x 64 tokens, SW128)
 constexpr uint32_t C_SM = C_V + 4 * 8192;          // Sm per half: MN-major B (K = key ch, N = 64)
 constexpr uint32_t C_U = C_SM + 2 * 16384;         // U per half: MN-major B (K = token, N = 64)
 constexpr uint32_t C_OST = C_U + 2 * 8192;         // O staging per half (64 ch x 64 tokens, SW128)
@@ -136,17 +132,14 @@ constexpr uint32_t M_TMP = 260;       // unit_of scratch
 constexpr uint32_t M_SMID = 264;      // consumer: its SM id (selects the global ring)
 // producer barriers
 constexpr uint32_t M_QK_FULL = 0, M_G_FULL = 8, M_RAW_FREE = 16, M_LKQ_READY = 24, M_LKQ_FREE = 32,
-                   M_ST_READY = 40, M_ST_FREE = 48, M_AP = 56, M_YW = 64, M_A_DONE = 72,
-                   M_ANNC = 80, M_GFREE = 88, M_FOLD = M_GFREE + 8 * kRing, M_GT_FREE = M_FOLD + 8;
-constexpr int kBarsP = 13 + kRing;
-constexpr uint32_t M_BETA = 512;      // beta [task % 2][64]
-constexpr uint32_t M_GA = 1024;       // gamma at token 31, per channel (log2 units)
-constexpr uint32_t M_GC = 1536;       // gamma at token 63 (log2 units)
-constexpr uint32_t M_RHF = 2048;      // e^{gamma_C - gamma_s} per channel [task % 2][128]
-constexpr uint32_t M_DT = 3072;       // kGate: dt_bias of this head [128]
-constexpr uint32_t M_BAD = 3584;      // range-test result [task % 2]
-constexpr uint32_t M_WSUM = 4096;     // the front end's per-warp decay sums [8][128]
-constexpr uint32_t kMiscP = M_WSUM + 8 * 128 * 4;
+                   M_ST_READY = 40, M_ST_FREE = 48, M_AP = 56, M_YW = 64, M_GFREE = 72;
+constexpr int kBarsP = 9 + kRing;
+constexpr uint32_t M_BETA = 512;      // beta[64]
+constexpr uint32_t M_GA = 768;        // gamma at token 31, per channel (log2 units)
+constexpr uint32_t M_GC = 1280;       // gamma at token 63 (log2 units)
+constexpr uint32_t M_RHF = 1792;      // e^{gamma_C - gamma_s} per channel
+constexpr uint32_t M_DT = 2304;       // kGate: dt_bias of this head [128]
+constexpr uint32_t kMiscP = M_DT + 512;
 // consumer barriers ([X ; O] and delta per half; A, B parts per slot; V per half and slot)
 constexpr uint32_t M_XO = 0, M_DS = 16, M_AFULL = 32, M_BFULL = 48, M_AFREE = 64, M_BFREE = 80,
                    M_VFULL = 96, M_VFREE = 128, M_GFULL = 160, M_NRM = 208;
@@ -154,7 +147,7 @@ constexpr int kBarsC = 28;
 constexpr uint32_t M_WN = 512;        // kNorm: the norm weight [128]
 constexpr uint32_t M_SS = 1024;       // kNorm: sums of squares [chunk % 2][half][column part][64]
 constexpr uint32_t kMiscC = M_SS + 2 * 2 * 2 * 64 * 4;
-static_assert(M_GT_FREE + 8 <= M_TMEM && 8 * kBarsP == M_GT_FREE + 8 && M_NRM + 16 <= M_TMEM && M_GFULL + 8 * kRing <= M_NRM &&
+static_assert(M_GFREE + 8 * kRing <= M_TMEM && M_NRM + 16 <= M_TMEM && M_GFULL + 8 * kRing <= M_NRM &&
               8 * kBarsC == M_NRM + 16, "barrier area");
 
 constexpr uint32_t kSmemBytes =
@@ -167,10 +160,9 @@ constexpr uint32_t TP_AP = 0, TP_Y = 64, TP_W = 128, kTmemP = 256;
 // state delta at 256 + 64 h
 constexpr uint32_t kTmemC = 512;
 
-// producer warps: 0..7 the back end, 8..15 the front end, 16 I/O. Named barriers: 1 = back end,
-// 2 = front end, 5 = the back end's inverse warps; 1 + h = consumer half h, 3 + h = its output warps
-constexpr int kBack = 256, kFront = 256;
-constexpr int kBarBack = 1, kBarFront = 2, kBarInverse = 5;
+// named barriers: 1 = producer compute warps, 5 = its inverse warps; 1 + h = consumer half h,
+// 3 + h = that half's output warps
+constexpr int kBarCompute = 1, kBarInverse = 5;
 
 struct Params {
     CUtensorMap tq, tk, tg;           // q, k [T,H,128] bf16, g [T,H,128] f32: (128, 1, 64) boxes
@@ -298,9 +290,8 @@ __device__ void unit_of(const Params& p, int unit, int* s_tmp, int& n, int& h, i
 
 // Exact A and P on CUDA cores for a chunk whose decay fails the range test: natural-log gamma
 // from the global g (thread = channel), then one warp per (r, i) pair with lanes over channels,
-// reading q and k from the chunk's shared tiles (kept until the exact path is done). Writes
-// N = diag(beta) A into the inverse's scratch and P into its operand. Rare, so kept out of line.
-// Every back-end thread calls it.
+// reading q and k from the chunk's shared tiles (kept until the exact path is done). Writes N = diag(beta) A into the inverse's scratch and P
+// into its operand. Rare, so kept out of line. Every compute thread calls it.
 template <int MODE>
 __device__ __noinline__ void exact_ap(const Params& p, uint8_t* sm, const float* s_beta, int h,
                                       int64_t c0, int L) {
@@ -324,8 +315,8 @@ __device__ __noinline__ void exact_ap(const Params& p, uint8_t* sm, const float*
             Gx[t * kD + tid] = a;
         }
     }
-    bar_sync(kBarBack, kBack);
-    for (int pidx = warp; pidx < kC * (kC + 1) / 2; pidx += kBack / 32) {
+    bar_sync(kBarCompute, kCompute);
+    for (int pidx = warp; pidx < kC * (kC + 1) / 2; pidx += kCompute / 32) {
         int r = (int)((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
         while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
         while (r * (r + 1) / 2 > pidx) --r;
@@ -469,423 +460,6 @@ __device__ void inverse(uint8_t* sm, const float* s_beta) {
     }
 }
 
-// The front end (warps 8..15) folds task t + 1 while the back end (warps 0..7) finishes task t.
-// Front end, per task: (kConv: the conv prologue in place), the decay sums and the range test,
-// then the folded operands [Lk ; Lq | factors] and R. Back end: [A ; P] = [Lk ; Lq] R^T, the
-// extraction of N and P', the inverse, Yh^T | Wh^T and the staging. They hand over through
-// M_FOLD (front -> back); the front end writes task t + 1's operands only once the back end's
-// A|P product of task t is done (the back end works in order, so every buffer of task t - 1 is
-// free by then) and, with one R buffer (kConv), its Yh product too.
-template <int MODE>
-__device__ __forceinline__ uint32_t r_buf(int task) {
-    return ((MODE & kConv) == 0 && (task & 1)) ? P_V : P_R;
-}
-
-template <int MODE>
-__device__ void front_end(const Params& p, uint8_t* sm, int prank, int n_seq, int h, int64_t bos,
-                          int64_t eos, int ntasks) {
-    constexpr bool kG = (MODE & kGate) != 0;
-    constexpr bool kCv = (MODE & kConv) != 0;
-    constexpr int halo = kCv ? kHalo : 0;
-    const int ft = threadIdx.x - kBack, fw = ft >> 5, lane = threadIdx.x & 31;
-    uint8_t* misc = sm + P_MISC;
-    const int H = p.H;
-    float* s_ga = reinterpret_cast<float*>(misc + M_GA);
-    float* s_gc = reinterpret_cast<float*>(misc + M_GC);
-    float* s_wsum = reinterpret_cast<float*>(misc + M_WSUM);
-    float* facs = reinterpret_cast<float*>(sm + P_LKQ + S_FAC);
-    const int cg = lane & 15, tq = lane >> 4;         // channel group of 8, token quad
-    const int tb = 8 * fw + 4 * tq;                    // this thread's tokens tb .. tb + 3
-    auto chunk_of = [&](int task) { return prank - 1 + kProducers * task; };
-    auto beta_at = [&](int64_t t) {
-        if constexpr (kG) return sigmoid_f(__bfloat162float(p.beta_raw[t * H + h]));
-        else return p.beta[t * H + h];
-    };
-    float cneg = 0.f;                                  // kGate: -exp(A_log[h]) log2(e)
-    if constexpr (kG) {
-        cneg = -expf(p.A_log[h]) * kLog2e;
-        if (ft < kD) reinterpret_cast<float*>(misc + M_DT)[ft] = p.dt_bias[h * kD + ft];
-        bar_sync(kBarFront, kFront);
-    }
-    float beta_nx = 0.f;                               // beta of the next task (threads < 64)
-    if (ntasks > 0 && ft < kC) {
-        const int64_t c0 = bos + (int64_t)chunk_of(0) * kC;
-        if (c0 + ft < eos) beta_nx = beta_at(c0 + ft);
-    }
-    int fail = 0;
-    for (int task = 0; task < ntasks; ++task) {
-        const int n = chunk_of(task);
-        const int64_t c0 = bos + (int64_t)n * kC;
-        const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
-        const uint32_t ph = (uint32_t)task & 1u;
-        const float beta_cur = beta_nx;
-        beta_nx = 0.f;
-        if (task + 1 < ntasks && ft < kC) {
-            const int64_t c1 = bos + (int64_t)chunk_of(task + 1) * kC;
-            if (c1 + ft < eos) beta_nx = beta_at(c1 + ft);
-        }
-        trace_mark(prank, n, 0, kBack);
-        bool ok = wait_warp(bar_at(misc, M_QK_FULL), ph, p);
-        if constexpr (kCv) {
-            // ---- conv prologue, in place: q, k, v of tokens tb .. tb + 3 (8 channels) from the raw
-            //      rows tb - 3 .. tb + 3 (history before the sequence: the conv cache or zero), SiLU,
-            //      and the L2 norm of q and k over the 16 lanes that hold a token's 128 channels.
-            //      Tile row = token + 3. The three rows before tb belong to the thread below and are
-            //      overwritten by it, so every thread reads them first; v goes back row-swizzled
-            //      (16-byte chunk c of a 128-byte half at c ^ (token & 7)), the slot's V layout.
-            uint4 hr[3][3];
-#pragma unroll
-            for (int z = 0; z < 3; ++z) {
-                const uint32_t tile = z == 0 ? P_Q : (z == 1 ? P_K : P_V);
-#pragma unroll
-                for (int j = 0; j < 3; ++j) {
-                    const int r = tb - kHalo + j;                 // token relative to c0
-                    hr[z][j] = ok ? ld16(sm, tile + (r + kHalo) * 256 + cg * 16) : make_uint4(0, 0, 0, 0);
-                    if (ok && c0 + r < bos) {                     // before the sequence
-                        float x[8];
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            float hv = 0.f;
-                            if (p.conv_state != nullptr) {
-                                const int64_t ch = (int64_t)z * H * kD + (int64_t)h * kD + 8 * cg + c;
-                                hv = __bfloat162float(p.conv_state[((int64_t)n_seq * H * 3 * kD + ch) * 3 +
-                                                                   (kHalo - (int)(bos - (c0 + r)))]);
-                            }
-                            x[c] = hv;
-                        }
-                        hr[z][j] = pack8(x);
-                    }
-                }
-            }
-            bar_sync(kBarFront, kFront);
-            if (ok) {
-#pragma unroll
-                for (int z = 0; z < 3; ++z) {
-                    const uint32_t tile = z == 0 ? P_Q : (z == 1 ? P_K : P_V);
-                    const float4* wz = reinterpret_cast<const float4*>(p.wconv[z]) + (size_t)h * kD + 8 * cg;
-                    uint4 w0 = hr[z][0], w1 = hr[z][1], w2 = hr[z][2];   // tokens t - 3, t - 2, t - 1
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int t = tb + u;
-                        const uint4 xt = ld16(sm, tile + (t + kHalo) * 256 + cg * 16);
-                        __syncwarp();                   // (v: the row's other chunks are read first)
-                        float x0[8], x1[8], x2[8], x3[8], y[8];
-                        unpack8(w0, x0);
-                        unpack8(w1, x1);
-                        unpack8(w2, x2);
-                        unpack8(xt, x3);
-                        float ss = 0.f;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const float4 w = __ldg(wz + c);
-                            y[c] = silu_fast(fmaf(w.x, x0[c], fmaf(w.y, x1[c], fmaf(w.z, x2[c], w.w * x3[c]))));
-                            ss = fmaf(y[c], y[c], ss);
-                        }
-                        if (z < 2) {
-#pragma unroll
-                            for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                            const float inv = rsqrtf(ss + p.l2_eps);
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) y[c] *= inv;
-                            st16(sm, tile + (t + kHalo) * 256 + cg * 16, pack8(y));
-                        } else {
-                            st16(sm, P_V + (t + kHalo) * 256 + (cg >> 3) * 128 + (((cg & 7) ^ (t & 7)) << 4),
-                                 pack8(y));
-                        }
-                        w0 = w1;
-                        w1 = w2;
-                        w2 = xt;
-                    }
-                }
-            }
-        }
-        ok = ok && wait_warp(bar_at(misc, M_G_FULL), ph, p);
-        trace_mark(prank, n, 1, kBack);
-        // ---- fold, part 1: decay sums (log2 units) over this thread's 4 tokens, then the warp's 8 ----
-        float s[4][8], xo[8];
-        if (ok) {
-            const float* dt = reinterpret_cast<const float*>(misc + M_DT) + 8 * cg;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int t = tb + u;
-                float gv[8];
-                if constexpr (kG) {
-                    float x[8];
-                    unpack8(ld16(sm, P_G + t * 256 + cg * 16), x);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) gv[c] = cneg * softplus_fast(x[c] + dt[c]);
-                } else {
-                    const float4* G = reinterpret_cast<const float4*>(sm + P_G);
-                    const float4 a0 = G[t * 32 + 2 * cg], a1 = G[t * 32 + 2 * cg + 1];
-                    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) gv[c] = av[c] * kLog2e;
-                }
-                const float m = t < L ? 1.f : 0.f;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) s[u][c] = fmaf(gv[c], m, u ? s[u - 1][c] : 0.f);
-            }
-        } else {
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) s[u][c] = 0.f;
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) xo[c] = __shfl_xor_sync(0xffffffffu, s[3][c], 16);
-        if (ok && tq == 0) {
-            float4* W = reinterpret_cast<float4*>(s_wsum + fw * kD + 8 * cg);
-            W[0] = make_float4(s[3][0] + xo[0], s[3][1] + xo[1], s[3][2] + xo[2], s[3][3] + xo[3]);
-            W[1] = make_float4(s[3][4] + xo[4], s[3][5] + xo[5], s[3][6] + xo[6], s[3][7] + xo[7]);
-        }
-        fail |= !ok;
-        if (bar_sync_or(kBarFront, kFront, fail)) break;
-        if (ft == 0) mbar_arrive(bar_at(misc, M_GT_FREE));   // the g tile is dead
-        // ---- exclusive prefix over the 8 warps, per channel; range test ----
-        int bad_c = 0;
-        if (ft < kD) {
-            float run = 0.f, ga = 0.f;
-#pragma unroll
-            for (int ww = 0; ww < 8; ++ww) {
-                const float v = s_wsum[ww * kD + ft];
-                s_wsum[ww * kD + ft] = run;
-                run += v;
-                if (ww == 3) ga = run;
-            }
-            s_ga[ft] = ga;
-            s_gc[ft] = run;
-            const float kHalf2 = kHalfRange * kLog2e;
-            bad_c = (ga < -kHalf2) || (run - ga < -kHalf2);
-        }
-        const bool bad = bar_sync_or(kBarFront, kFront, bad_c) != 0;
-        // ---- the buffers of task - 1 (see above) ----
-        if (task > 0) {
-            const uint32_t pp = ph ^ 1u;
-            ok = wait_warp(bar_at(misc, M_AP), pp, p) && wait_warp(bar_at(misc, M_LKQ_FREE), pp, p) &&
-                 (!kCv || wait_warp(bar_at(misc, M_YW), pp, p));
-        }
-        trace_mark(prank, n, 2, kBack);
-        // ---- fold, part 2: folded operands Lk, Lq (A of A|P and of the consumer's X | O), R ----
-        if (ok) {
-            const int ac = cg >> 3, ch = cg & 7;
-            const uint32_t rb = r_buf<MODE>(task);
-            {
-                const float4* W = reinterpret_cast<const float4*>(s_wsum + fw * kD + 8 * cg);
-                const float4 w0 = W[0], w1 = W[1];
-                const float off[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float base = off[c] + (tq ? xo[c] : 0.f);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) s[u][c] += base;
-                }
-            }
-            float gr[8], gs[8];
-            {
-                const float4* GA = reinterpret_cast<const float4*>(s_ga + 8 * cg);
-                const float4* GC = reinterpret_cast<const float4*>(s_gc + 8 * cg);
-                const float4 ga0 = GA[0], ga1 = GA[1], gc0 = GC[0], gc1 = GC[1];
-                const float gav[8] = {ga0.x, ga0.y, ga0.z, ga0.w, ga1.x, ga1.y, ga1.z, ga1.w};
-                const float gcv[8] = {gc0.x, gc0.y, gc0.z, gc0.w, gc1.x, gc1.y, gc1.z, gc1.w};
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    gr[c] = bad ? 0.f : gav[c];
-                    gs[c] = bad ? gcv[c] : gav[c];
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int t = tb + u;
-                const bool valid = t < L;
-                float qv[8], kv[8];
-                unpack8(ld16(sm, P_Q + (t + halo) * 256 + cg * 16), qv);
-                unpack8(ld16(sm, P_K + (t + halo) * 256 + cg * 16), kv);
-                uint32_t lk[4], lq[4], rr[4];
-#pragma unroll
-                for (int c = 0; c < 8; c += 2) {
-                    const float a0 = ex2_approx(s[u][c] - gr[c]), a1 = ex2_approx(s[u][c + 1] - gr[c + 1]);
-                    const float b0 = ex2_approx(gs[c] - s[u][c]), b1 = ex2_approx(gs[c + 1] - s[u][c + 1]);
-                    const float k0 = valid ? kv[c] : 0.f, k1 = valid ? kv[c + 1] : 0.f;
-                    const float q0 = valid ? qv[c] : 0.f, q1 = valid ? qv[c + 1] : 0.f;
-                    lk[c / 2] = pack_bf16(k0 * a0, k1 * a1);
-                    lq[c / 2] = pack_bf16(q0 * a0, q1 * a1);
-                    rr[c / 2] = pack_bf16(k0 * b0, k1 * b1);
-                }
-                st16(sm, P_LKQ + sw128(t, ch, ac, 128), make_uint4(lk[0], lk[1], lk[2], lk[3]));
-                st16(sm, P_LKQ + sw128(64 + t, ch, ac, 128), make_uint4(lq[0], lq[1], lq[2], lq[3]));
-                st16(sm, rb + sw128(t, ch, ac, 64), make_uint4(rr[0], rr[1], rr[2], rr[3]));
-            }
-            if (ft < kD) {
-                const float ga = s_ga[ft], gc = s_gc[ft];
-                const float gra = bad ? 0.f : ga, gsa = bad ? gc : ga;
-                facs[ft] = ex2_approx(gra);
-                facs[kD + ft] = ex2_approx(gc);
-                reinterpret_cast<float*>(misc + M_RHF)[128 * ph + ft] = ex2_approx(gc - gsa);
-            }
-            if (ft < kC) reinterpret_cast<float*>(misc + M_BETA)[64 * ph + ft] = beta_cur;
-            if (ft == 0) reinterpret_cast<int*>(misc + M_BAD)[ph] = bad ? 1 : 0;
-        }
-        fail |= !ok;
-        fence_async_smem();
-        if (bar_sync_or(kBarFront, kFront, fail)) break;
-        trace_mark(prank, n, 3, kBack);
-        if (ft == 0) {
-            if (!bad) mbar_arrive(bar_at(misc, M_RAW_FREE));   // the q, k (v) tiles are dead
-            mbar_arrive(bar_at(misc, M_LKQ_READY));            // [Lk ; Lq | factors] may leave
-            mbar_arrive(bar_at(misc, M_FOLD));                 // the back end may start
-        }
-    }
-}
-
-template <int MODE>
-__device__ void back_end(const Params& p, uint8_t* sm, uint32_t sb, int prank, int h, int64_t bos,
-                         int64_t eos, int ntasks) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint8_t* misc = sm + P_MISC;
-    const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
-    const int q4 = warp & 3, cb = warp >> 2;           // TMEM lane quarter, 32-column block
-    const uint32_t lane_sel = (uint32_t)(32 * q4) << 16;
-    auto chunk_of = [&](int task) { return prank - 1 + kProducers * task; };
-    int ap_issued = 0, ap_waited = 0, yw_issued = 0, yw_waited = 0;   // warp 0's products
-    int fail = 0;
-    for (int task = 0; task < ntasks; ++task) {
-        const int n = chunk_of(task);
-        const int64_t c0 = bos + (int64_t)n * kC;
-        const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
-        const uint32_t ph = (uint32_t)task & 1u;
-        const uint32_t rb = r_buf<MODE>(task);
-        const float* s_beta = reinterpret_cast<const float*>(misc + M_BETA) + 64 * ph;
-        const float* s_rhf = reinterpret_cast<const float*>(misc + M_RHF) + 128 * ph;
-        bool ok = wait_warp(bar_at(misc, M_FOLD), ph, p);
-        const bool bad = ok && reinterpret_cast<const volatile int*>(misc + M_BAD)[ph] != 0;
-        trace_mark(prank, n, 4);
-        if (warp == 0 && ok) {                          // [A ; P] = [Lk ; Lq] R^T
-            tc_fence_after();
-            if (elect_one()) {
-                const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16(tm + TP_AP, make_desc(sb + P_LKQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             make_desc(sb + rb + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), id, s > 0);
-                mma_commit(bar_at(misc, M_AP));
-            }
-            __syncwarp();
-            ++ap_issued;
-        }
-        // ---- extraction: N = diag(beta) A (strictly lower, fp32), P' (inclusive, bf16) ----
-        ok = ok && wait_warp(bar_at(misc, M_AP), ph, p);
-        trace_mark(prank, n, 5);
-        if (warp == 0 && ok) ++ap_waited;
-        tc_fence_after();
-        if (ok && !bad) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                float val[16];
-                const int i0 = 32 * cb + 16 * j;
-                tmem_ld16(tm + lane_sel + TP_AP + i0, val);
-                if (q4 < 2) {
-                    const int r = 32 * q4 + lane;
-                    const float br = s_beta[r];
-                    float* Nr = reinterpret_cast<float*>(sm + P_NM) + r * kLd + i0;
-#pragma unroll
-                    for (int i4 = 0; i4 < 4; ++i4) {
-                        float4 w;
-                        w.x = (i0 + 4 * i4 + 0 < r) ? br * val[4 * i4 + 0] : 0.f;
-                        w.y = (i0 + 4 * i4 + 1 < r) ? br * val[4 * i4 + 1] : 0.f;
-                        w.z = (i0 + 4 * i4 + 2 < r) ? br * val[4 * i4 + 2] : 0.f;
-                        w.w = (i0 + 4 * i4 + 3 < r) ? br * val[4 * i4 + 3] : 0.f;
-                        reinterpret_cast<float4*>(Nr)[i4] = w;
-                    }
-                } else {
-                    const int r = 32 * (q4 - 2) + lane;
-#pragma unroll
-                    for (int k8 = 0; k8 < 2; ++k8) {
-                        float pv[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) pv[u] = (i0 + 8 * k8 + u <= r) ? val[8 * k8 + u] : 0.f;
-                        st16(sm, P_PO + sw128(r, (i0 >> 3) + k8, 0, 0), pack8(pv));
-                    }
-                }
-            }
-        }
-        fail |= !ok;
-        if (bad) {
-            // the exact path uses the staging as scratch: the previous chunk must have left it
-            ok = task == 0 || wait_warp(bar_at(misc, M_ST_FREE), ph ^ 1u, p);
-            fail |= !ok;
-            if (bar_sync_or(kBarBack, kBack, fail)) break;
-            exact_ap<MODE>(p, sm, s_beta, h, c0, L);
-        }
-        fence_async_smem();
-        if (bar_sync_or(kBarBack, kBack, fail)) break;
-        if (bad && tid == 0) mbar_arrive(bar_at(misc, M_RAW_FREE));   // the exact path is done
-        trace_mark(prank, n, 6);
-        // ---- T' = (I + N)^-1 diag(beta) on warps 0..3 ----
-        if (warp < 4) inverse(sm, s_beta);
-        fence_async_smem();
-        bar_sync(kBarBack, kBack);
-        trace_mark(prank, n, 7);
-        // ---- Yh^T = R^T T' (M = key ch) and Wh^T = P' T' (M = token) ----
-        if (warp == 0) {
-            tc_fence_after();
-            if (elect_one()) {
-                const uint32_t idY = idesc_bf16(128, 64, true, true);
-                const uint32_t idW = idesc_bf16(128, 64, false, true);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tm + TP_Y, make_desc(sb + rb + s * 2048, 8192, 1024),
-                             make_desc(sb + P_TP + s * 2048, 8192, 1024), idY, s > 0);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tm + TP_W, make_desc(sb + P_PO + s * 32, 16, 1024),
-                             make_desc(sb + P_TP + s * 2048, 8192, 1024), idW, s > 0);
-                mma_commit(bar_at(misc, M_YW));
-            }
-            __syncwarp();
-            ++yw_issued;
-        }
-        ok = wait_warp(bar_at(misc, M_YW), ph, p);
-        trace_mark(prank, n, 8);
-        if (warp == 0 && ok) ++yw_waited;
-        if (ok && !bad && task > 0) ok = wait_warp(bar_at(misc, M_ST_FREE), ph ^ 1u, p);
-        tc_fence_after();
-        // ---- staging: Yh^T rows scaled by e^{gamma_C - gamma_s}, then Wh^T, as bf16 ----
-        if (ok) {
-            const int c = 32 * q4 + lane;
-            const float f = s_rhf[c];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int k16 = 2 * cb + j;              // 16-column block
-                float val[16];
-                tmem_ld16(tm + lane_sel + TP_Y + 16 * k16, val);
-#pragma unroll
-                for (int u = 0; u < 16; ++u) val[u] *= f;
-                st16(sm, P_ST + sw128(c, 2 * k16, 0, 0), pack8(val));
-                st16(sm, P_ST + sw128(c, 2 * k16 + 1, 0, 0), pack8(val + 8));
-                if (q4 < 2) {
-                    tmem_ld16(tm + lane_sel + TP_W + 16 * k16, val);
-                    st16(sm, P_ST + sw128(128 + c, 2 * k16, 0, 0), pack8(val));
-                    st16(sm, P_ST + sw128(128 + c, 2 * k16 + 1, 0, 0), pack8(val + 8));
-                }
-            }
-        }
-        fail |= !ok;
-        fence_async_smem();
-        tc_fence_before();
-        if (bar_sync_or(kBarBack, kBack, fail)) break;
-        if (tid == 0) mbar_arrive(bar_at(misc, M_ST_READY));
-        trace_mark(prank, n, 9);
-    }
-    // products still in flight must finish before the tensor memory is freed (the last commit
-    // on each barrier covers every earlier product)
-    if (warp == 0) {
-        if (ap_issued > ap_waited)
-            mbar_wait(bar_at(misc, M_AP), (uint32_t)(ap_issued - 1) & 1u, kDefaultWaitCycles);
-        if (yw_issued > yw_waited)
-            mbar_wait(bar_at(misc, M_YW), (uint32_t)(yw_issued - 1) & 1u, kDefaultWaitCycles);
-    }
-}
-
 template <int MODE>
 __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, int n_seq, int h,
                          int64_t bos, int64_t eos, bool aborted) {
@@ -894,16 +468,18 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
     constexpr uint32_t kGBytes = kG ? 16384u : 32768u;   // raw logits bf16, or g fp32
     constexpr int halo = kCv ? kHalo : 0;
     constexpr uint32_t kTileBytes = (kC + halo) * 256;   // one q / k / v tile
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* misc = sm + P_MISC;
+    const uint32_t tm = *reinterpret_cast<uint32_t*>(misc + M_TMEM);
+    const int H = p.H;
     const int nchunks = (int)((eos - bos + kC - 1) / kC);
-    const int ntasks = aborted ? 0 : (nchunks >= prank ? (nchunks - prank) / kProducers + 1 : 0);
+    const int ntasks = nchunks >= prank ? (nchunks - prank) / kProducers + 1 : 0;
     const uint32_t c_misc = map_to_rank(sb + C_MISC, 0);
     auto chunk_of = [&](int task) { return prank - 1 + kProducers * task; };
 
     if (warp == kIoWarp) {
-        // ---------------- I/O warp: lane 0 loads tiles, lanes 1 and 2 store and announce ----------
-        if (lane == 0 && ntasks > 0) {
+        // ---------------- I/O warp: lane 0 loads tiles, lane 1 stores and announces ----------
+        if (lane == 0 && !aborted && ntasks > 0) {
             auto issue_qkv = [&](int task) {
                 const int c0 = (int)(bos + (int64_t)chunk_of(task) * kC) - halo;
                 mbar_arrive_expect_tx(bar_at(misc, M_QK_FULL), (kCv ? 3u : 2u) * kTileBytes);
@@ -920,21 +496,18 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             issue_g(0);
             int last_qkv = 0, last_g = 0;
             for (int task = 0; task + 1 < ntasks; ++task) {
-                // the g tile is dead after the fold's first part, the q, k tiles after its second
-                if (!wait_one(bar_at(misc, M_GT_FREE), task & 1, p)) break;
-                issue_g(task + 1);
-                last_g = task + 1;
                 if (!wait_one(bar_at(misc, M_RAW_FREE), task & 1, p)) break;
-                // with kConv the v tile holds the conv's v until that leaves with the A part
-                if (kCv && !wait_one(bar_at(misc, M_LKQ_FREE), task & 1, p)) break;
                 issue_qkv(task + 1);
                 last_qkv = task + 1;
+                // with kConv the g tile holds the conv's v until that leaves with the A part
+                if (kCv && !wait_one(bar_at(misc, M_LKQ_FREE), task & 1, p)) break;
+                issue_g(task + 1);
+                last_g = task + 1;
             }
             // the tiles of the last loads must land before the CTA may leave
             mbar_wait(bar_at(misc, M_QK_FULL), last_qkv & 1, kDefaultWaitCycles);
             mbar_wait(bar_at(misc, M_G_FULL), last_g & 1, kDefaultWaitCycles);
-        } else if (lane == 1 && ntasks > 0) {
-            // A parts (and v after the conv) into the ring as soon as the fold is done
+        } else if (lane == 1 && !aborted && ntasks > 0) {
             uint8_t* ring = p.ring + (size_t)ld_cluster_u32(c_misc + M_SMID) * ((size_t)kRing * kSlotBytes);
             uint32_t ph_gfree = 0;
             for (int task = 0; task < ntasks; ++task) {
@@ -948,50 +521,387 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                     if (!ok) break;
                 }
                 bulk_store(slot + S_LKQ, sb + P_LKQ, kAPart);
-                if constexpr (kCv) bulk_store(slot + S_V, sb + P_V + kHalo * 256, kVPart);
+                if constexpr (kCv) bulk_store(slot + S_V, sb + P_G, kVPart);
                 bulk_commit();
                 bulk_wait_read0();
                 mbar_arrive(bar_at(misc, M_LKQ_FREE));
-                bulk_wait0();                          // written: lane 2 may announce the chunk
-                // (not before lane 2 has announced the previous one, so that the barrier is
-                // never two phases ahead of its waiter)
-                if (task > 0 && !wait_one(bar_at(misc, M_ANNC), (task - 1) & 1, p)) break;
-                mbar_arrive(bar_at(misc, M_A_DONE));
-            }
-            bulk_wait0();
-        } else if (lane == 2 && ntasks > 0) {
-            // B parts, then the announcement once both parts of the chunk are written. Like lane 1,
-            // this lane waits until the consumer has handed the slot back (the slot's next hand-back
-            // needs this chunk's announcement, so the wait never sees a later phase)
-            uint8_t* ring = p.ring + (size_t)ld_cluster_u32(c_misc + M_SMID) * ((size_t)kRing * kSlotBytes);
-            uint32_t ph_gfree = 0;
-            for (int task = 0; task < ntasks; ++task) {
-                const int n = chunk_of(task);
-                const int rs = n % kRing;
-                uint8_t* slot = ring + (size_t)rs * kSlotBytes;
                 if (!wait_one(bar_at(misc, M_ST_READY), task & 1, p)) break;
-                if (n >= kRing) {
-                    const bool ok = wait_one(bar_at(misc, M_GFREE + 8u * rs), (ph_gfree >> rs) & 1u, p, true);
-                    ph_gfree ^= 1u << rs;
-                    if (!ok) break;
-                }
                 bulk_store(slot + S_YW, sb + P_ST, kBPart);
                 bulk_commit();
                 bulk_wait_read0();
                 mbar_arrive(bar_at(misc, M_ST_FREE));
                 bulk_wait0();
-                if (!wait_one(bar_at(misc, M_A_DONE), task & 1, p)) break;
                 fence_proxy_async_global();
                 mbar_arrive_remote(c_misc + M_GFULL + 8u * (uint32_t)rs);
-                mbar_arrive(bar_at(misc, M_ANNC));
             }
             bulk_wait0();
         }
         __syncwarp();
         return;
     }
-    if (warp >= kBack / 32) front_end<MODE>(p, sm, prank, n_seq, h, bos, eos, ntasks);
-    else back_end<MODE>(p, sm, sb, prank, h, bos, eos, ntasks);
+
+    // ---------------- compute warps ----------------
+    float* s_beta = reinterpret_cast<float*>(misc + M_BETA);
+    float* s_ga = reinterpret_cast<float*>(misc + M_GA);
+    float* s_gc = reinterpret_cast<float*>(misc + M_GC);
+    float* s_rhf = reinterpret_cast<float*>(misc + M_RHF);
+    float* s_wsum = reinterpret_cast<float*>(sm + P_NM);   // (the inverse's scratch is idle)
+    float* facs = reinterpret_cast<float*>(sm + P_LKQ + S_FAC);
+    const int cg = lane & 15, tp = lane >> 4;           // fold: channel group of 8, token pair
+    const int t0 = 4 * warp + 2 * tp;                   // fold: tokens t0, t0 + 1
+    const int q4 = warp & 3, cb = warp >> 2;            // TMEM lane quarter, 16-column block
+    const uint32_t lane_sel = (uint32_t)(32 * q4) << 16;
+    int ap_issued = 0, ap_waited = 0, yw_issued = 0, yw_waited = 0;   // warp 0's products
+    auto beta_at = [&](int64_t t) {
+        if constexpr (kG) return sigmoid_f(__bfloat162float(p.beta_raw[t * H + h]));
+        else return p.beta[t * H + h];
+    };
+    float cneg = 0.f;                                   // kGate: -exp(A_log[h]) log2(e)
+    if constexpr (kG) {
+        cneg = -expf(p.A_log[h]) * kLog2e;
+        if (tid < kD) reinterpret_cast<float*>(misc + M_DT)[tid] = p.dt_bias[h * kD + tid];
+        bar_sync(kBarCompute, kCompute);
+    }
+    float beta_nx = 0.f;                                // beta of the next task (threads < 64)
+    if (ntasks > 0 && tid < kC) {
+        const int64_t c0 = bos + (int64_t)chunk_of(0) * kC;
+        if (c0 + tid < eos) beta_nx = beta_at(c0 + tid);
+    }
+    int fail = aborted ? 1 : 0;
+    for (int task = 0; task < ntasks && !aborted; ++task) {
+        const int n = chunk_of(task);
+        const int64_t c0 = bos + (int64_t)n * kC;
+        const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
+        const uint32_t ph = (uint32_t)task & 1u;
+        if (tid < kC) s_beta[tid] = beta_nx;
+        beta_nx = 0.f;
+        if (task + 1 < ntasks && tid < kC) {
+            const int64_t c1 = bos + (int64_t)chunk_of(task + 1) * kC;
+            if (c1 + tid < eos) beta_nx = beta_at(c1 + tid);
+        }
+        trace_mark(prank, n, 0);
+        bool ok = wait_warp(bar_at(misc, M_QK_FULL), ph, p) && wait_warp(bar_at(misc, M_G_FULL), ph, p) &&
+                  (task == 0 || wait_warp(bar_at(misc, M_LKQ_FREE), ph ^ 1u, p));
+        trace_mark(prank, n, 1);
+        // ---- fold, part 1: decay sums (log2 units) of the token pair, then of the warp's 4 tokens ----
+        float s0[8], s1[8], xo[8];
+        if (ok) {
+            float ga[8], gb[8];                          // log-decay of tokens t0, t0 + 1 (log2)
+            if constexpr (kG) {
+                float xa[8], xb[8];
+                unpack8(ld16(sm, P_G + t0 * 256 + cg * 16), xa);
+                unpack8(ld16(sm, P_G + (t0 + 1) * 256 + cg * 16), xb);
+                const float* dt = reinterpret_cast<const float*>(misc + M_DT) + 8 * cg;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    ga[c] = cneg * softplus_fast(xa[c] + dt[c]);
+                    gb[c] = cneg * softplus_fast(xb[c] + dt[c]);
+                }
+            } else {
+                const float4* G = reinterpret_cast<const float4*>(sm + P_G);
+                const float4 a0 = G[t0 * 32 + 2 * cg], a1 = G[t0 * 32 + 2 * cg + 1];
+                const float4 b0 = G[(t0 + 1) * 32 + 2 * cg], b1 = G[(t0 + 1) * 32 + 2 * cg + 1];
+                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    ga[c] = av[c] * kLog2e;
+                    gb[c] = bv[c] * kLog2e;
+                }
+            }
+            const float m0 = t0 < L ? 1.f : 0.f, m1 = t0 + 1 < L ? 1.f : 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                s0[c] = ga[c] * m0;
+                s1[c] = fmaf(gb[c], m1, s0[c]);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) s0[c] = s1[c] = 0.f;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xo[c] = __shfl_xor_sync(0xffffffffu, s1[c], 16);
+        if (ok && tp == 0) {
+            float4* W = reinterpret_cast<float4*>(s_wsum + warp * kD + 8 * cg);
+            W[0] = make_float4(s1[0] + xo[0], s1[1] + xo[1], s1[2] + xo[2], s1[3] + xo[3]);
+            W[1] = make_float4(s1[4] + xo[4], s1[5] + xo[5], s1[6] + xo[6], s1[7] + xo[7]);
+        }
+        fail |= !ok;
+        if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+        // ---- exclusive prefix over the 16 warps, per channel; range test ----
+        int bad_c = 0;
+        if (tid < kD) {
+            float run = 0.f, ga = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < 16; ++ww) {
+                const float v = s_wsum[ww * kD + tid];
+                s_wsum[ww * kD + tid] = run;
+                run += v;
+                if (ww == 7) ga = run;
+            }
+            s_ga[tid] = ga;
+            s_gc[tid] = run;
+            const float kHalf2 = kHalfRange * kLog2e;
+            bad_c = (ga < -kHalf2) || (run - ga < -kHalf2);
+        }
+        const bool bad = bar_sync_or(kBarCompute, kCompute, bad_c) != 0;
+        if constexpr (kCv) {
+            // ---- conv prologue: q, k, v of tokens t0, t0 + 1 (8 channels each) from raw rows
+            //      t0 - 3 .. t0 + 1 (history before the sequence: the conv cache or zero), SiLU,
+            //      and the L2 norm of q and k over the 16 lanes that hold a token's 128 channels
+            uint4 outv[2][2];                            // q, k after the conv (v is stored at once)
+#pragma unroll
+            for (int z = 2; z >= 0; --z) {
+                const uint32_t tile = z == 0 ? P_Q : (z == 1 ? P_K : P_V);
+                float y0[8], y1[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) y0[c] = y1[c] = 0.f;
+                const float4* wz = reinterpret_cast<const float4*>(p.wconv[z]) + (size_t)h * kD + 8 * cg;
+#pragma unroll
+                for (int j = 0; j < 5; ++j) {
+                    const int r = t0 - kHalo + j;                 // token row relative to c0
+                    float x[8];
+                    unpack8(ld16(sm, tile + (r + kHalo) * 256 + cg * 16), x);
+                    if (c0 + r < bos) {                           // before the sequence
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            float hv = 0.f;
+                            if (p.conv_state != nullptr) {
+                                const int64_t ch = (int64_t)z * H * kD + (int64_t)h * kD + 8 * cg + c;
+                                hv = __bfloat162float(p.conv_state[((int64_t)n_seq * H * 3 * kD + ch) * 3 +
+                                                                   (kHalo - (int)(bos - (c0 + r)))]);
+                            }
+                            x[c] = hv;
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 w = __ldg(wz + c);
+                        const float wa[4] = {w.x, w.y, w.z, w.w};
+                        if (j <= 3) y0[c] = fmaf(wa[j], x[c], y0[c]);
+                        if (j >= 1) y1[c] = fmaf(wa[j - 1], x[c], y1[c]);
+                    }
+                }
+                float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    y0[c] = silu_fast(y0[c]);
+                    y1[c] = silu_fast(y1[c]);
+                    ss0 = fmaf(y0[c], y0[c], ss0);
+                    ss1 = fmaf(y1[c], y1[c], ss1);
+                }
+                if (z < 2) {
+#pragma unroll
+                    for (int o = 1; o < 16; o <<= 1) {
+                        ss0 += __shfl_xor_sync(0xffffffffu, ss0, o);
+                        ss1 += __shfl_xor_sync(0xffffffffu, ss1, o);
+                    }
+                    const float i0 = rsqrtf(ss0 + p.l2_eps), i1 = rsqrtf(ss1 + p.l2_eps);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        y0[c] *= i0;
+                        y1[c] *= i1;
+                    }
+                }
+                if (z == 2) {                            // the g tile is dead: v goes there now
+                    st16(sm, P_G + (uint32_t)(cg >> 3) * 8192 + sw128(t0, cg & 7, 0, 0), pack8(y0));
+                    st16(sm, P_G + (uint32_t)(cg >> 3) * 8192 + sw128(t0 + 1, cg & 7, 0, 0), pack8(y1));
+                } else {
+                    outv[z][0] = pack8(y0);
+                    outv[z][1] = pack8(y1);
+                }
+            }
+            bar_sync(kBarCompute, kCompute);             // every raw row has been read
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int t = t0 + u;
+                st16(sm, P_Q + (t + kHalo) * 256 + cg * 16, outv[0][u]);
+                st16(sm, P_K + (t + kHalo) * 256 + cg * 16, outv[1][u]);
+            }
+            bar_sync(kBarCompute, kCompute);
+        }
+        // ---- fold, part 2: folded operands Lk, Lq (A of A|P and of the consumer's X | O), R ----
+        {
+            const int ac = cg >> 3, ch = cg & 7;
+            float gam0[8], gam1[8], gr[8], gs[8];
+            {
+                const float4* W = reinterpret_cast<const float4*>(s_wsum + warp * kD + 8 * cg);
+                const float4 w0 = W[0], w1 = W[1];
+                const float off[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float base = off[c] + (tp ? xo[c] : 0.f);
+                    gam0[c] = base + s0[c];
+                    gam1[c] = base + s1[c];
+                }
+                const float4* GA = reinterpret_cast<const float4*>(s_ga + 8 * cg);
+                const float4* GC = reinterpret_cast<const float4*>(s_gc + 8 * cg);
+                const float4 ga0 = GA[0], ga1 = GA[1], gc0 = GC[0], gc1 = GC[1];
+                const float gav[8] = {ga0.x, ga0.y, ga0.z, ga0.w, ga1.x, ga1.y, ga1.z, ga1.w};
+                const float gcv[8] = {gc0.x, gc0.y, gc0.z, gc0.w, gc1.x, gc1.y, gc1.z, gc1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    gr[c] = bad ? 0.f : gav[c];
+                    gs[c] = bad ? gcv[c] : gav[c];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int t = t0 + u;
+                const bool valid = t < L;
+                float qv[8], kv[8];
+                unpack8(ld16(sm, P_Q + (t + halo) * 256 + cg * 16), qv);
+                unpack8(ld16(sm, P_K + (t + halo) * 256 + cg * 16), kv);
+                uint32_t lk[4], lq[4], rr[4];
+#pragma unroll
+                for (int c = 0; c < 8; c += 2) {
+                    const float gm0 = u ? gam1[c] : gam0[c], gm1 = u ? gam1[c + 1] : gam0[c + 1];
+                    const float a0 = ex2_approx(gm0 - gr[c]), a1 = ex2_approx(gm1 - gr[c + 1]);
+                    const float b0 = ex2_approx(gs[c] - gm0), b1 = ex2_approx(gs[c + 1] - gm1);
+                    const float k0 = valid ? kv[c] : 0.f, k1 = valid ? kv[c + 1] : 0.f;
+                    const float q0 = valid ? qv[c] : 0.f, q1 = valid ? qv[c + 1] : 0.f;
+                    lk[c / 2] = pack_bf16(k0 * a0, k1 * a1);
+                    lq[c / 2] = pack_bf16(q0 * a0, q1 * a1);
+                    rr[c / 2] = pack_bf16(k0 * b0, k1 * b1);
+                }
+                st16(sm, P_LKQ + sw128(t, ch, ac, 128), make_uint4(lk[0], lk[1], lk[2], lk[3]));
+                st16(sm, P_LKQ + sw128(64 + t, ch, ac, 128), make_uint4(lq[0], lq[1], lq[2], lq[3]));
+                st16(sm, P_R + sw128(t, ch, ac, 64), make_uint4(rr[0], rr[1], rr[2], rr[3]));
+            }
+            if (tid < kD) {
+                const float ga = s_ga[tid], gc = s_gc[tid];
+                const float gra = bad ? 0.f : ga, gsa = bad ? gc : ga;
+                facs[tid] = ex2_approx(gra);
+                facs[kD + tid] = ex2_approx(gc);
+                s_rhf[tid] = ex2_approx(gc - gsa);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        bar_sync(kBarCompute, kCompute);
+        trace_mark(prank, n, 2);
+        if (tid == 0) {
+            if (!bad) mbar_arrive(bar_at(misc, M_RAW_FREE));   // the q, k (v) tiles are dead
+            mbar_arrive(bar_at(misc, M_LKQ_READY));            // [Lk ; Lq | factors] may leave
+        }
+        if (warp == 0) {                               // [A ; P] = [Lk ; Lq] R^T
+            tc_fence_after();
+            if (elect_one()) {
+                const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tm + TP_AP, make_desc(sb + P_LKQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                             make_desc(sb + P_R + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), id, s > 0);
+                mma_commit(bar_at(misc, M_AP));
+            }
+            __syncwarp();
+            ++ap_issued;
+        }
+        // ---- extraction: N = diag(beta) A (strictly lower, fp32), P' (inclusive, bf16) ----
+        ok = wait_warp(bar_at(misc, M_AP), ph, p);
+        trace_mark(prank, n, 3);
+        if (warp == 0 && ok) ++ap_waited;
+        tc_fence_after();
+        if (ok && !bad) {
+            float val[16];
+            tmem_ld16(tm + lane_sel + TP_AP + 16 * cb, val);
+            const int i0 = 16 * cb;
+            if (q4 < 2) {
+                const int r = 32 * q4 + lane;
+                const float br = s_beta[r];
+                float* Nr = reinterpret_cast<float*>(sm + P_NM) + r * kLd + i0;
+#pragma unroll
+                for (int i4 = 0; i4 < 4; ++i4) {
+                    float4 w;
+                    w.x = (i0 + 4 * i4 + 0 < r) ? br * val[4 * i4 + 0] : 0.f;
+                    w.y = (i0 + 4 * i4 + 1 < r) ? br * val[4 * i4 + 1] : 0.f;
+                    w.z = (i0 + 4 * i4 + 2 < r) ? br * val[4 * i4 + 2] : 0.f;
+                    w.w = (i0 + 4 * i4 + 3 < r) ? br * val[4 * i4 + 3] : 0.f;
+                    reinterpret_cast<float4*>(Nr)[i4] = w;
+                }
+            } else {
+                const int r = 32 * (q4 - 2) + lane;
+#pragma unroll
+                for (int k8 = 0; k8 < 2; ++k8) {
+                    float pv[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) pv[u] = (i0 + 8 * k8 + u <= r) ? val[8 * k8 + u] : 0.f;
+                    st16(sm, P_PO + sw128(r, 2 * cb + k8, 0, 0), pack8(pv));
+                }
+            }
+        }
+        fail |= !ok;
+        if (bad) {
+            // the exact path uses the staging as scratch: the previous chunk must have left it
+            ok = task == 0 || wait_warp(bar_at(misc, M_ST_FREE), ph ^ 1u, p);
+            fail |= !ok;
+            if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+            exact_ap<MODE>(p, sm, s_beta, h, c0, L);
+        }
+        fence_async_smem();
+        if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+        if (bad && tid == 0) mbar_arrive(bar_at(misc, M_RAW_FREE));   // the exact path is done
+        trace_mark(prank, n, 4);
+        // ---- T' = (I + N)^-1 diag(beta) on warps 0..3 ----
+        if (warp < 4) inverse(sm, s_beta);
+        fence_async_smem();
+        bar_sync(kBarCompute, kCompute);
+        trace_mark(prank, n, 5);
+        // ---- Yh^T = R^T T' (M = key ch) and Wh^T = P' T' (M = token) ----
+        if (warp == 0) {
+            tc_fence_after();
+            if (elect_one()) {
+                const uint32_t idY = idesc_bf16(128, 64, true, true);
+                const uint32_t idW = idesc_bf16(128, 64, false, true);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tm + TP_Y, make_desc(sb + P_R + s * 2048, 8192, 1024),
+                             make_desc(sb + P_TP + s * 2048, 8192, 1024), idY, s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tm + TP_W, make_desc(sb + P_PO + s * 32, 16, 1024),
+                             make_desc(sb + P_TP + s * 2048, 8192, 1024), idW, s > 0);
+                mma_commit(bar_at(misc, M_YW));
+            }
+            __syncwarp();
+            ++yw_issued;
+        }
+        ok = wait_warp(bar_at(misc, M_YW), ph, p);
+        trace_mark(prank, n, 6);
+        if (warp == 0 && ok) ++yw_waited;
+        if (ok && !bad && task > 0) ok = wait_warp(bar_at(misc, M_ST_FREE), ph ^ 1u, p);
+        tc_fence_after();
+        // ---- staging: Yh^T rows scaled by e^{gamma_C - gamma_s}, then Wh^T, as bf16 ----
+        if (ok) {
+            float val[16];
+            const int c = 32 * q4 + lane;
+            tmem_ld16(tm + lane_sel + TP_Y + 16 * cb, val);
+            const float f = s_rhf[c];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) val[u] *= f;
+            st16(sm, P_ST + sw128(c, 2 * cb, 0, 0), pack8(val));
+            st16(sm, P_ST + sw128(c, 2 * cb + 1, 0, 0), pack8(val + 8));
+            if (q4 < 2) {
+                tmem_ld16(tm + lane_sel + TP_W + 16 * cb, val);
+                st16(sm, P_ST + sw128(128 + c, 2 * cb, 0, 0), pack8(val));
+                st16(sm, P_ST + sw128(128 + c, 2 * cb + 1, 0, 0), pack8(val + 8));
+            }
+        }
+        fail |= !ok;
+        fence_async_smem();
+        tc_fence_before();
+        if (bar_sync_or(kBarCompute, kCompute, fail)) break;
+        if (tid == 0) mbar_arrive(bar_at(misc, M_ST_READY));
+        trace_mark(prank, n, 7);
+    }
+    // products still in flight must finish before the tensor memory is freed (the last commit
+    // on each barrier covers every earlier product)
+    if (warp == 0) {
+        if (ap_issued > ap_waited)
+            mbar_wait(bar_at(misc, M_AP), (uint32_t)(ap_issued - 1) & 1u, kDefaultWaitCycles);
+        if (yw_issued > yw_waited)
+            mbar_wait(bar_at(misc, M_YW), (uint32_t)(yw_issued - 1) & 1u, kDefaultWaitCycles);
+    }
 }
 
 // ============================== consumer ==============================
@@ -1022,8 +932,10 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 if (!wait_one(bar_at(misc, M_AFULL + 8 * (mm & 1)), par, p) ||
                     !wait_one(bar_at(misc, M_BFULL + 8 * (mm & 1)), par, p))
                     return false;
-                if constexpr (kCv) {        // the V tile was read from the slot too
-                    if (!wait_one(bar_at(misc, M_VFULL + 8 * (mm & 1)), par, p)) return false;
+                if constexpr (kCv) {        // the V tiles were read from the slot too
+                    if (!wait_one(bar_at(misc, M_VFULL + 8 * (mm & 1)), par, p) ||
+                        !wait_one(bar_at(misc, M_VFULL + 8 * (2 + (mm & 1))), par, p))
+                        return false;
                 }
                 if (mm + kRing < nchunks)
                     mbar_arrive_remote(map_to_rank(sb + P_MISC + M_GFREE + 8u * (uint32_t)(mm % kRing),
@@ -1052,15 +964,14 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 if (!ok) break;
                 fence_proxy_async_global();
                 if constexpr (kCv) {
-                    // the conv's v for both halves in one copy (rows of 128 channels, each 128-byte
-                    // half row-swizzled), once both halves are done with the buffer
-                    if (m >= 2 && !((ok = wait_one(bar_at(misc, M_VFREE + 8 * sl), pfree, p)) &&
-                                    (ok = wait_one(bar_at(misc, M_VFREE + 8 * (2 + sl)), pfree, p))))
-                        break;
-                    uint64_t* vf = bar_at(misc, M_VFULL + 8 * sl);
-                    mbar_arrive_expect_tx(vf, 2 * 8192u);
-                    bulk_load(sb + C_V + (uint32_t)sl * 16384, slot + S_V, 2 * 8192u, vf);
-                    v_issued = m + 1;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint64_t* vf = bar_at(misc, M_VFULL + 8 * (2 * hh + sl));
+                        if (m >= 2 && !(ok = wait_one(bar_at(misc, M_VFREE + 8 * (2 * hh + sl)), pfree, p))) break;
+                        mbar_arrive_expect_tx(vf, 8192u);
+                        bulk_load(sb + C_V + (uint32_t)(2 * hh + sl) * 8192, slot + S_V + hh * 8192, 8192u, vf);
+                        v_issued = m + 1;
+                    }
+                    if (!ok) break;
                 }
                 if (m >= 2 && !(ok = wait_one(bar_at(misc, M_AFREE + 8 * sl), pfree, p))) break;
                 mbar_arrive_expect_tx(bar_at(misc, M_AFULL + 8 * sl), kAPart);
@@ -1083,7 +994,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 mbar_wait(bar_at(misc, M_BFULL + 8 * (mm & 1)), par, kDefaultWaitCycles);
             }
             for (int mm = (v_issued > 2 ? v_issued - 2 : 0); mm < v_issued; ++mm)
-                for (int hh = 0; hh < (kCv ? 1 : 2); ++hh)
+                for (int hh = 0; hh < 2; ++hh)
                     mbar_wait(bar_at(misc, M_VFULL + 8 * (2 * hh + (mm & 1))), (uint32_t)(mm >> 1) & 1u,
                               kDefaultWaitCycles);
         }
@@ -1247,13 +1158,10 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         tc_fence_after();
         if (ok && n > 0 && tid_h == 0) mbar_arrive(bar_at(misc, M_BFREE + 8 * ((n - 1) & 1)));
         if (q < 2) {
-            if (ok) ok = wait_warp(bar_at(misc, M_VFULL + 8 * (kCv ? b : 2 * half + b)), (uint32_t)(n >> 1) & 1u, p);
+            if (ok) ok = wait_warp(bar_at(misc, M_VFULL + 8 * (2 * half + b)), (uint32_t)(n >> 1) & 1u, p);
             if (ok) {
                 const int t = 32 * q + lane;
-                // this half's 64 columns of token t: a 128-byte SW128 row (kConv: half of a 256-byte
-                // row of both halves, swizzled the same way)
-                const uint8_t* vt = kCv ? sm + C_V + (uint32_t)b * 16384 + t * 256 + half * 128
-                                        : sm + C_V + (uint32_t)(2 * half + b) * 8192 + t * 128;
+                const uint8_t* vt = sm + C_V + (uint32_t)(2 * half + b) * 8192;
 #pragma unroll
                 for (int hx = 0; hx < 2; ++hx) {
                     float xv[16];
@@ -1262,7 +1170,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                     for (int k2 = 0; k2 < 2; ++k2) {
                         const int ck = 4 * cp + 2 * hx + k2;
                         float vv[8];
-                        unpack8(ld16(vt, (ck ^ (t & 7)) << 4), vv);
+                        unpack8(ld16(vt, t * 128 + ((ck ^ (t & 7)) << 4)), vv);
 #pragma unroll
                         for (int u = 0; u < 8; ++u) vv[u] -= xv[8 * k2 + u];
                         st16(sm, u_h + sw128(t, ck, 0, 0), pack8(vv));
@@ -1281,7 +1189,6 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         // (2) state delta Yh^T U (commit), then O(n) += Wh^T U
         if (issuer) {
             if (wait_warp(bar_at(misc, M_BFULL + 8 * b), (uint32_t)(n >> 1) & 1u, p)) {
-                trace_mark(0, n, 8 * half + 4, 256 * half);
                 tc_fence_after();
                 if (elect_one()) {
                     const uint32_t id = idesc_bf16(128, 64, false, true);
@@ -1318,7 +1225,6 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             }
             if (n + 1 < nchunks) {
                 ok = wait_warp(bar_at(misc, M_AFULL + 8 * ((n + 1) & 1)), (uint32_t)((n + 1) >> 1) & 1u, p);
-                trace_mark(0, n, 8 * half + 5, 256 * half);
                 if (ok) write_sm(n + 1);
             }
         }
