@@ -140,15 +140,16 @@ constexpr uint32_t M_GC = 1280;       // gamma at token 63 (log2 units)
 constexpr uint32_t M_RHF = 1792;      // e^{gamma_C - gamma_s} per channel
 constexpr uint32_t M_DT = 2304;       // kGate: dt_bias of this head [128]
 constexpr uint32_t kMiscP = M_DT + 512;
-// consumer barriers ([X ; O] and delta per half; A, B parts per slot; V per half and slot)
+// consumer barriers ([X ; O] and delta per half; A, B parts per slot; V per half and slot;
+// kNorm: the halves' sums of squares per chunk parity, the output gate z per half)
 constexpr uint32_t M_XO = 0, M_DS = 16, M_AFULL = 32, M_BFULL = 48, M_AFREE = 64, M_BFREE = 80,
-                   M_VFULL = 96, M_VFREE = 128, M_GFULL = 160, M_NRM = 208;
-constexpr int kBarsC = 28;
+                   M_VFULL = 96, M_VFREE = 128, M_GFULL = 160, M_NRM = 208, M_ZFULL = 224;
+constexpr int kBarsC = 30;
 constexpr uint32_t M_WN = 512;        // kNorm: the norm weight [128]
 constexpr uint32_t M_SS = 1024;       // kNorm: sums of squares [chunk % 2][half][column part][64]
 constexpr uint32_t kMiscC = M_SS + 2 * 2 * 2 * 64 * 4;
-static_assert(M_GFREE + 8 * kRing <= M_TMEM && M_NRM + 16 <= M_TMEM && M_GFULL + 8 * kRing <= M_NRM &&
-              8 * kBarsC == M_NRM + 16, "barrier area");
+static_assert(M_GFREE + 8 * kRing <= M_TMEM && M_ZFULL + 16 <= M_TMEM && M_GFULL + 8 * kRing <= M_NRM &&
+              8 * kBarsC == M_ZFULL + 16, "barrier area");
 
 constexpr uint32_t kSmemBytes =
     ((P_MISC + kMiscP) > (C_MISC + kMiscC) ? (P_MISC + kMiscP) : (C_MISC + kMiscC)) + 1024;
@@ -167,6 +168,7 @@ constexpr int kBarCompute = 1, kBarInverse = 5;
 struct Params {
     CUtensorMap tq, tk, tg;           // q, k [T,H,128] bf16, g [T,H,128] f32: (128, 1, 64) boxes
     CUtensorMap tv, to;               // v, o [T,H,128] bf16: (64, 1, 64) boxes, 128B swizzle
+    CUtensorMap tz;                   // kNorm: the output gate z [T,H,128] bf16, as v
     const __nv_bfloat16* q;           // the exact path reads q, k, g directly
     const __nv_bfloat16* k;
     const float* g;
@@ -1064,11 +1066,12 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         float inv = 0.f;                            // kNorm: 1 / rms of token t over 128 columns
         uint4 zr[4];
         if constexpr (kN) {
-            // the output's gate for this thread's 32 columns (loads in flight during the sums)
-            const uint4* zsrc = reinterpret_cast<const uint4*>(
-                p.z + ((c0 + (t < L ? t : 0)) * H + h) * kD + jg0);
+            // the output's gate for this thread's 32 columns: TMA-loaded into this half's staging
+            // tile a chunk ahead (each thread overwrites exactly the chunks it reads)
+            ok = ok && wait_warp(bar_at(misc, M_ZFULL + 8 * half), (uint32_t)nn & 1u, p);
 #pragma unroll
-            for (int k8 = 0; k8 < 4; ++k8) zr[k8] = ok ? zsrc[k8] : make_uint4(0, 0, 0, 0);
+            for (int k8 = 0; k8 < 4; ++k8)
+                zr[k8] = ok ? ld16(sm, ost_h + sw128(t, 4 * cp + k8, 0, 0)) : make_uint4(0, 0, 0, 0);
             float ss = 0.f;
             if (ok) {
 #pragma unroll
@@ -1139,6 +1142,16 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
 
     bool stop = aborted;
     int fail = aborted ? 1 : 0;
+    // kNorm: the storer of each half loads the output gate of chunk n into its staging tile once
+    // the output of chunk n - 1 has been read from it
+    int z_issued = 0;
+    auto issue_z = [&](int nn) {
+        uint64_t* zf = bar_at(misc, M_ZFULL + 8 * half);
+        mbar_arrive_expect_tx(zf, 8192u);
+        tma_load_3d(sb + ost_h, &p.tz, 64 * half, h, (int)(bos + (int64_t)nn * kC), zf);
+        z_issued = nn + 1;
+    };
+    if (kN && !stop && nchunks > 0 && lw == 2 && lane == 0) issue_z(0);
     // prologue: Sm(0), then [X ; O](0)
     if (!stop && nchunks > 0) {
         const bool ok = wait_warp(bar_at(misc, M_AFULL), 0, p);
@@ -1186,6 +1199,10 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         if (bar_sync_or(bar_half, 256, fail)) { stop = true; break; }
         trace_mark(0, n, 8 * half + 1, 256 * half);
         if (tid_h == 0) mbar_arrive(bar_at(misc, M_VFREE + 8 * (2 * half + b)));
+        if (kN && n > 0 && lw == 2 && lane == 0) {   // (this warp waits for the delta next anyway)
+            bulk_wait_read0();
+            issue_z(n);
+        }
         // (2) state delta Yh^T U (commit), then O(n) += Wh^T U
         if (issuer) {
             if (wait_warp(bar_at(misc, M_BFULL + 8 * b), (uint32_t)(n >> 1) & 1u, p)) {
@@ -1258,7 +1275,11 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) dst[c4] = make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
     }
-    if (lw == 2 && lane == 0) bulk_wait0();
+    if (lw == 2 && lane == 0) {
+        bulk_wait0();
+        if (kN && z_issued > 0)                 // the last gate tile has landed
+            mbar_wait(bar_at(misc, M_ZFULL + 8 * half), (uint32_t)(z_issued - 1) & 1u, kDefaultWaitCycles);
+    }
     // products still in flight must finish before the tensor memory is freed
     if (issuer) {
         if (xo_issued > xo_waited) mbar_wait(bar_xo, (uint32_t)((xo_issued - 1) & 1), kDefaultWaitCycles);
@@ -1291,7 +1312,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
         if (is_consumer) {
             for (int b = 0; b < kBarsC; ++b) {
                 const uint32_t off = 8u * b;
-                const bool two = (off >= M_AFREE && off < M_VFULL) || off >= M_NRM;
+                const bool two = (off >= M_AFREE && off < M_VFULL) || (off >= M_NRM && off < M_ZFULL);
                 mbar_init(bar_at(misc, off), two ? 2 : 1);
             }
             const uint32_t id = smid();
@@ -1355,7 +1376,8 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
               : make_tmap_thd(&p.tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.T_tot, a.H, kD, kD, kC, false)) &&
         (conv ? make_tmap_thd(&p.tv, a.v, BF, 2, a.T_tot, a.H, kD, kD, tile_rows, false)
               : make_tmap_thd(&p.tv, a.v, BF, 2, a.T_tot, a.H, kD, 64, kC, true)) &&
-        make_tmap_thd(&p.to, a.o, BF, 2, a.T_tot, a.H, kD, 64, kC, true);
+        make_tmap_thd(&p.to, a.o, BF, 2, a.T_tot, a.H, kD, 64, kC, true) &&
+        (a.z == nullptr || make_tmap_thd(&p.tz, a.z, BF, 2, a.T_tot, a.H, kD, 64, kC, true));
     if (!maps_ok) return cudaErrorInvalidValue;
     p.q = static_cast<const __nv_bfloat16*>(a.q);
     p.k = static_cast<const __nv_bfloat16*>(a.k);

@@ -89,8 +89,10 @@ __device__ __forceinline__ float silu(float z) {
     }
 }
 
+// The general tile: sequence boundaries inside the tile or its history, the conv cache, and the
+// decode form. Out of line, so that the common tile's code stays small.
 template <typename T, int D>
-__device__ __forceinline__ void conv_unit(const ConvParams& p, int z, int h, int64_t t0) {
+__device__ __noinline__ void conv_unit(const ConvParams& p, int z, int h, int64_t t0) {
     constexpr int CPL = D / 32;
     using Word = typename RawVec<T, CPL>::Word;
     const int lane = threadIdx.x & 31;
@@ -209,6 +211,76 @@ __device__ __forceinline__ void conv_unit(const ConvParams& p, int z, int h, int
     }
 }
 
+// The common tile: kTile tokens and their three predecessors all in one sequence, prefill form.
+// No branch per token; the weights are halved once so that SiLU is h + h tanh(h) straight from
+// the sum (bf16 outputs; the fp32 path keeps its exact SiLU).
+template <typename T, int D>
+__device__ __forceinline__ void conv_tile_inner(const ConvParams& p, int z, int h, int64_t t0) {
+    constexpr int CPL = D / 32;
+    constexpr bool kHalf = sizeof(T) == 2;
+    using Word = typename RawVec<T, CPL>::Word;
+    const int lane = threadIdx.x & 31;
+    const T* __restrict__ x = static_cast<const T*>(z == 0 ? p.x[0] : z == 1 ? p.x[1] : p.x[2]);
+    T* __restrict__ y = static_cast<T*>(z == 0 ? p.y[0] : z == 1 ? p.y[1] : p.y[2]);
+    const float* wz = z == 0 ? p.w[0] : z == 1 ? p.w[1] : p.w[2];
+    const int H = p.H;
+    const int cl = lane * CPL;
+    const int64_t rs = (int64_t)H * D;                             // elements per token
+    const T* xp = x + ((t0 - kHist) * H + h) * D + cl;
+    Word raw[kHist + kTile];
+#pragma unroll
+    for (int m = 0; m < kHist + kTile; ++m) raw[m] = *reinterpret_cast<const Word*>(xp + m * rs);
+    float w[CPL][kTaps];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        const float4 wv = *reinterpret_cast<const float4*>(wz + (int64_t)(h * D + cl + c) * kTaps);
+        const float sc = kHalf ? 0.5f : 1.f;
+        w[c][0] = wv.x * sc; w[c][1] = wv.y * sc; w[c][2] = wv.z * sc; w[c][3] = wv.w * sc;
+    }
+    float hist[kHist][CPL];
+#pragma unroll
+    for (int m = 0; m < kHist; ++m) RawVec<T, CPL>::unpack(raw[m], hist[m]);
+    T* yrow = y + (t0 * H + h) * D + cl;
+    const bool norm = (z < 2);
+#pragma unroll
+    for (int tt = 0; tt < kTile; ++tt) {
+        float xt[CPL], out[CPL];
+        RawVec<T, CPL>::unpack(raw[kHist + tt], xt);
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            float zc = w[c][0] * hist[0][c];
+            zc = fmaf(w[c][1], hist[1][c], zc);
+            zc = fmaf(w[c][2], hist[2][c], zc);
+            zc = fmaf(w[c][3], xt[c], zc);
+            float sv;
+            if constexpr (kHalf) {                                  // zc is already z / 2
+                float th;
+                asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(zc));
+                sv = fmaf(zc, th, zc);
+            } else {
+                sv = silu<T>(zc);
+            }
+            out[c] = sv;
+            ss = fmaf(sv, sv, ss);
+        }
+        if (norm) {
+            ss = warp_sum(ss);
+            const float inv = rsqrtf(ss + p.eps);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) out[c] *= inv;
+        }
+        Vec<T, CPL>::store(yrow, out);
+        yrow += rs;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            hist[0][c] = hist[1][c];
+            hist[1][c] = hist[2][c];
+            hist[2][c] = xt[c];
+        }
+    }
+}
+
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kConvWarps * 32)
 conv_kernel(const ConvParams p) {
@@ -216,8 +288,22 @@ conv_kernel(const ConvParams p) {
     const int h = blockIdx.y * kConvWarps + (threadIdx.x >> 5);
     const int64_t t0 = (int64_t)blockIdx.x * kTile;
     if (h >= p.H || t0 >= p.T_tot) return;
-    if (z < 2) conv_unit<T, DK>(p, z, h, t0);
-    else conv_unit<T, DV>(p, z, h, t0);
+    bool inner = !p.step_mode && t0 >= kHist && t0 + kTile <= p.T_tot;
+    if (inner) {                       // the tile and its history within one sequence?
+        if (p.cu) {
+            const int n = find_seq(p.cu, p.N, t0);
+            inner = t0 - kHist >= p.cu[n] && t0 + kTile <= p.cu[n + 1];
+        } else {
+            inner = (t0 - kHist) / p.T_pad == (t0 + kTile - 1) / p.T_pad;
+        }
+    }
+    if (z < 2) {
+        if (inner) conv_tile_inner<T, DK>(p, z, h, t0);
+        else conv_unit<T, DK>(p, z, h, t0);
+    } else {
+        if (inner) conv_tile_inner<T, DV>(p, z, h, t0);
+        else conv_unit<T, DV>(p, z, h, t0);
+    }
 }
 
 // Prefill mode: new cache[n, c, p] = ext[L + p], ext = (old cache of n, then x of n).
