@@ -39,9 +39,9 @@ MEASURED_TRAFFIC = {
     "prefill_8k": (("chunk_tcx.cu", "tc.cuh", "common.cuh", "tma_host.h"),
                    "0716dc2e7752154918079bf0d08a5f9add4073aca64e868a6b4dd04c972ee6fe", 392807168),
     "conv_8k": (("conv.cu", "common.cuh"),
-                "57851013be10bf43df46ad41c337896a25884525ab4b3b12a15eae74d91c97b3", 357546240),
+                "28908a4c60fb3f184b90005e406d903129202d5acbbcbca4cb52243982fcf542", 365856512),
     "decode_256x32": (("recurrent_step.cu", "common.cuh"),
-                      "77c4ec89d7d467c1f5a8ac71bee67eacdc51b3a44d5a73ae884d6db155449850", 1030215424),
+                      "a963466ab8982d94dcf368779351935ba00f725c3c02a9b04e8dababc04db62e", 1028144128),
 }
 
 
