@@ -139,15 +139,19 @@ constexpr uint32_t M_GA = 768;        // gamma at token 31, per channel (log2 un
 constexpr uint32_t M_GC = 1280;       // gamma at token 63 (log2 units)
 constexpr uint32_t M_RHF = 1792;      // e^{gamma_C - gamma_s} per channel
 constexpr uint32_t M_DT = 2304;       // kGate: dt_bias of this head [128]
-constexpr uint32_t kMiscP = M_DT + 512;
+constexpr uint32_t M_WCV = 2816;      // kConv: this head's conv weights, halved, as float4 (4 taps)
+                                      //   [q, k, v][channel % 8][channel / 8] (a warp's 16
+                                      //   channel groups read 16 consecutive float4)
+constexpr uint32_t kMiscP = M_WCV + 3 * 128 * 16;
 // consumer barriers ([X ; O] and delta per half; A, B parts per slot; V per half and slot;
-// kNorm: the halves' sums of squares per chunk parity, the output gate z per half)
+// kNorm: the halves' sums of squares per chunk parity, each half's output complete, each half's
+// output gate tile)
 constexpr uint32_t M_XO = 0, M_DS = 16, M_AFULL = 32, M_BFULL = 48, M_AFREE = 64, M_BFREE = 80,
-                   M_VFULL = 96, M_VFREE = 128, M_GFULL = 160, M_NRM = 208, M_ZFULL = 224;
-constexpr int kBarsC = 30;
+                   M_VFULL = 96, M_VFREE = 128, M_GFULL = 160, M_NRM = 208, M_OD = 224, M_ZFULL = 240;
+constexpr int kBarsC = 32;
 constexpr uint32_t M_WN = 512;        // kNorm: the norm weight [128]
-constexpr uint32_t M_SS = 1024;       // kNorm: sums of squares [chunk % 2][half][column part][64]
-constexpr uint32_t kMiscC = M_SS + 2 * 2 * 2 * 64 * 4;
+constexpr uint32_t M_SS = 1024;       // kNorm: sums of squares [chunk % 3][half][column part][64]
+constexpr uint32_t kMiscC = M_SS + 3 * 2 * 2 * 64 * 4;
 static_assert(M_GFREE + 8 * kRing <= M_TMEM && M_ZFULL + 16 <= M_TMEM && M_GFULL + 8 * kRing <= M_NRM &&
               8 * kBarsC == M_ZFULL + 16, "barrier area");
 
@@ -168,7 +172,7 @@ constexpr int kBarCompute = 1, kBarInverse = 5;
 struct Params {
     CUtensorMap tq, tk, tg;           // q, k [T,H,128] bf16, g [T,H,128] f32: (128, 1, 64) boxes
     CUtensorMap tv, to;               // v, o [T,H,128] bf16: (64, 1, 64) boxes, 128B swizzle
-    CUtensorMap tz;                   // kNorm: the output gate z [T,H,128] bf16, as v
+    CUtensorMap tz;                   // kNorm: the output gate z [T,H,128] bf16, as o
     const __nv_bfloat16* q;           // the exact path reads q, k, g directly
     const __nv_bfloat16* k;
     const float* g;
@@ -210,11 +214,11 @@ __device__ __forceinline__ float softplus_fast(float x) {
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.f + e));
     return fmaxf(x, 0.f) + l * kLn2;
 }
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
-// silu(z) = z sigmoid(z) = h + h tanh(h), h = z / 2: one tanh.approx (relative error below 2^-10,
-// under the bf16 rounding of its result).
-__device__ __forceinline__ float silu_fast(float z) {
-    const float hz = 0.5f * z;
+// sigmoid with the fast divide (two ulp, far below the bf16 rounding of what it scales; the
+// correctly rounded divide's software sequence cost the normed prefill half its time)
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// silu(z) from h = z / 2: h + h tanh(h) (the conv prologue sums with halved weights).
+__device__ __forceinline__ float silu_half(float hz) {
     float th;
     asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hz));
     return fmaf(hz, th, hz);
@@ -647,6 +651,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             bad_c = (ga < -kHalf2) || (run - ga < -kHalf2);
         }
         const bool bad = bar_sync_or(kBarCompute, kCompute, bad_c) != 0;
+        trace_mark(prank, n, 8);
         if constexpr (kCv) {
             // ---- conv prologue: q, k, v of tokens t0, t0 + 1 (8 channels each) from raw rows
             //      t0 - 3 .. t0 + 1 (history before the sequence: the conv cache or zero), SiLU,
@@ -655,16 +660,14 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
 #pragma unroll
             for (int z = 2; z >= 0; --z) {
                 const uint32_t tile = z == 0 ? P_Q : (z == 1 ? P_K : P_V);
-                float y0[8], y1[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) y0[c] = y1[c] = 0.f;
-                const float4* wz = reinterpret_cast<const float4*>(p.wconv[z]) + (size_t)h * kD + 8 * cg;
+                // the five raw rows t0 - 3 .. t0 + 1 of this thread's 8 channels, packed
+                uint4 rows[5];
 #pragma unroll
                 for (int j = 0; j < 5; ++j) {
                     const int r = t0 - kHalo + j;                 // token row relative to c0
-                    float x[8];
-                    unpack8(ld16(sm, tile + (r + kHalo) * 256 + cg * 16), x);
+                    rows[j] = ld16(sm, tile + (r + kHalo) * 256 + cg * 16);
                     if (c0 + r < bos) {                           // before the sequence
+                        float x[8];
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
                             float hv = 0.f;
@@ -675,20 +678,29 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
                             }
                             x[c] = hv;
                         }
+                        rows[j] = pack8(x);
                     }
+                }
+                // y = (weights / 2) . x, so that SiLU is h + h tanh(h) straight from the sum
+                float y0[8], y1[8];
+                const float4* wz = reinterpret_cast<const float4*>(misc + M_WCV) + z * kD + cg;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float4 w = __ldg(wz + c);
-                        const float wa[4] = {w.x, w.y, w.z, w.w};
-                        if (j <= 3) y0[c] = fmaf(wa[j], x[c], y0[c]);
-                        if (j >= 1) y1[c] = fmaf(wa[j - 1], x[c], y1[c]);
+                for (int c = 0; c < 8; ++c) {
+                    const float4 w = wz[16 * c];
+                    float xc[5];
+#pragma unroll
+                    for (int j = 0; j < 5; ++j) {
+                        const uint32_t wd = (&rows[j].x)[c >> 1];
+                        xc[j] = __uint_as_float((c & 1) ? (wd & 0xffff0000u) : (wd << 16));
                     }
+                    y0[c] = fmaf(w.w, xc[3], fmaf(w.z, xc[2], fmaf(w.y, xc[1], w.x * xc[0])));
+                    y1[c] = fmaf(w.w, xc[4], fmaf(w.z, xc[3], fmaf(w.y, xc[2], w.x * xc[1])));
                 }
                 float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    y0[c] = silu_fast(y0[c]);
-                    y1[c] = silu_fast(y1[c]);
+                    y0[c] = silu_half(y0[c]);
+                    y1[c] = silu_half(y1[c]);
                     ss0 = fmaf(y0[c], y0[c], ss0);
                     ss1 = fmaf(y1[c], y1[c], ss1);
                 }
@@ -722,6 +734,7 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
             }
             bar_sync(kBarCompute, kCompute);
         }
+        trace_mark(prank, n, 9);
         // ---- fold, part 2: folded operands Lk, Lq (A of A|P and of the consumer's X | O), R ----
         {
             const int ac = cg >> 3, ch = cg & 7;
@@ -1066,26 +1079,14 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         float inv = 0.f;                            // kNorm: 1 / rms of token t over 128 columns
         uint4 zr[4];
         if constexpr (kN) {
-            // the output's gate for this thread's 32 columns: TMA-loaded into this half's staging
-            // tile a chunk ahead (each thread overwrites exactly the chunks it reads)
+            // the gate of this thread's 32 outputs: TMA-loaded into the staging tile beforehand
+            // (each thread overwrites exactly the 16-byte chunks it reads)
             ok = ok && wait_warp(bar_at(misc, M_ZFULL + 8 * half), (uint32_t)nn & 1u, p);
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8)
                 zr[k8] = ok ? ld16(sm, ost_h + sw128(t, 4 * cp + k8, 0, 0)) : make_uint4(0, 0, 0, 0);
-            float ss = 0.f;
-            if (ok) {
-#pragma unroll
-                for (int hx = 0; hx < 2; ++hx) {
-                    float ov[16];
-                    tmem_ld16(src + 16 * hx, ov);
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) ss = fmaf(ov[u], ov[u], ss);
-                }
-            }
-            float* s_ss = reinterpret_cast<float*>(misc + M_SS) + (nn & 1) * 256;
-            s_ss[(2 * half + cp) * 64 + t] = ss * p.scale * p.scale;
-            bar_sync(bar_out, 128);
-            if (ok && lw == 2 && lane == 0) mbar_arrive(bar_at(misc, M_NRM + 8 * (nn & 1)));
+            // both halves' sums of squares of chunk nn, published a step earlier (see (3))
+            const float* s_ss = reinterpret_cast<const float*>(misc + M_SS) + (nn % 3) * 256;
             ok = ok && wait_warp(bar_at(misc, M_NRM + 8 * (nn & 1)), (uint32_t)(nn >> 1) & 1u, p);
             if (ok) {
                 const float tot = s_ss[t] + s_ss[64 + t] + s_ss[128 + t] + s_ss[192 + t];
@@ -1142,16 +1143,10 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
 
     bool stop = aborted;
     int fail = aborted ? 1 : 0;
-    // kNorm: the storer of each half loads the output gate of chunk n into its staging tile once
-    // the output of chunk n - 1 has been read from it
+    // kNorm: the storer of each half loads chunk n's output gate into its staging tile in step (4)
+    // of chunk n, well after chunk n - 1's output has been read from it; the epilogue of chunk n
+    // reads it a step later
     int z_issued = 0;
-    auto issue_z = [&](int nn) {
-        uint64_t* zf = bar_at(misc, M_ZFULL + 8 * half);
-        mbar_arrive_expect_tx(zf, 8192u);
-        tma_load_3d(sb + ost_h, &p.tz, 64 * half, h, (int)(bos + (int64_t)nn * kC), zf);
-        z_issued = nn + 1;
-    };
-    if (kN && !stop && nchunks > 0 && lw == 2 && lane == 0) issue_z(0);
     // prologue: Sm(0), then [X ; O](0)
     if (!stop && nchunks > 0) {
         const bool ok = wait_warp(bar_at(misc, M_AFULL), 0, p);
@@ -1190,8 +1185,6 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                     }
                 }
             }
-        } else if (n > 0) {
-            epilogue_o(n - 1, ok);
         }
         fail |= !ok;
         fence_async_smem();
@@ -1199,10 +1192,11 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         if (bar_sync_or(bar_half, 256, fail)) { stop = true; break; }
         trace_mark(0, n, 8 * half + 1, 256 * half);
         if (tid_h == 0) mbar_arrive(bar_at(misc, M_VFREE + 8 * (2 * half + b)));
-        if (kN && n > 0 && lw == 2 && lane == 0) {   // (this warp waits for the delta next anyway)
-            bulk_wait_read0();
-            issue_z(n);
-        }
+        // the output of chunk n - 1, by the output warps, while the delta product runs (this
+        // keeps it off the path from X(n) to the delta)
+        trace_mark(0, n, 8 * half + 4, 256 * half + 64);
+        if (q >= 2 && n > 0) epilogue_o(n - 1, ok);
+        trace_mark(0, n, 8 * half + 6, 256 * half + 64);
         // (2) state delta Yh^T U (commit), then O(n) += Wh^T U
         if (issuer) {
             if (wait_warp(bar_at(misc, M_BFULL + 8 * b), (uint32_t)(n >> 1) & 1u, p)) {
@@ -1219,6 +1213,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                     for (int s = 0; s < 4; ++s)
                         mma_bf16(t_xo + 64 * b, make_desc(bp + 8192 + s * 32, 16, 1024),
                                  make_desc(sb + u_h + s * 2048, 8192, 1024), id, 1);
+                    if (kN) mma_commit(bar_at(misc, M_OD + 8 * half));   // O(n) is complete
                 }
                 __syncwarp();
                 ++ds_issued;
@@ -1240,6 +1235,31 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
 #pragma unroll
                 for (int u = 0; u < 16; ++u) S[16 * hx + u] = fmaf(eC, S[16 * hx + u], dv[u]);
             }
+        }
+        if (kN && q >= 2) {
+            // the output's per-token sums of squares over this half's 64 columns, published for
+            // both halves' epilogues of chunk n (one step later). Three buffers: a half can run
+            // at most two chunks ahead of the other (they share the A buffers).
+            bool oko = ok && wait_warp(bar_at(misc, M_OD + 8 * half), (uint32_t)b, p);
+            trace_mark(0, n, 8 * half + 7, 256 * half + 64);
+            tc_fence_after();
+            float ss = 0.f;
+            if (oko) {
+#pragma unroll
+                for (int hx = 0; hx < 2; ++hx) {
+                    float ov[16];
+                    tmem_ld16(t_xo + 64 * b + lane_sel + 32 * cp + 16 * hx, ov);
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) ss = fmaf(ov[u], ov[u], ss);
+                }
+            }
+            float* s_ss = reinterpret_cast<float*>(misc + M_SS) + (n % 3) * 256;
+            s_ss[(2 * half + cp) * 64 + 32 * (q - 2) + lane] = ss * p.scale * p.scale;
+            bar_sync(bar_out, 128);
+            if (oko && lw == 2 && lane == 0) mbar_arrive(bar_at(misc, M_NRM + 8 * (n & 1)));
+            ok = oko;
+        }
+        if (ok) {
             if (n + 1 < nchunks) {
                 ok = wait_warp(bar_at(misc, M_AFULL + 8 * ((n + 1) & 1)), (uint32_t)((n + 1) >> 1) & 1u, p);
                 if (ok) write_sm(n + 1);
@@ -1251,6 +1271,13 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         if (bar_sync_or(bar_half, 256, fail)) { stop = true; break; }
         trace_mark(0, n, 8 * half + 3, 256 * half);
         if (tid_h == 0) mbar_arrive(bar_at(misc, M_AFREE + 8 * b));
+        if (kN && lw == 2 && lane == 0) {
+            bulk_wait_read0();
+            uint64_t* zf = bar_at(misc, M_ZFULL + 8 * half);
+            mbar_arrive_expect_tx(zf, 8192u);
+            tma_load_3d(sb + ost_h, &p.tz, 64 * half, h, (int)(bos + (int64_t)n * kC), zf);
+            z_issued = n + 1;
+        }
         // (4) the next chunk's [X ; O], or a commit that covers O(n) after the last chunk
         if (issuer) {
             if (n + 1 < nchunks) {
@@ -1312,7 +1339,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
         if (is_consumer) {
             for (int b = 0; b < kBarsC; ++b) {
                 const uint32_t off = 8u * b;
-                const bool two = (off >= M_AFREE && off < M_VFULL) || (off >= M_NRM && off < M_ZFULL);
+                const bool two = (off >= M_AFREE && off < M_VFULL) || (off >= M_NRM && off < M_OD);
+                // (M_OD: one commit per chunk and half)
                 mbar_init(bar_at(misc, off), two ? 2 : 1);
             }
             const uint32_t id = smid();
@@ -1325,6 +1353,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
     }
     if (is_consumer && (MODE & kNorm) != 0)          // the output norm's weight
         for (int i = threadIdx.x; i < kD; i += kThreads) reinterpret_cast<float*>(misc + M_WN)[i] = p.w_norm[i];
+    if (!is_consumer && (MODE & kConv) != 0) {       // this head's conv weights, halved
+        for (int i = threadIdx.x; i < 3 * kD; i += kThreads) {
+            const int zz = i / kD, ch = i % kD;
+            const float4 w = reinterpret_cast<const float4*>(p.wconv[zz])[(size_t)h * kD + ch];
+            reinterpret_cast<float4*>(misc + M_WCV)[zz * kD + (ch % 8) * 16 + ch / 8] =
+                make_float4(0.5f * w.x, 0.5f * w.y, 0.5f * w.z, 0.5f * w.w);
+        }
+    }
     if (!is_consumer) {     // T' blocks above the diagonal are never written: zero them once
         for (int e = threadIdx.x; e < 8192 / 16; e += kThreads) st16(sm, P_TP + 16 * e, make_uint4(0, 0, 0, 0));
         fence_async_smem();
