@@ -61,6 +61,9 @@ def _declare(lib):
     lib.kda_oracle_gated_rmsnorm.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int,
                                              ctypes.c_double]
     lib.kda_oracle_gated_rmsnorm.restype = None
+    lib.kda_oracle_transition.argtypes = [_dp, _dp, _dp, _dp, _i64p, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int]
+    lib.kda_oracle_transition.restype = None
     return lib
 
 
@@ -114,6 +117,23 @@ def kda_fwd(q, k, v, g, beta, scale=1.0, h0=None, cu_seqlens=None, nthreads=None
     lib.kda_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(h0),
                        _ptr(ht), _ptr(o), cu.ctypes.data_as(_i64p), N, H, dk, dv, int(nthreads))
     return o, ht
+
+
+def transition(k, g, beta, cu_seqlens=None, nthreads=None, lib=None):
+    """Transition M of each (sequence, head): the product over its tokens, latest on the left,
+    of (I - beta k k^T) diag(exp(g)), so that the sequence started from S ends in
+    M S + (the state it ends in from zero). k, g: [T_tot, H, dk]; beta: [T_tot, H].
+    Returns m [N, H, dk, dk] (float64)."""
+    lib = lib or load()
+    k, g, beta = map(_f64, (k, g, beta))
+    T_tot, H, dk = k.shape
+    cu = _cu(cu_seqlens, T_tot)
+    N = cu.shape[0] - 1
+    m = np.zeros((N, H, dk, dk), dtype=np.float64)
+    nthreads = nthreads or os.cpu_count() or 1
+    lib.kda_oracle_transition(_ptr(k), _ptr(g), _ptr(beta), _ptr(m), cu.ctypes.data_as(_i64p), N,
+                              H, dk, int(nthreads))
+    return m
 
 
 def gdn_fwd(q, k, v, alpha, beta, scale=1.0, h0=None, cu_seqlens=None, nthreads=None, lib=None):

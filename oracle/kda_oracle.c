@@ -149,6 +149,62 @@ void kda_oracle_fwd(const double* q, const double* k, const double* v, const dou
 }
 
 /* ------------------------------------------------------------------------ */
+/* Transition of a stretch of tokens ([P1], [P4]). Each token maps the state */
+/* affinely: S -> (I - beta k k^T) diag(exp(g)) S + beta k v^T. Composing    */
+/* the maps of a stretch gives S_end = M S_start + (S_end started from 0),   */
+/* with M the product of the linear parts (I - beta k k^T) diag(exp(g)), the */
+/* latest token's on the left. This routine forms M by that product, one     */
+/* token at a time. A prefill split into stretches (context parallelism)     */
+/* joins them with it.                                                       */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const double *k, *g, *beta;
+    double* m;
+    const int64_t* cu;
+    int H, dk;
+} trans_ctx;
+
+static void trans_pair(void* vctx, int64_t pair) {
+    const trans_ctx* c = (const trans_ctx*)vctx;
+    const int H = c->H, dk = c->dk;
+    const int64_t n = pair / H;
+    const int h = (int)(pair % H);
+    double* M = (double*)calloc((size_t)dk * dk, sizeof(double));
+    double* w = (double*)malloc(sizeof(double) * (size_t)dk);
+    for (int i = 0; i < dk; ++i) M[(size_t)i * dk + i] = 1.0;
+    for (int64_t t = c->cu[n]; t < c->cu[n + 1]; ++t) {
+        const double* kt = c->k + ((size_t)t * H + h) * dk;
+        const double* gt = c->g + ((size_t)t * H + h) * dk;
+        const double bt = c->beta[(size_t)t * H + h];
+        /* left-multiply by diag(exp(g)): row r of M scales by exp(g_r) */
+        for (int r = 0; r < dk; ++r) {
+            const double decay = exp(gt[r]);
+            for (int col = 0; col < dk; ++col) M[(size_t)r * dk + col] *= decay;
+        }
+        /* left-multiply by (I - beta k k^T): M -= beta k (k^T M) */
+        for (int col = 0; col < dk; ++col) {
+            double acc = 0.0;
+            for (int r = 0; r < dk; ++r) acc += kt[r] * M[(size_t)r * dk + col];
+            w[col] = acc;
+        }
+        for (int r = 0; r < dk; ++r)
+            for (int col = 0; col < dk; ++col) M[(size_t)r * dk + col] -= bt * kt[r] * w[col];
+    }
+    memcpy(c->m + (size_t)pair * dk * dk, M, sizeof(double) * (size_t)dk * dk);
+    free(w);
+    free(M);
+}
+
+/* m : [N, H, dk, dk], the transition of every (sequence, head). */
+void kda_oracle_transition(const double* k, const double* g, const double* beta, double* m,
+                           const int64_t* cu_seqlens, int N, int H, int dk, int nthreads) {
+    trans_ctx c;
+    c.k = k; c.g = g; c.beta = beta; c.m = m; c.cu = cu_seqlens; c.H = H; c.dk = dk;
+    run_pairs(trans_pair, &c, (int64_t)N * H, nthreads);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Scalar-gated DeltaNet in Householder form, written independently of the   */
 /* KDA loop above: S <- exp(alpha) (I - beta k k^T) S + beta k v^T,          */
 /* o = scale S^T q. [P1] contrasts KDA's per-row gate with this scalar gate.  */

@@ -230,6 +230,41 @@ def pin_contraction(lib):
         S = Sn
 
 
+def pin_transition_affine(lib):
+    """A stretch started from S ends in M S + (its end state from zero): checked against the
+    recurrence itself from several starting states, over packed sequences of uneven length."""
+    q, k, v, g, beta, _ = random_inputs(12, 23, 2, 6, 5, strong=True, h0=False)
+    cu = np.array([0, 9, 9, 23])
+    rng = np.random.default_rng(13)
+    m = oracle.transition(k, g, beta, cu, lib=lib)
+    _, S_zero = oracle.kda_fwd(q, k, v, g, beta, 1.0, None, cu, lib=lib)
+    for _ in range(2):
+        S0 = rng.normal(0.0, 1.0, (3, 2, 6, 5))
+        _, S = oracle.kda_fwd(q, k, v, g, beta, 1.0, S0, cu, lib=lib)
+        _close(S, np.einsum("nhij,nhjc->nhic", m, S0) + S_zero, tol=1e-12, what="affine in h0")
+    _close(m[1], np.broadcast_to(np.eye(6), (2, 6, 6)), tol=0.0, what="empty sequence")
+
+
+def pin_transition_closed_forms(lib):
+    """beta = 0: M = diag(exp(sum_t g_t)). One token with g = 0: M = I - beta k k^T (M k =
+    (1 - beta |k|^2) k, M x = x for x orthogonal to k). det M = exp(sum g) prod (1 - beta_t |k_t|^2)
+    (the matrix determinant lemma). Two stretches compose as M(later) M(earlier)."""
+    _, k, _, g, beta, _ = random_inputs(14, 7, 1, 5, 5, h0=False)
+    m = oracle.transition(k, g, np.zeros_like(beta), lib=lib)
+    _close(m[0, 0], np.diag(np.exp(g[:, 0].sum(axis=0))), tol=1e-14, what="beta = 0")
+    kk = np.array([[[0.6, 0.0, -0.8, 0.0, 0.0]]])
+    m1 = oracle.transition(kk, np.zeros_like(kk), np.array([[0.3]]), lib=lib)[0, 0]
+    _close(m1 @ kk[0, 0], 0.7 * kk[0, 0], tol=1e-15, what="M k")
+    x = np.array([0.8, 0.1, 0.6, -2.0, 0.5])
+    _close(m1 @ x, x, tol=1e-15, what="M x, x orthogonal to k")
+    m = oracle.transition(k, g, beta, lib=lib)[0, 0]
+    det = np.exp(g[:, 0].sum()) * np.prod(1.0 - beta[:, 0] * np.sum(k[:, 0] ** 2, axis=-1))
+    _close(np.linalg.det(m), det, tol=1e-12, what="determinant")
+    ma = oracle.transition(k[:3], g[:3], beta[:3], lib=lib)[0, 0]
+    mb = oracle.transition(k[3:], g[3:], beta[3:], lib=lib)[0, 0]
+    _close(m, mb @ ma, tol=1e-13, what="composition order")
+
+
 # --------------------------------------------------------------------------- #
 # Conv prologue                                                                #
 # --------------------------------------------------------------------------- #
@@ -384,6 +419,7 @@ ALL_PINS = [
     pin_orthonormal_write_read, pin_same_key_last_value_wins, pin_beta_zero_pure_decay,
     pin_equal_gates_are_gated_deltanet, pin_T1_closed_form, pin_T2_closed_form, pin_linearity,
     pin_column_permutation, pin_varlen_equals_separate, pin_split_resume, pin_contraction,
+    pin_transition_affine, pin_transition_closed_forms,
     pin_conv_matches_torch, pin_conv_varlen_and_cache, pin_l2norm, pin_prologue_composition,
     pin_gate_closed_form, pin_gate_matches_torch, pin_sigmoid, pin_gated_rmsnorm,
 ]

@@ -80,6 +80,14 @@ MUTANTS = {
     "rmsnorm_sum_not_mean": ("const double inv = 1.0 / sqrt(ss / dv + eps);",
                              "const double inv = 1.0 / sqrt(ss + eps);"),
     "rmsnorm_weight_dropped": ("y[i] = o[i] * inv * w[j] * (1.0", "y[i] = o[i] * inv * (1.0"),
+    "transition_decay_on_columns": ("M[(size_t)r * dk + col] *= decay;",
+                                    "M[(size_t)r * dk + col] *= exp(gt[col]);"),
+    "transition_readout_transposed": ("acc += kt[r] * M[(size_t)r * dk + col];",
+                                      "acc += kt[r] * M[(size_t)col * dk + r];"),
+    "transition_beta_dropped": ("M[(size_t)r * dk + col] -= bt * kt[r] * w[col];",
+                                "M[(size_t)r * dk + col] -= kt[r] * w[col];"),
+    "transition_update_sign": ("M[(size_t)r * dk + col] -= bt * kt[r] * w[col];",
+                               "M[(size_t)r * dk + col] += bt * kt[r] * w[col];"),
     "rmsnorm_gate_silu": ("y[i] = o[i] * inv * w[j] * (1.0 / (1.0 + exp(-z[i])));",
                           "y[i] = o[i] * inv * w[j] * (z[i] / (1.0 + exp(-z[i])));"),
 }
