@@ -2,7 +2,8 @@
 """Benchmark of libkda's KDA hot path on B200; prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload prefill_8k|varlen_prologue|long_256k|decode_256x32] [--no-rows]
+                  [--workload prefill_8k|varlen_prologue|long_256k|long_256k_tp4|decode_256x32|conv_8k]
+                  [--no-rows]
 
 Headline (default workload prefill_8k: B=1, H=32, T=8192, dk=dv=128, bf16 I/O, fp32
 gates/beta/state, chunk 64): prefill tokens/s of kda_chunk_fwd with inputs resident in
@@ -51,6 +52,9 @@ WL_DESC = {
                   "zero h0,final state returned",
     "long_256k": "long_256k: B=1,H=32,T=262144,dk=dv=128,bf16 q/k/v/o,fp32 g/beta/state,chunk 64,"
                  "13/128 channels per head with exp(g)<0.5,final state returned",
+    "long_256k_tp4": "long_256k_tp4: B=1,H=8,T=262144,dk=dv=128,bf16 q/k/v/o,fp32 g/beta/state,"
+                     "chunk 64,13/128 channels per head with exp(g)<0.5,final state returned,"
+                     "split prefill",
 }
 
 
@@ -333,6 +337,17 @@ def run_ours(args):
             kda.chunk_fwd(q, k, v, d["g"], d["beta"], 1.0, h0=d["h0"], ht=ht, o=o,
                           cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], workspace=ws,
                           stream=stream)
+        if args.workload == "long_256k_tp4":
+            # too few (sequence, head) pairs to fill the GPU: the split prefill (stretch bounds,
+            # stretch states and transitions, the join, the stretches' outputs)
+            P, need = kda.chunk_fwd_split_plan(q, v, d["cu_seqlens"], d["cu_host"], 0)
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+            launches_per_step = 4 if P > 1 else 1
+
+            def step():
+                kda.chunk_fwd_split(q, k, v, d["g"], d["beta"], 1.0, h0=d["h0"], ht=ht, o=o,
+                                    cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], n_split=P,
+                                    workspace=ws, stream=stream)
         units = T_tot
         algo_bytes = prefill_bytes(T_tot, H, dk, dv, N, h0=d["h0"] is not None)
         wl_desc = dict(WL_DESC, varlen_prologue=f"varlen_prologue: 64 packed sequences "
@@ -507,6 +522,33 @@ def _gated_row(torch, kda, dev, flush, hbm_peak, stream, steps=5):
             "frac_hbm": algo / ms / 1e6 / hbm_peak}
 
 
+def _split_row(torch, kda, dev, flush, hbm_peak, stream, steps=3):
+    """long_256k_tp4 (8 heads of one of four tensor-parallel GPUs, 262144 tokens): the prefill
+    as one cluster per (sequence, head), and split into stretches that run side by side (the
+    count chosen by the library). Same algorithmic bytes for both."""
+    from kimi_delta_attention_32_b200.workloads import WORKLOADS, make_prefill
+    wl = WORKLOADS["long_256k_tp4"]
+    d = make_prefill(wl, dev)
+    T_tot, N, H, dk, dv = d["T_tot"], d["N"], d["H"], d["dk"], d["dv"]
+    o = torch.empty_like(d["v"])
+    ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    P, need = kda.chunk_fwd_split_plan(d["q"], d["v"], d["cu_seqlens"], d["cu_host"], 0)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def run(n_split):
+        return lambda: kda.chunk_fwd_split(d["q"], d["k"], d["v"], d["g"], d["beta"], 1.0, ht=ht,
+                                           o=o, cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"],
+                                           n_split=n_split, workspace=ws, stream=stream)
+    ms1 = statistics.mean(_events_time(torch, run(1), steps, 2, flush=flush, stream=stream))
+    msP = statistics.mean(_events_time(torch, run(P), steps, 2, flush=flush, stream=stream))
+    algo = prefill_bytes(T_tot, H, dk, dv, N, h0=False)
+    return {"workload": "long_256k_tp4: B=1,H=8,T=262144,dk=dv=128,bf16,skewed gates",
+            "stretches": P, "one_cluster_per_head_ms": ms1, "split_ms": msP,
+            "tokens/s": T_tot / msP * 1e3, "algorithmic_bytes": algo,
+            "frac_hbm": algo / msP / 1e6 / hbm_peak,
+            "one_cluster_per_head_frac_hbm": algo / ms1 / 1e6 / hbm_peak}
+
+
 def measure_rows(torch, kda, dev, flush, hbm_peak, stream):
     """Every other config of the path, measured in the same run: the conv prologue and the
     packed prefill with its prologue (64 sequences), the long-context prefill, and the decode
@@ -536,6 +578,8 @@ def measure_rows(torch, kda, dev, flush, hbm_peak, stream):
     out["long_256k"] = _prefill_row(torch, kda, dev, flush, hbm_peak, stream, "long_256k", steps=3)
     torch.cuda.empty_cache()
     out["prefill_8k_gated_norm"] = _gated_row(torch, kda, dev, flush, hbm_peak, stream)
+    torch.cuda.empty_cache()
+    out["long_256k_tp4_split"] = _split_row(torch, kda, dev, flush, hbm_peak, stream)
     torch.cuda.empty_cache()
 
     wl = WORKLOADS["decode_256x32"]
@@ -613,7 +657,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill_8k",
                     choices=["prefill_8k", "varlen_prologue", "long_256k", "decode_256x32",
-                             "conv_8k"])
+                             "conv_8k", "long_256k_tp4"])
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

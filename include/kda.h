@@ -146,6 +146,84 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          void* stream);
 
 /*
+ * kda_chunk_states -- the end states of a prefill, without its output, and optionally each
+ * sequence's transition: the pieces of a prefill split into stretches of tokens (context
+ * parallelism), joined by kda_state_scan.
+ * (sarnas.ru, section "Что именно изменилось", and m.lqnn.cn/news/205170, section "KDA 与
+ *  Gated Attention ...": the per-token update state = state*exp(gate) + delta is affine in the
+ *  state, S -> (I - beta k k^T) diag(exp(g)) S + beta k v^T; sarnas.ru, section "Как проходило
+ *  обучение": the model is trained at 8K, 32K and 256K contexts, which a split spreads over more
+ *  SMs or GPUs.)
+ *
+ * For each (sequence n, head h) of the batch:
+ *   ht[n,h] = the state after the sequence, started from h0[n,h] (zero when h0 is NULL),
+ *             as kda_chunk_fwd returns it;
+ *   m[n,h]  = the transition M = prod over the sequence's tokens, latest on the left, of
+ *             (I - beta_t k_t k_t^T) diag(exp(g_t))  (dk x dk, fp32, row i = key channel i),
+ *             so that started from any S the sequence would end in M S + (ht from zero).
+ * Either output may be NULL, not both. The transitions run in as many extra clusters as
+ * (sequence, head) pairs in the same launch. Inputs, layouts, workspace and errors as for
+ * kda_chunk_fwd (q is read though no output is formed).
+ *  m : [N, H, dk, dk] fp32 or NULL.   Supported: bf16 I/O, dk == dv == 128, chunk 64.
+ */
+kda_status kda_chunk_states(const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, const float* h0, float* ht, float* m,
+                            const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int B,
+                            int T, int N, int H, int dk, int dv, int chunk, kda_io_dtype io,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kda_state_scan -- joins the stretches of a split prefill in order (same sources as
+ * kda_chunk_states): for every sequence n and head h,
+ *     H_0 = h0[n,h] (zero when h0 is NULL),  H_{p+1} = M_p H_p + Z_p  for p = 0 .. P-1,
+ * with stretch p of sequence n at index j = n*seq_stride + p*seg_stride of m (M_j) and s_zero
+ * (Z_j, the stretch's end state from zero). h_start[j] receives H_p (the state entering
+ * stretch p) and ht[n] receives H_P; either may be NULL. fp32 throughout.
+ *  m : [*, H, dk, dk]   s_zero, h_start : [*, H, dk, dv]   h0, ht : [N, H, dk, dv]
+ *  (* = every index j reached). h_start must not overlap m, s_zero or h0.
+ *  Supported: dk, dv in {64, 128}.
+ */
+kda_status kda_state_scan(const float* m, const float* s_zero, const float* h0, float* h_start,
+                          float* ht, int N, int P, int H, int dk, int dv, int64_t seq_stride,
+                          int64_t seg_stride, void* stream);
+
+/*
+ * kda_chunk_fwd_split_workspace_size -- stretches per sequence and workspace bytes of
+ * kda_chunk_fwd_split for this batch (host-only, apart from reading the device's SM count when
+ * n_split == 0).
+ *  cu_seqlens_host, B, T, N: the batch as for kda_chunk_fwd (host data only).
+ *  n_split: stretches per sequence, or 0 to choose: the split is taken when the (sequence,
+ *  head) pairs leave most of the GPU's 4-SM clusters idle and the cost model (serial chunks
+ *  per stretch, waves of clusters) gains more than 10%; 1 otherwise.
+ *  n_split_out: host, receives the stretch count; bytes: host, receives the size.
+ */
+kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_host, int B, int T,
+                                              int N, int H, int dk, int dv, int chunk,
+                                              kda_io_dtype io, int n_split, int* n_split_out,
+                                              size_t* bytes);
+
+/*
+ * kda_chunk_fwd_split -- kda_chunk_fwd with every sequence split into stretches of whole
+ * chunks that run side by side (context parallelism inside one GPU; same sources as
+ * kda_chunk_states). Four launches on the stream: the stretch bounds; every stretch's end
+ * state from zero and transition (kda_chunk_states); the join (kda_state_scan); every
+ * stretch's output from the state entering it (kda_chunk_fwd over the stretches).
+ * Results equal kda_chunk_fwd's up to rounding: the entering states pass through the bf16
+ * products of the transitions.
+ *  n_split: as for kda_chunk_fwd_split_workspace_size (0 = choose; 1 = kda_chunk_fwd).
+ *  workspace: at least kda_chunk_fwd_split_workspace_size() bytes for the same batch and
+ *  n_split, 16-byte aligned.
+ * Other arguments, results and errors as for kda_chunk_fwd; also KDA_ERR_UNSUPPORTED when the
+ * batch has 2^31 tokens or more. Supported: bf16 I/O, dk == dv == 128, chunk 64.
+ */
+kda_status kda_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, float scale, const float* h0, float* ht,
+                               void* o, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                               int B, int T, int N, int H, int dk, int dv, int chunk,
+                               kda_io_dtype io, int n_split, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
  * kda_chunk_fwd_fused -- kda_chunk_fwd with the surrounding steps of the KDA layer fused into the
  * prefill kernel, each optional:
  *  - conv prologue (w_q, w_k, w_v given): q, k, v are the RAW projections; each is passed

@@ -45,6 +45,8 @@
 // Every wait is bounded (a launch parameter); a wait that gives up sets the error word, and the
 // CTA leaves its loop, waits for its own copies and products in flight, and frees its tensor
 // memory.
+#include <atomic>
+
 #include "common.cuh"
 #include "launchers.h"
 #include "tc.cuh"
@@ -70,6 +72,8 @@ constexpr float kHalfRange = 80.f;       // largest natural-log decay allowed pe
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr long long kDefaultWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
 constexpr int kGate = 1, kNorm = 2, kConv = 4;   // variant bits
+constexpr int kStates = 8;    // states-only launch: no output; the second half of the clusters
+                              // forms transitions
 constexpr int kHalo = 3;                 // kConv: the conv's three earlier tokens
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -180,7 +184,11 @@ struct Params {
     float scale;
     const float* h0;
     float* ht;
-    __nv_bfloat16* o;
+    __nv_bfloat16* o;                 // (unused by kStates launches)
+    // kStates: clusters units .. 2 units - 1 form each unit's transition instead (the state
+    // started from the identity, v taken as zero), written to mt [N,H,128,128] (or null: none)
+    float* mt;
+    int units;                        // N * H
     const int32_t* cu;
     uint8_t* ring;                    // workspace: ring_sms x kRing x kSlotBytes
     int ring_sms;
@@ -923,8 +931,10 @@ __device__ void producer(const Params& p, uint8_t* sm, uint32_t sb, int prank, i
 
 template <int MODE>
 __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, int h,
-                         int64_t bos, int64_t eos, bool aborted) {
+                         int64_t bos, int64_t eos, bool aborted, bool trans_unit) {
     constexpr bool kN = (MODE & kNorm) != 0;
+    constexpr bool kSt = (MODE & kStates) != 0;
+    const bool trans = kSt && trans_unit;
     constexpr bool kCv = (MODE & kConv) != 0;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* misc = sm + C_MISC;
@@ -963,8 +973,9 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 const int c0 = (int)(bos + (int64_t)m * kC);
                 const int rs = m % kRing;
                 const uint8_t* slot = ring + (size_t)rs * kSlotBytes;
-                // V tiles: by TMA from v, or (kConv) the conv's output from the ring slot
-                if constexpr (!kCv) {
+                // V tiles: by TMA from v, or (kConv) the conv's output from the ring slot; none
+                // for a transition (v is taken as zero)
+                if (!kCv && !trans) {
                     for (int hh = 0; hh < 2; ++hh) {
                         uint64_t* vf = bar_at(misc, M_VFULL + 8 * (2 * hh + sl));
                         if (m >= 2 && !(ok = wait_one(bar_at(misc, M_VFREE + 8 * (2 * hh + sl)), pfree, p))) break;
@@ -1036,7 +1047,12 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
 #pragma unroll
     for (int c4 = 0; c4 < 8; ++c4) {
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (p.h0) v = reinterpret_cast<const float4*>(p.h0 + sbase + (int64_t)i_row * kD + jg0)[c4];
+        if (trans) {                             // the identity
+            const int d = i_row - (jg0 + 4 * c4);
+            v = make_float4(d == 0, d == 1, d == 2, d == 3);
+        } else if (p.h0) {
+            v = reinterpret_cast<const float4*>(p.h0 + sbase + (int64_t)i_row * kD + jg0)[c4];
+        }
         S[4 * c4] = v.x; S[4 * c4 + 1] = v.y; S[4 * c4 + 2] = v.z; S[4 * c4 + 3] = v.w;
     }
     auto fac = [&](int nn) {
@@ -1166,7 +1182,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         tc_fence_after();
         if (ok && n > 0 && tid_h == 0) mbar_arrive(bar_at(misc, M_BFREE + 8 * ((n - 1) & 1)));
         if (q < 2) {
-            if (ok) ok = wait_warp(bar_at(misc, M_VFULL + 8 * (2 * half + b)), (uint32_t)(n >> 1) & 1u, p);
+            if (ok && !trans) ok = wait_warp(bar_at(misc, M_VFULL + 8 * (2 * half + b)), (uint32_t)(n >> 1) & 1u, p);
             if (ok) {
                 const int t = 32 * q + lane;
                 const uint8_t* vt = sm + C_V + (uint32_t)(2 * half + b) * 8192;
@@ -1177,8 +1193,8 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
                         const int ck = 4 * cp + 2 * hx + k2;
-                        float vv[8];
-                        unpack8(ld16(vt, t * 128 + ((ck ^ (t & 7)) << 4)), vv);
+                        float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (!trans) unpack8(ld16(vt, t * 128 + ((ck ^ (t & 7)) << 4)), vv);
 #pragma unroll
                         for (int u = 0; u < 8; ++u) vv[u] -= xv[8 * k2 + u];
                         st16(sm, u_h + sw128(t, ck, 0, 0), pack8(vv));
@@ -1195,7 +1211,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         // the output of chunk n - 1, by the output warps, while the delta product runs (this
         // keeps it off the path from X(n) to the delta)
         trace_mark(0, n, 8 * half + 4, 256 * half + 64);
-        if (q >= 2 && n > 0) epilogue_o(n - 1, ok);
+        if (!kSt && q >= 2 && n > 0) epilogue_o(n - 1, ok);
         trace_mark(0, n, 8 * half + 6, 256 * half + 64);
         // (2) state delta Yh^T U (commit), then O(n) += Wh^T U
         if (issuer) {
@@ -1294,11 +1310,12 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         const bool ok = wait_warp(bar_xo, (uint32_t)(nchunks & 1), p);
         if (issuer && ok) ++xo_waited;
         tc_fence_after();
-        if (q >= 2) epilogue_o(nchunks - 1, ok);
+        if (!kSt && q >= 2) epilogue_o(nchunks - 1, ok);
         stop = bar_sync_or(bar_half, 256, !ok) != 0;
     }
-    if (!stop && p.ht) {
-        float4* dst = reinterpret_cast<float4*>(p.ht + sbase + (int64_t)i_row * kD + jg0);
+    float* const hdst = trans ? p.mt : p.ht;
+    if (!stop && hdst != nullptr) {
+        float4* dst = reinterpret_cast<float4*>(hdst + sbase + (int64_t)i_row * kD + jg0);
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) dst[c4] = make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
     }
@@ -1326,7 +1343,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
 
     int n_seq, h;
     int64_t bos, eos;
-    unit_of(p, (int)(blockIdx.x / kCluster), reinterpret_cast<int*>(misc + M_TMP), n_seq, h, bos, eos);
+    const int cid = (int)(blockIdx.x / kCluster);
+    const bool trans = (MODE & kStates) != 0 && cid >= p.units;
+    unit_of(p, trans ? cid - p.units : cid, reinterpret_cast<int*>(misc + M_TMP), n_seq, h, bos, eos);
 
     const uint32_t ncols = is_consumer ? kTmemC : kTmemP;
     if (warp == 0) {
@@ -1371,7 +1390,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
 
     // a consumer SM outside the workspace's ring table (flagged above): nobody touches the ring
     const bool aborted = (int)ld_cluster_u32(map_to_rank(sb + C_MISC + M_SMID, 0)) >= p.ring_sms;
-    if (is_consumer) consumer<MODE>(p, sm, sb, n_seq, h, bos, eos, aborted);
+    if (is_consumer) consumer<MODE>(p, sm, sb, n_seq, h, bos, eos, aborted, trans);
     else producer<MODE>(p, sm, sb, (int)crank, n_seq, h, bos, eos, aborted);
 
     tc_fence_before();
@@ -1387,17 +1406,48 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
 
 size_t chunk_tcx_workspace_bytes() { return kTcxWorkspaceBytes; }
 
+int chunk_tcx_cluster_slots() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    static std::atomic<int> cached[64];
+    if (dev < 64) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    const auto kernel = chunk_tcx_kernel<0>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
+        cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kCluster * 64, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) return 0;
+    if (dev < 64 && n > 0) cached[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspace_bytes,
                              unsigned int* err, cudaStream_t stream) {
     const int64_t units = (int64_t)a.N * a.H;
     if (units == 0) return cudaSuccess;
     const int mode = (a.g_raw != nullptr ? kGate : 0) | (a.z != nullptr ? kNorm : 0) |
                      (a.wconv[0] != nullptr ? kConv : 0);
+    const bool states = (a.o == nullptr);
+    if (states && mode != 0) return cudaErrorInvalidValue;    // states-only: the plain inputs
     using KernelFn = void (*)(Params);
     static const KernelFn kernels[8] = {
         chunk_tcx_kernel<0>, chunk_tcx_kernel<1>, chunk_tcx_kernel<2>, chunk_tcx_kernel<3>,
         chunk_tcx_kernel<4>, chunk_tcx_kernel<5>, chunk_tcx_kernel<6>, chunk_tcx_kernel<7>};
-    const KernelFn kernel = kernels[mode];
+    const KernelFn kernel = states ? chunk_tcx_kernel<kStates> : kernels[mode];
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -1412,7 +1462,7 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
               : make_tmap_thd(&p.tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.T_tot, a.H, kD, kD, kC, false)) &&
         (conv ? make_tmap_thd(&p.tv, a.v, BF, 2, a.T_tot, a.H, kD, kD, tile_rows, false)
               : make_tmap_thd(&p.tv, a.v, BF, 2, a.T_tot, a.H, kD, 64, kC, true)) &&
-        make_tmap_thd(&p.to, a.o, BF, 2, a.T_tot, a.H, kD, 64, kC, true) &&
+        (a.o == nullptr || make_tmap_thd(&p.to, a.o, BF, 2, a.T_tot, a.H, kD, 64, kC, true)) &&
         (a.z == nullptr || make_tmap_thd(&p.tz, a.z, BF, 2, a.T_tot, a.H, kD, 64, kC, true));
     if (!maps_ok) return cudaErrorInvalidValue;
     p.q = static_cast<const __nv_bfloat16*>(a.q);
@@ -1423,6 +1473,8 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
     p.h0 = a.h0;
     p.ht = a.ht;
     p.o = static_cast<__nv_bfloat16*>(a.o);
+    p.mt = a.mt;
+    p.units = (int)units;
     p.cu = a.cu;
     p.T_pad = a.T_pad;
     p.N = a.N;
@@ -1442,7 +1494,7 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
     p.conv_state = static_cast<const __nv_bfloat16*>(a.conv_state);
     p.l2_eps = a.l2_eps;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(units * kCluster), 1, 1);
+    cfg.gridDim = dim3((unsigned)(units * (states && a.mt != nullptr ? 2 : 1) * kCluster), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;

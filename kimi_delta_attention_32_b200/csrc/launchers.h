@@ -80,6 +80,9 @@ struct ChunkArgs {
     const float* wconv[3] = {nullptr, nullptr, nullptr};
     const void* conv_state = nullptr;
     float l2_eps = 0.f;
+    // tensor-core path only: a states-only launch (o null) may also form each unit's transition
+    // into mt [N, H, dk, dk] fp32 (mt non-null), in as many extra clusters as units
+    float* mt = nullptr;
 };
 cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 
@@ -97,9 +100,29 @@ inline bool chunk_tc_supported(const ChunkArgs& a) {
     return a.io == Io::BF16 && a.dk == 128 && a.dv == 128 && a.chunk == 64;
 }
 size_t chunk_tcx_workspace_bytes();
+// Clusters of the prefill kernel that can be resident at once on the current device (0 if the
+// query fails); cached per device.
+int chunk_tcx_cluster_slots();
 // Bound (SM cycles) of every device-side wait of later prefill launches; 0 restores the default.
 extern long long g_chunk_wait_cycles;
 cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspace_bytes,
                              unsigned int* err, cudaStream_t stream);
+
+// Splits every sequence of a batch into P stretches of whole chunks (the last one ragged):
+// stretch p of sequence n is stretch index n * P + p, and seg_cu [N * P + 1] receives their
+// bounds in packed form. cu: device cu_seqlens, or null for a padded batch of N x T_pad tokens.
+cudaError_t launch_split_stretches(const int32_t* cu, int T_pad, int N, int P, int32_t* seg_cu,
+                                   cudaStream_t stream);
+
+struct ScanArgs {
+    const float* m;          // [*, H, dk, dk] stretch transitions
+    const float* s_zero;     // [*, H, dk, dv] stretch end states from zero
+    const float* h0;         // [N, H, dk, dv] or null (zero)
+    float* h_start;          // [*, H, dk, dv] the state entering each stretch, or null
+    float* ht;               // [N, H, dk, dv] the state after each sequence's last stretch, or null
+    int N, P, H, dk, dv;
+    int64_t seq_stride, seg_stride;   // stretch p of sequence n is index n * seq_stride + p * seg_stride
+};
+cudaError_t launch_state_scan(const ScanArgs& a, cudaStream_t stream);
 
 }  // namespace kda

@@ -23,7 +23,8 @@ KDA_IO_F32, KDA_IO_BF16 = 0, 1
 EXPORTED = ("kda_status_string", "kda_version", "kda_conv_fwd", "kda_chunk_fwd_workspace_size",
             "kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_fwd_noalloc", "kda_recurrent_step",
             "kda_conv_recurrent_step", "kda_fused_recurrent_step", "kda_set_wait_limit",
-            "kda_last_device_error")
+            "kda_last_device_error", "kda_chunk_states", "kda_state_scan",
+            "kda_chunk_fwd_split_workspace_size", "kda_chunk_fwd_split")
 
 _lock = threading.Lock()
 _lib = None
@@ -83,6 +84,19 @@ def load_library(path: str = LIB_PATH):
         lib.kda_set_wait_limit.restype = ci
         lib.kda_last_device_error.argtypes = [vp]
         lib.kda_last_device_error.restype = ci
+        cip = ctypes.POINTER(ctypes.c_int32)
+        lib.kda_chunk_states.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, i32p, cip, ci, ci, ci, ci,
+                                         ci, ci, ci, ci, vp, cs, vp]
+        lib.kda_chunk_states.restype = ci
+        lib.kda_state_scan.argtypes = [fp, fp, fp, fp, fp, ci, ci, ci, ci, ci, ctypes.c_int64,
+                                       ctypes.c_int64, vp]
+        lib.kda_state_scan.restype = ci
+        lib.kda_chunk_fwd_split_workspace_size.argtypes = [cip, ci, ci, ci, ci, ci, ci, ci, ci, ci,
+                                                           ctypes.POINTER(ci), ctypes.POINTER(cs)]
+        lib.kda_chunk_fwd_split_workspace_size.restype = ci
+        lib.kda_chunk_fwd_split.argtypes = [vp, vp, vp, fp, fp, cf, fp, fp, vp, i32p, cip, ci, ci,
+                                            ci, ci, ci, ci, ci, ci, ci, vp, cs, vp]
+        lib.kda_chunk_fwd_split.restype = ci
         if path == LIB_PATH:
             _lib = lib
         return lib
@@ -180,6 +194,89 @@ def chunk_fwd(q, k, v, g, beta, scale=1.0, h0=None, ht=None, o=None, cu_seqlens=
                            _stream(stream))
     del keep
     _check("kda_chunk_fwd", st)
+    return o, ht
+
+
+def _batch(q, cu_seqlens, cu_host):
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape if q.dim() == 4 else (1, *q.shape)
+        return B, T, B, B * T, H, dk
+    T_tot, H, dk = q.shape
+    return 1, 0, len(cu_host) - 1, T_tot, H, dk
+
+
+def chunk_states(q, k, v, g, beta, h0=None, cu_seqlens=None, cu_host=None, chunk=64,
+                 end_state=True, transition=True, workspace=None, stream=None):
+    """End states (started from h0, or zero) and transitions of every (sequence, head), without
+    the output. Returns (ht [N,H,dk,dv] or None, m [N,H,dk,dk] or None), both fp32."""
+    lib = load_library()
+    B, T, N, T_tot, H, dk = _batch(q, cu_seqlens, cu_host)
+    dv = v.shape[-1]
+    ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device) if end_state else None
+    m = torch.empty((N, H, dk, dk), dtype=torch.float32, device=q.device) if transition else None
+    io = _io(q)
+    if workspace is None:
+        need = chunk_fwd_workspace_size(N, T_tot, H, dk, dv, chunk, io)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    keep, cuh = _host_cu(cu_host)
+    st = lib.kda_chunk_states(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(ht),
+                              _ptr(m), _ptr(cu_seqlens), cuh, B, T, N, H, dk, dv, chunk, io,
+                              _ptr(workspace), workspace.numel(), _stream(stream))
+    del keep
+    _check("kda_chunk_states", st)
+    return ht, m
+
+
+def state_scan(m, s_zero, h0=None, *, N, P, seq_stride, seg_stride, h_start=None, ht=None,
+               stream=None):
+    """Joins stretches: H_0 = h0, H_{p+1} = M_p H_p + Z_p, stretch p of sequence n at index
+    n * seq_stride + p * seg_stride of m [*,H,dk,dk] and s_zero [*,H,dk,dv].
+    Returns (h_start [*,H,dk,dv], ht [N,H,dk,dv])."""
+    lib = load_library()
+    H, dk, dv = s_zero.shape[1], s_zero.shape[2], s_zero.shape[3]
+    if h_start is None:
+        h_start = torch.empty_like(s_zero)
+    if ht is None:
+        ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=s_zero.device)
+    _check("kda_state_scan", lib.kda_state_scan(_ptr(m), _ptr(s_zero), _ptr(h0), _ptr(h_start),
+                                                _ptr(ht), N, P, H, dk, dv, seq_stride, seg_stride,
+                                                _stream(stream)))
+    return h_start, ht
+
+
+def chunk_fwd_split_plan(q, v, cu_seqlens=None, cu_host=None, n_split=0, chunk=64):
+    """(stretches per sequence, workspace bytes) of chunk_fwd_split for this batch."""
+    lib = load_library()
+    B, T, N, _, H, dk = _batch(q, cu_seqlens, cu_host)
+    keep, cuh = _host_cu(cu_host)
+    P, nbytes = ctypes.c_int(0), ctypes.c_size_t(0)
+    st = lib.kda_chunk_fwd_split_workspace_size(cuh, B, T, N, H, dk, v.shape[-1], chunk, _io(q),
+                                                n_split, ctypes.byref(P), ctypes.byref(nbytes))
+    del keep
+    _check("kda_chunk_fwd_split_workspace_size", st)
+    return P.value, nbytes.value
+
+
+def chunk_fwd_split(q, k, v, g, beta, scale=1.0, h0=None, ht=None, o=None, cu_seqlens=None,
+                    cu_host=None, n_split=0, chunk=64, workspace=None, stream=None):
+    """chunk_fwd with every sequence split into stretches that run side by side (n_split = 0:
+    chosen for the batch). Returns (o, ht)."""
+    lib = load_library()
+    B, T, N, _, H, dk = _batch(q, cu_seqlens, cu_host)
+    dv = v.shape[-1]
+    o = torch.empty_like(v) if o is None else o
+    if ht is None:
+        ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        _, need = chunk_fwd_split_plan(q, v, cu_seqlens, cu_host, n_split, chunk)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    keep, cuh = _host_cu(cu_host)
+    st = lib.kda_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                 _ptr(h0), _ptr(ht), _ptr(o), _ptr(cu_seqlens), cuh, B, T, N, H,
+                                 dk, dv, chunk, _io(q), n_split, _ptr(workspace), workspace.numel(),
+                                 _stream(stream))
+    del keep
+    _check("kda_chunk_fwd_split", st)
     return o, ht
 
 

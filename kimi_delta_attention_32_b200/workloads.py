@@ -66,6 +66,13 @@ WORKLOADS = {
     "long_256k": Workload("long_256k", N=1, H=32, T=262144, dk=128, dv=128, io="bf16",
                           skew_channels=13, seed=1004,
                           notes="B=1,H=32,T=262144, 13/128 channels per head with exp(g)<0.5"),
+    # one of four tensor-parallel GPUs (the 4-GPU serving set-up of the model card) holds 8 of
+    # the 32 heads: too few (sequence, head) pairs to fill the GPU, the case the split prefill
+    # serves
+    "long_256k_tp4": Workload("long_256k_tp4", N=1, H=8, T=262144, dk=128, dv=128, io="bf16",
+                              skew_channels=13, seed=1005,
+                              notes="B=1,H=8,T=262144 (32 heads over 4 tensor-parallel GPUs), "
+                                    "13/128 channels per head with exp(g)<0.5"),
 }
 
 

@@ -233,3 +233,89 @@ def test_fused_prefill_checks_arguments(lib):
     assert _fused(lib, io=0) == kda.KDA_ERR_UNSUPPORTED               # tensor-core path only
     assert _fused(lib, dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
     assert _fused(lib, ws=None) == kda.KDA_ERR_WORKSPACE
+
+
+def test_split_workspace_query(lib):
+    P, out = ctypes.c_int(0), ctypes.c_size_t(0)
+    ring = ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_workspace_size(1, 8192, 4, 128, 128, 64, 1, ctypes.byref(ring)) == 0
+    sizes = []
+    for n_split in (1, 2, 8):
+        assert lib.kda_chunk_fwd_split_workspace_size(None, 1, 8192, 0, 4, 128, 128, 64, 1, n_split,
+                                                      ctypes.byref(P), ctypes.byref(out)) == 0
+        assert P.value == n_split
+        sizes.append(out.value)
+    assert sizes[0] == ring.value                       # one stretch: kda_chunk_fwd's rings
+    # rings + stretch bounds + (transition, end state, entering state) per stretch and head
+    per = 4 * 128 * 128 * 3
+    assert sizes[1] >= ring.value + 2 * 4 * per and sizes[2] >= ring.value + 8 * 4 * per
+    assert sizes[2] - sizes[1] < 6 * 4 * per + 1024
+    keep, cuh = _cu_host([0, 100, 100, 5000])
+    assert lib.kda_chunk_fwd_split_workspace_size(cuh, 0, 0, 3, 4, 128, 128, 64, 1, 3,
+                                                  ctypes.byref(P), ctypes.byref(out)) == 0
+    assert P.value == 3 and out.value >= ring.value + 9 * 4 * per
+    bad = _cu_host([0, 100, 50])
+    assert lib.kda_chunk_fwd_split_workspace_size(bad[1], 0, 0, 2, 4, 128, 128, 64, 1, 2,
+                                                  ctypes.byref(P), ctypes.byref(out)) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_split_workspace_size(None, 1, 8192, 0, 4, 128, 128, 64, 1, -1,
+                                                  ctypes.byref(P), ctypes.byref(out)) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_split_workspace_size(None, 1, 8192, 0, 4, 128, 128, 64, 0, 2,
+                                                  ctypes.byref(P), ctypes.byref(out)) == \
+        kda.KDA_ERR_UNSUPPORTED                          # fp32 I/O has no split path
+    assert lib.kda_chunk_fwd_split_workspace_size(None, 1, 8192, 0, 4, 128, 128, 64, 1, 2, None,
+                                                  ctypes.byref(out)) == kda.KDA_ERR_INVALID_ARG
+    del keep
+
+
+def _states(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, h0=None, ht=FAKE, m=FAKE, cu=None,
+             cuh=None, B=1, T=64, N=1, H=2, dk=128, dv=128, chunk=64, io=1, ws=FAKE,
+             wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.kda_chunk_states(a["q"], a["k"], a["v"], a["g"], a["beta"], a["h0"], a["ht"], a["m"],
+                                a["cu"], a["cuh"], a["B"], a["T"], a["N"], a["H"], a["dk"], a["dv"],
+                                a["chunk"], a["io"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_chunk_states_checks_arguments(lib):
+    assert _states(lib, ht=None, m=None) == kda.KDA_ERR_INVALID_ARG     # nothing to form
+    assert _states(lib, q=None) == kda.KDA_ERR_INVALID_ARG
+    assert _states(lib, m=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert _states(lib, beta=None) == kda.KDA_ERR_INVALID_ARG
+    assert _states(lib, io=0) == kda.KDA_ERR_UNSUPPORTED                 # tensor-core path only
+    assert _states(lib, dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
+    assert _states(lib, ws=None) == kda.KDA_ERR_WORKSPACE
+    assert _states(lib, wsb=16) == kda.KDA_ERR_WORKSPACE
+
+
+def test_state_scan_checks_arguments(lib):
+    def scan(**kw):
+        a = dict(m=FAKE, z=FAKE, h0=None, hs=FAKE, ht=None, N=2, P=3, H=2, dk=128, dv=128, sn=3,
+                 sp=1)
+        a.update(kw)
+        return lib.kda_state_scan(a["m"], a["z"], a["h0"], a["hs"], a["ht"], a["N"], a["P"], a["H"],
+                                  a["dk"], a["dv"], a["sn"], a["sp"], None)
+    assert scan(P=0) == kda.KDA_ERR_INVALID_ARG
+    assert scan(m=None) == kda.KDA_ERR_INVALID_ARG
+    assert scan(z=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert scan(sn=-1) == kda.KDA_ERR_INVALID_ARG
+    assert scan(H=0) == kda.KDA_ERR_INVALID_ARG
+    assert scan(dk=96) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_chunk_fwd_split_checks_arguments(lib):
+    def split(**kw):
+        a = dict(o=FAKE, q=FAKE, n=2, io=1, ws=FAKE, wsb=16, chunk=64)
+        a.update(kw)
+        return lib.kda_chunk_fwd_split(a["q"], FAKE, FAKE, FAKE, FAKE, 1.0, None, None, a["o"], None,
+                                       None, 1, 8192, 0, 4, 128, 128, a["chunk"], a["io"], a["n"],
+                                       a["ws"], a["wsb"], None)
+    assert split(o=None) == kda.KDA_ERR_INVALID_ARG
+    assert split(q=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert split(n=-2) == kda.KDA_ERR_INVALID_ARG
+    assert split(io=0) == kda.KDA_ERR_UNSUPPORTED
+    assert split(chunk=32) == kda.KDA_ERR_UNSUPPORTED
+    assert split() == kda.KDA_ERR_WORKSPACE                            # 16 bytes is too small
+    assert split(ws=None, wsb=1 << 40) == kda.KDA_ERR_WORKSPACE
