@@ -146,31 +146,35 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          void* stream);
 
 /*
- * kda_chunk_states -- the end states of a prefill, without its output, and optionally each
- * sequence's transition: the pieces of a prefill split into stretches of tokens (context
- * parallelism), joined by kda_state_scan.
+ * kda_chunk_states -- a prefill's pieces for a split into stretches of tokens (context
+ * parallelism), joined by kda_state_scan: per sequence its end state, output and transition,
+ * and the queries carried back to its start.
  * (sarnas.ru, section "Что именно изменилось", and m.lqnn.cn/news/205170, section "KDA 与
  *  Gated Attention ...": the per-token update state = state*exp(gate) + delta is affine in the
  *  state, S -> (I - beta k k^T) diag(exp(g)) S + beta k v^T; sarnas.ru, section "Как проходило
  *  обучение": the model is trained at 8K, 32K and 256K contexts, which a split spreads over more
  *  SMs or GPUs.)
  *
- * For each (sequence n, head h) of the batch:
- *   ht[n,h] = the state after the sequence, started from h0[n,h] (zero when h0 is NULL),
- *             as kda_chunk_fwd returns it;
- *   m[n,h]  = the transition M = prod over the sequence's tokens, latest on the left, of
- *             (I - beta_t k_t k_t^T) diag(exp(g_t))  (dk x dk, fp32, row i = key channel i),
- *             so that started from any S the sequence would end in M S + (ht from zero).
- * Either output may be NULL, not both. The transitions run in as many extra clusters as
- * (sequence, head) pairs in the same launch. Inputs, layouts, workspace and errors as for
- * kda_chunk_fwd (q is read though no output is formed).
- *  m : [N, H, dk, dk] fp32 or NULL.   Supported: bf16 I/O, dk == dv == 128, chunk 64.
+ * For each (sequence n, head h) of the batch, with M_t the product over the sequence's tokens
+ * up to t, latest on the left, of (I - beta k k^T) diag(exp(g)) (dk x dk):
+ *   ht[n,h] = the state after the sequence, started from h0[n,h] (zero when h0 is NULL), as
+ *             kda_chunk_fwd returns it;
+ *   o       = the output from that start, as kda_chunk_fwd returns it;
+ *   m[n,h]  = the transition M = M_T of the whole sequence (fp32, row i = key channel i), so
+ *             that started from any S the sequence ends in M S + (ht from zero);
+ *   w[t,h]  = scale * M_t^T q_t, so that started from any S the output is
+ *             o_t(from zero) + S^T w_t.
+ * Each output may be NULL, not all. m and w come from as many extra clusters as (sequence,
+ * head) pairs in the same launch. Inputs, layouts, workspace and errors as for kda_chunk_fwd.
+ *  o : [T_tot, H, dv] bf16 or NULL   m : [N, H, dk, dk] fp32 or NULL   w : [T_tot, H, dk] bf16
+ *  or NULL.   Supported: bf16 I/O, dk == dv == 128, chunk 64.
  */
 kda_status kda_chunk_states(const void* q, const void* k, const void* v, const float* g,
-                            const float* beta, const float* h0, float* ht, float* m,
-                            const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int B,
-                            int T, int N, int H, int dk, int dv, int chunk, kda_io_dtype io,
-                            void* workspace, size_t workspace_bytes, void* stream);
+                            const float* beta, float scale, const float* h0, float* ht, void* o,
+                            float* m, void* w, const int32_t* cu_seqlens,
+                            const int32_t* cu_seqlens_host, int B, int T, int N, int H, int dk,
+                            int dv, int chunk, kda_io_dtype io, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 /*
  * kda_state_scan -- joins the stretches of a split prefill in order (same sources as
@@ -186,6 +190,22 @@ kda_status kda_chunk_states(const void* q, const void* k, const void* v, const f
 kda_status kda_state_scan(const float* m, const float* s_zero, const float* h0, float* h_start,
                           float* ht, int N, int P, int H, int dk, int dv, int64_t seq_stride,
                           int64_t seg_stride, void* stream);
+
+/*
+ * kda_output_correct -- adds the entering state's share to outputs formed from a zero state
+ * (same sources as kda_chunk_states): for every sequence n, head h and token t of it,
+ *     o[t,h,:] += h[n,h]^T w[t,h,:]
+ * with w from kda_chunk_states and h[n,h] the state the sequence was entered with (from
+ * kda_state_scan). The product runs on the tensor cores in bf16 with fp32 accumulation; h is
+ * split into two bf16 halves, which keep 16 of its mantissa bits (relative error below 2^-16
+ * per product).
+ *  w : [T_tot, H, dk] bf16   h : [N, H, dk, dv] fp32   o : [T_tot, H, dv] bf16, updated in place.
+ *  Packed batches only (cu_seqlens and cu_seqlens_host given; KDA_ERR_UNSUPPORTED otherwise).
+ *  Supported: bf16 I/O, dk == dv == 128.
+ */
+kda_status kda_output_correct(const void* w, const float* h, void* o, const int32_t* cu_seqlens,
+                              const int32_t* cu_seqlens_host, int B, int T, int N, int H, int dk,
+                              int dv, kda_io_dtype io, void* stream);
 
 /*
  * kda_chunk_fwd_split_workspace_size -- stretches per sequence and workspace bytes of
@@ -205,11 +225,13 @@ kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_host, in
 /*
  * kda_chunk_fwd_split -- kda_chunk_fwd with every sequence split into stretches of whole
  * chunks that run side by side (context parallelism inside one GPU; same sources as
- * kda_chunk_states). Four launches on the stream: the stretch bounds; every stretch's end
- * state from zero and transition (kda_chunk_states); the join (kda_state_scan); every
- * stretch's output from the state entering it (kda_chunk_fwd over the stretches).
- * Results equal kda_chunk_fwd's up to rounding: the entering states pass through the bf16
- * products of the transitions.
+ * kda_chunk_states). Four launches on the stream: the stretch bounds; every stretch from a
+ * zero state, with its output, end state, transition and carried-back queries
+ * (kda_chunk_states); the join (kda_state_scan), which gives each stretch's entering state H;
+ * and the correction o_t += H^T w_t of every stretch's output (a dense product on the tensor
+ * cores). Results equal kda_chunk_fwd's up to rounding: the entering states pass through the
+ * bf16 products of the transitions, and the output from zero and w are rounded to bf16 before
+ * the correction.
  *  n_split: as for kda_chunk_fwd_split_workspace_size (0 = choose; 1 = kda_chunk_fwd).
  *  workspace: at least kda_chunk_fwd_split_workspace_size() bytes for the same batch and
  *  n_split, 16-byte aligned.

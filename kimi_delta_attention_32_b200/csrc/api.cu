@@ -60,9 +60,9 @@ unsigned int* device_error_word() {
 
 // A prefill split into P stretches per sequence: the layout of its workspace after the rings.
 struct SplitLayout {
-    size_t seg_cu, m, z, hs, total;
+    size_t seg_cu, m, z, hs, w, total;
 };
-SplitLayout split_layout(int N, int P, int H, int dk, int dv) {
+SplitLayout split_layout(int N, int64_t T_tot, int P, int H, int dk, int dv) {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
     const size_t stretches = (size_t)N * P * H;
     SplitLayout l;
@@ -70,26 +70,29 @@ SplitLayout split_layout(int N, int P, int H, int dk, int dv) {
     l.m = l.seg_cu + up(sizeof(int32_t) * ((size_t)N * P + 1));
     l.z = l.m + up(sizeof(float) * stretches * dk * dk);
     l.hs = l.z + up(sizeof(float) * stretches * dk * dv);
-    l.total = l.hs + up(sizeof(float) * stretches * dk * dv);
+    l.w = l.hs + up(sizeof(float) * stretches * dk * dv);
+    l.total = l.w + up(sizeof(uint16_t) * (size_t)T_tot * H * dk);
     return l;
 }
 
 // Stretches per sequence for a split prefill. The per-head recurrence is serial over chunks,
 // and one cluster of 4 SMs carries one (stretch, head) at a time; `clusters` of them fit on the
 // GPU at once (33 on a B200: clusters are placed within GPCs). The split runs 2 U P units
-// (end states and transitions) over stretches P times shorter, then U P units again for the
-// outputs; it pays when U = N H units leave most clusters idle. Cost in chunk steps, one per
-// stretch for the join; the split is taken only for a gain above 10%.
-int auto_split(int64_t longest, int64_t units, int clusters) {
+// (outputs and end states from zero, and the transitions) over stretches P times shorter; it
+// pays when U = N H units leave most clusters idle. Cost in chunk steps (~2 us each): one per
+// stretch for the join, and the output correction, an HBM-bound pass of 768 bytes per token and
+// head (~1/16384 of a step). The split is taken only for a gain above 10%.
+int auto_split(int64_t longest, int64_t T_tot, int H, int64_t units, int clusters) {
     if (units <= 0 || longest <= 0 || clusters <= 0) return 1;
     const int64_t chunks = (longest + 63) / 64;
     auto waves = [&](int64_t u) { return (u + clusters - 1) / clusters; };
+    const int64_t correct = T_tot * H / 16384 + 1;
     int best_p = 1;
     int64_t best = waves(units) * chunks;
     for (int P = 2; P <= 64; ++P) {
         const int64_t per = (chunks + P - 1) / P;
         if (per < 2) break;
-        const int64_t cost = (waves(2 * units * P) + waves(units * P)) * per + P;
+        const int64_t cost = waves(2 * units * P) * per + P + correct;
         if (10 * cost < 9 * best) {
             best = cost;
             best_p = P;
@@ -191,11 +194,11 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
 }
 
 KDA_API kda_status kda_chunk_states(const void* q, const void* k, const void* v, const float* g,
-                                    const float* beta, const float* h0, float* ht, float* m,
-                                    const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
-                                    int B, int T, int N, int H, int dk, int dv, int chunk,
-                                    kda_io_dtype io, void* workspace, size_t workspace_bytes,
-                                    void* stream) {
+                                    const float* beta, float scale, const float* h0, float* ht,
+                                    void* o, float* m, void* w, const int32_t* cu_seqlens,
+                                    const int32_t* cu_seqlens_host, int B, int T, int N, int H,
+                                    int dk, int dv, int chunk, kda_io_dtype io, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
     if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
     if (H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0) return KDA_ERR_INVALID_ARG;
     int64_t T_tot = 0;
@@ -205,16 +208,17 @@ KDA_API kda_status kda_chunk_states(const void* q, const void* k, const void* v,
     for (const void* p : req)
         if (!ok_req(p)) return KDA_ERR_INVALID_ARG;
     if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
-    if (!ok_opt(h0) || !ok_opt(ht) || !ok_opt(m) || !ok_opt(cu_seqlens)) return KDA_ERR_INVALID_ARG;
-    if (ht == nullptr && m == nullptr) return KDA_ERR_INVALID_ARG;
+    if (!ok_opt(h0) || !ok_opt(ht) || !ok_opt(m) || !ok_opt(o) || !ok_opt(w) || !ok_opt(cu_seqlens))
+        return KDA_ERR_INVALID_ARG;
+    if (ht == nullptr && m == nullptr && o == nullptr && w == nullptr) return KDA_ERR_INVALID_ARG;
     if (!cluster_prefill_path(io, dk, dv, chunk)) return KDA_ERR_UNSUPPORTED;
     if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < kda::chunk_tcx_workspace_bytes())
         return KDA_ERR_WORKSPACE;
     unsigned int* err = device_error_word();
     if (err == nullptr) return KDA_ERR_CUDA;
     kda::ChunkArgs a;
-    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.scale = 1.f;
-    a.h0 = h0; a.ht = ht; a.o = nullptr; a.mt = m;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.scale = scale;
+    a.h0 = h0; a.ht = ht; a.o = o; a.mt = m; a.o_trans = w;
     a.cu = cu_seqlens; a.cu_host = cu_seqlens_host;
     a.T_tot = T_tot;
     a.T_pad = cu_seqlens ? 0 : T;
@@ -239,6 +243,36 @@ KDA_API kda_status kda_state_scan(const float* m, const float* s_zero, const flo
     return from_cuda(kda::launch_state_scan(a, static_cast<cudaStream_t>(stream)));
 }
 
+KDA_API kda_status kda_output_correct(const void* w, const float* h, void* o,
+                                      const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                                      int B, int T, int N, int H, int dk, int dv, kda_io_dtype io,
+                                      void* stream) {
+    if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
+    if (H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    int64_t T_tot = 0;
+    int Nn = 0;
+    if (!batch_geometry(cu_seqlens, cu_seqlens_host, B, T, N, &T_tot, &Nn)) return KDA_ERR_INVALID_ARG;
+    if (!ok_req(w) || !ok_req(h) || !ok_req(o) || !ok_opt(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    if (io != KDA_IO_BF16 || dk != 128 || dv != 128) return KDA_ERR_UNSUPPORTED;
+    if (T_tot > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens == nullptr) return KDA_ERR_UNSUPPORTED;      // packed batches (the split's form)
+    int64_t longest = 0;
+    for (int n = 0; n < Nn; ++n) {
+        const int64_t len = (int64_t)cu_seqlens_host[n + 1] - cu_seqlens_host[n];
+        if (len > longest) longest = len;
+    }
+    kda::CorrectArgs c;
+    c.w = static_cast<const __nv_bfloat16*>(w);
+    c.h_ent = h;
+    c.o = static_cast<__nv_bfloat16*>(o);
+    c.seg_cu = cu_seqlens;
+    c.n_stretch = Nn; c.H = H; c.P = 1;
+    c.max_len = longest;
+    c.skip_first = false;
+    c.blocks_per_stretch = 0;
+    return from_cuda(kda::launch_stretch_correct(c, static_cast<cudaStream_t>(stream)));
+}
+
 KDA_API kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_host, int B, int T,
                                                       int N, int H, int dk, int dv, int chunk,
                                                       kda_io_dtype io, int n_split, int* n_split_out,
@@ -251,6 +285,7 @@ KDA_API kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_
     if (!cluster_prefill_path(io, dk, dv, chunk)) return KDA_ERR_UNSUPPORTED;
     const int Nn = cu_seqlens_host ? N : B;
     int64_t longest = cu_seqlens_host ? 0 : T;
+    const int64_t T_tot = cu_seqlens_host ? (int64_t)cu_seqlens_host[N] : (int64_t)B * T;
     if (cu_seqlens_host) {
         if (cu_seqlens_host[0] != 0) return KDA_ERR_INVALID_ARG;
         for (int n = 0; n < N; ++n) {
@@ -263,10 +298,10 @@ KDA_API kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_
     if (P == 0) {
         const int slots = kda::chunk_tcx_cluster_slots();
         if (slots == 0) return KDA_ERR_CUDA;
-        P = auto_split(longest, (int64_t)Nn * H, slots);
+        P = auto_split(longest, T_tot, H, (int64_t)Nn * H, slots);
     }
     *n_split_out = P;
-    *bytes = P == 1 ? kda::chunk_tcx_workspace_bytes() : split_layout(Nn, P, H, dk, dv).total;
+    *bytes = P == 1 ? kda::chunk_tcx_workspace_bytes() : split_layout(Nn, T_tot, P, H, dk, dv).total;
     return KDA_OK;
 }
 
@@ -308,29 +343,43 @@ KDA_API kda_status kda_chunk_fwd_split(const void* q, const void* k, const void*
     const size_t ring = kda::chunk_tcx_workspace_bytes();
     if (P == 1) return from_cuda(kda::launch_chunk_tcx(a, workspace, ring, err, st));
     if (Nn == 0) return KDA_OK;
-    // (1) stretch bounds, (2) each stretch's end state from zero and transition, (3) the join,
-    // (4) each stretch's output from the state entering it
-    const SplitLayout l = split_layout(Nn, P, H, dk, dv);
+    // (1) stretch bounds; (2) every stretch from a zero state: its output, its end state Z, and
+    // in as many extra clusters its transition M and the queries carried back to its start W;
+    // (3) the join, giving each stretch's entering state H and the final states; (4) the
+    // output correction o += W H
+    const SplitLayout l = split_layout(Nn, T_tot, P, H, dk, dv);
     uint8_t* base = static_cast<uint8_t*>(workspace);
     int32_t* seg_cu = reinterpret_cast<int32_t*>(base + l.seg_cu);
     float* m = reinterpret_cast<float*>(base + l.m);
     float* z = reinterpret_cast<float*>(base + l.z);
     float* hs = reinterpret_cast<float*>(base + l.hs);
+    void* w = base + l.w;
     cudaError_t e = kda::launch_split_stretches(cu_seqlens, cu_seqlens ? 0 : T, Nn, P, seg_cu, st);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     kda::ChunkArgs s = a;
     s.cu = seg_cu; s.cu_host = nullptr; s.T_pad = 0; s.N = Nn * P;
-    s.h0 = nullptr; s.ht = z; s.o = nullptr; s.mt = m;
+    s.h0 = nullptr; s.ht = z; s.mt = m; s.o_trans = w;
     if ((e = kda::launch_chunk_tcx(s, workspace, ring, err, st)) != cudaSuccess) return KDA_ERR_CUDA;
     kda::ScanArgs j;
     j.m = m; j.s_zero = z; j.h0 = h0; j.h_start = hs; j.ht = ht;
     j.N = Nn; j.P = P; j.H = H; j.dk = dk; j.dv = dv;
     j.seq_stride = P; j.seg_stride = 1;
     if ((e = kda::launch_state_scan(j, st)) != cudaSuccess) return KDA_ERR_CUDA;
-    kda::ChunkArgs f = a;
-    f.cu = seg_cu; f.cu_host = nullptr; f.T_pad = 0; f.N = Nn * P;
-    f.h0 = hs; f.ht = nullptr;
-    return from_cuda(kda::launch_chunk_tcx(f, workspace, ring, err, st));
+    int64_t longest = cu_seqlens_host ? 0 : T;
+    for (int n = 0; cu_seqlens_host && n < Nn; ++n) {
+        const int64_t len = (int64_t)cu_seqlens_host[n + 1] - cu_seqlens_host[n];
+        if (len > longest) longest = len;
+    }
+    kda::CorrectArgs c;
+    c.w = static_cast<const __nv_bfloat16*>(w);
+    c.h_ent = hs;
+    c.o = static_cast<__nv_bfloat16*>(o);
+    c.seg_cu = seg_cu;
+    c.n_stretch = Nn * P; c.H = H; c.P = P;
+    c.max_len = (((longest + 63) / 64 + P - 1) / P) * 64;
+    c.skip_first = (h0 == nullptr);
+    c.blocks_per_stretch = 0;
+    return from_cuda(kda::launch_stretch_correct(c, st));
 }
 
 KDA_API kda_status kda_chunk_fwd_fused(

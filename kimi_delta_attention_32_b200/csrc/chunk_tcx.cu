@@ -72,8 +72,8 @@ constexpr float kHalfRange = 80.f;       // largest natural-log decay allowed pe
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr long long kDefaultWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
 constexpr int kGate = 1, kNorm = 2, kConv = 4;   // variant bits
-constexpr int kStates = 8;    // states-only launch: no output; the second half of the clusters
-                              // forms transitions
+constexpr int kStates = 8;    // stretch launch: the second half of the clusters forms
+                              // transitions; outputs optional
 constexpr int kHalo = 3;                 // kConv: the conv's three earlier tokens
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -184,9 +184,13 @@ struct Params {
     float scale;
     const float* h0;
     float* ht;
-    __nv_bfloat16* o;                 // (unused by kStates launches)
+    __nv_bfloat16* o;                 // kStates: may be null (no output)
     // kStates: clusters units .. 2 units - 1 form each unit's transition instead (the state
-    // started from the identity, v taken as zero), written to mt [N,H,128,128] (or null: none)
+    // started from the identity, v taken as zero), written to mt [N,H,128,128] (or null: none);
+    // their output, scale M_t^T q_t (the query carried back to the unit's start), goes to o2
+    // through the to2 map (or nowhere when o2 is null)
+    CUtensorMap to2;
+    __nv_bfloat16* o2;
     float* mt;
     int units;                        // N * H
     const int32_t* cu;
@@ -935,6 +939,8 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
     constexpr bool kN = (MODE & kNorm) != 0;
     constexpr bool kSt = (MODE & kStates) != 0;
     const bool trans = kSt && trans_unit;
+    // this unit's output (a transition's goes to o2 through to2), or none
+    const bool has_out = !kSt || (trans ? p.o2 : p.o) != nullptr;
     constexpr bool kCv = (MODE & kConv) != 0;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* misc = sm + C_MISC;
@@ -973,14 +979,16 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 const int c0 = (int)(bos + (int64_t)m * kC);
                 const int rs = m % kRing;
                 const uint8_t* slot = ring + (size_t)rs * kSlotBytes;
-                // V tiles: by TMA from v, or (kConv) the conv's output from the ring slot; none
-                // for a transition (v is taken as zero)
-                if (!kCv && !trans) {
+                // V tiles: by TMA from v, or (kConv) the conv's output from the ring slot. A
+                // transition takes v as zero: its tiles come from token rows before the tensor,
+                // which the copy fills with zeros (the column coordinate stays aligned)
+                if constexpr (!kCv) {
+                    const int vrow = trans ? -2 * kC : c0;
                     for (int hh = 0; hh < 2; ++hh) {
                         uint64_t* vf = bar_at(misc, M_VFULL + 8 * (2 * hh + sl));
                         if (m >= 2 && !(ok = wait_one(bar_at(misc, M_VFREE + 8 * (2 * hh + sl)), pfree, p))) break;
                         mbar_arrive_expect_tx(vf, 8192u);
-                        tma_load_3d(sb + C_V + (uint32_t)(2 * hh + sl) * 8192, &p.tv, 64 * hh, h, c0, vf);
+                        tma_load_3d(sb + C_V + (uint32_t)(2 * hh + sl) * 8192, &p.tv, 64 * hh, h, vrow, vf);
                         v_issued = m + 1;
                     }
                     if (!ok) break;
@@ -1139,11 +1147,14 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             fence_async_smem();
             bar_sync(bar_out, 128);
             if (storer && ok) {
-                tma_store_3d(&p.to, 64 * half, h, (int)c0, sb + ost_h);
+                if constexpr (kSt)
+                    tma_store_3d(trans ? &p.to2 : &p.to, 64 * half, h, (int)c0, sb + ost_h);
+                else
+                    tma_store_3d(&p.to, 64 * half, h, (int)c0, sb + ost_h);
                 bulk_commit();
             }
         } else if (ok) {
-            uint4* dst = reinterpret_cast<uint4*>(p.o + ((c0 + t) * H + h) * kD + jg0);
+            uint4* dst = reinterpret_cast<uint4*>((trans ? p.o2 : p.o) + ((c0 + t) * H + h) * kD + jg0);
 #pragma unroll
             for (int hx = 0; hx < 2; ++hx) {
                 float ov[16];
@@ -1182,7 +1193,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         tc_fence_after();
         if (ok && n > 0 && tid_h == 0) mbar_arrive(bar_at(misc, M_BFREE + 8 * ((n - 1) & 1)));
         if (q < 2) {
-            if (ok && !trans) ok = wait_warp(bar_at(misc, M_VFULL + 8 * (2 * half + b)), (uint32_t)(n >> 1) & 1u, p);
+            if (ok) ok = wait_warp(bar_at(misc, M_VFULL + 8 * (2 * half + b)), (uint32_t)(n >> 1) & 1u, p);
             if (ok) {
                 const int t = 32 * q + lane;
                 const uint8_t* vt = sm + C_V + (uint32_t)(2 * half + b) * 8192;
@@ -1193,8 +1204,8 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
                         const int ck = 4 * cp + 2 * hx + k2;
-                        float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        if (!trans) unpack8(ld16(vt, t * 128 + ((ck ^ (t & 7)) << 4)), vv);
+                        float vv[8];
+                        unpack8(ld16(vt, t * 128 + ((ck ^ (t & 7)) << 4)), vv);
 #pragma unroll
                         for (int u = 0; u < 8; ++u) vv[u] -= xv[8 * k2 + u];
                         st16(sm, u_h + sw128(t, ck, 0, 0), pack8(vv));
@@ -1211,7 +1222,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         // the output of chunk n - 1, by the output warps, while the delta product runs (this
         // keeps it off the path from X(n) to the delta)
         trace_mark(0, n, 8 * half + 4, 256 * half + 64);
-        if (!kSt && q >= 2 && n > 0) epilogue_o(n - 1, ok);
+        if (has_out && q >= 2 && n > 0) epilogue_o(n - 1, ok);
         trace_mark(0, n, 8 * half + 6, 256 * half + 64);
         // (2) state delta Yh^T U (commit), then O(n) += Wh^T U
         if (issuer) {
@@ -1310,7 +1321,7 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         const bool ok = wait_warp(bar_xo, (uint32_t)(nchunks & 1), p);
         if (issuer && ok) ++xo_waited;
         tc_fence_after();
-        if (!kSt && q >= 2) epilogue_o(nchunks - 1, ok);
+        if (has_out && q >= 2) epilogue_o(nchunks - 1, ok);
         stop = bar_sync_or(bar_half, 256, !ok) != 0;
     }
     float* const hdst = trans ? p.mt : p.ht;
@@ -1441,8 +1452,9 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
     if (units == 0) return cudaSuccess;
     const int mode = (a.g_raw != nullptr ? kGate : 0) | (a.z != nullptr ? kNorm : 0) |
                      (a.wconv[0] != nullptr ? kConv : 0);
-    const bool states = (a.o == nullptr);
-    if (states && mode != 0) return cudaErrorInvalidValue;    // states-only: the plain inputs
+    const bool transitions = (a.mt != nullptr || a.o_trans != nullptr);
+    const bool states = (a.o == nullptr || transitions);
+    if (states && mode != 0) return cudaErrorInvalidValue;    // stretch launches: plain inputs
     using KernelFn = void (*)(Params);
     static const KernelFn kernels[8] = {
         chunk_tcx_kernel<0>, chunk_tcx_kernel<1>, chunk_tcx_kernel<2>, chunk_tcx_kernel<3>,
@@ -1463,6 +1475,7 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
         (conv ? make_tmap_thd(&p.tv, a.v, BF, 2, a.T_tot, a.H, kD, kD, tile_rows, false)
               : make_tmap_thd(&p.tv, a.v, BF, 2, a.T_tot, a.H, kD, 64, kC, true)) &&
         (a.o == nullptr || make_tmap_thd(&p.to, a.o, BF, 2, a.T_tot, a.H, kD, 64, kC, true)) &&
+        (a.o_trans == nullptr || make_tmap_thd(&p.to2, a.o_trans, BF, 2, a.T_tot, a.H, kD, 64, kC, true)) &&
         (a.z == nullptr || make_tmap_thd(&p.tz, a.z, BF, 2, a.T_tot, a.H, kD, 64, kC, true));
     if (!maps_ok) return cudaErrorInvalidValue;
     p.q = static_cast<const __nv_bfloat16*>(a.q);
@@ -1474,6 +1487,7 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
     p.ht = a.ht;
     p.o = static_cast<__nv_bfloat16*>(a.o);
     p.mt = a.mt;
+    p.o2 = static_cast<__nv_bfloat16*>(a.o_trans);
     p.units = (int)units;
     p.cu = a.cu;
     p.T_pad = a.T_pad;
@@ -1494,7 +1508,7 @@ cudaError_t launch_chunk_tcx(const ChunkArgs& a, void* workspace, size_t workspa
     p.conv_state = static_cast<const __nv_bfloat16*>(a.conv_state);
     p.l2_eps = a.l2_eps;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(units * (states && a.mt != nullptr ? 2 : 1) * kCluster), 1, 1);
+    cfg.gridDim = dim3((unsigned)(units * (transitions ? 2 : 1) * kCluster), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;

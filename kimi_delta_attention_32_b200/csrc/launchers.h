@@ -2,6 +2,7 @@
 // Arguments are validated by api.cu before any of these is called.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -80,9 +81,12 @@ struct ChunkArgs {
     const float* wconv[3] = {nullptr, nullptr, nullptr};
     const void* conv_state = nullptr;
     float l2_eps = 0.f;
-    // tensor-core path only: a states-only launch (o null) may also form each unit's transition
-    // into mt [N, H, dk, dk] fp32 (mt non-null), in as many extra clusters as units
+    // tensor-core path only, plain inputs: a stretch launch (mt non-null, or o null) forms each
+    // unit's end state (ht) and output (o, may be null) and, in as many extra clusters as units,
+    // its transition M into mt [N, H, dk, dk] fp32 and the output of the transition's run,
+    // scale M_t^T q_t, into o_trans [T_tot, H, dk] bf16 (may be null)
     float* mt = nullptr;
+    void* o_trans = nullptr;
 };
 cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 
@@ -124,5 +128,19 @@ struct ScanArgs {
     int64_t seq_stride, seg_stride;   // stretch p of sequence n is index n * seq_stride + p * seg_stride
 };
 cudaError_t launch_state_scan(const ScanArgs& a, cudaStream_t stream);
+
+// o[t, h, :] += w[t, h, :] h_ent[j, h] over the tokens t of every stretch j (d = 128; bf16 o, w;
+// fp32 h_ent [n_stretch, H, 128, 128]); stretch j covers tokens [seg_cu[j], seg_cu[j+1]).
+struct CorrectArgs {
+    const __nv_bfloat16* w;
+    const float* h_ent;
+    __nv_bfloat16* o;
+    const int32_t* seg_cu;
+    int n_stretch, H, P;
+    int64_t max_len;         // longest stretch (tokens)
+    bool skip_first;         // stretches j with j % P == 0 enter with a zero state
+    int blocks_per_stretch;  // (set by the launcher)
+};
+cudaError_t launch_stretch_correct(const CorrectArgs& a, cudaStream_t stream);
 
 }  // namespace kda

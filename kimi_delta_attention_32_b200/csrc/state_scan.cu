@@ -93,6 +93,157 @@ __global__ void split_stretches_kernel(const int32_t* __restrict__ cu, int T_pad
     if (n == N - 1) seg_cu[(int64_t)N * P] = (int32_t)eos;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Output correction of a split prefill. A stretch's output from its entering state H is
+//     o_t = o_t(from zero) + H^T w_t,   w_t = scale M_t^T q_t,
+// with M_t the transition through token t (the output of the stretch's transition run), so each
+// stretch's output from zero takes one dense product with its entering state:
+//     O[t, :] += W[t, :] H   (W: tokens x dk bf16, H: dk x dv fp32).
+// HBM-bound (read W and O, write O: 768 bytes per token and head for d = 128), on the warp
+// tensor-core MMA (bf16 in, fp32 accumulate). H is split as H = Hhi + Hlo with both halves
+// bf16, which keeps 16 of its mantissa bits (each product within 2^-16 of exact, against 2^-8
+// for H in one bf16); W and O are bf16 in memory anyway.
+// One 256-thread CTA takes up to kCorrTiles tiles of 64 tokens of one (stretch, head): it
+// converts H once into shared memory, then streams the W tiles (cp.async, double-buffered).
+// 8 warps as 4 (16 tokens) x 2 (64 value columns); each warp runs 8 k-steps of 16 channels.
+// ---------------------------------------------------------------------------------------------
+constexpr int kCorrThreads = 256;
+constexpr int kCorrRows = 64;             // tokens per tile
+constexpr int kCorrTiles = 16;            // tiles per CTA
+constexpr int kPitch = 136;               // bf16 per shared row (128 + 8: 272 B, conflict-free)
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+                 "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kCorrThreads) stretch_correct_kernel(const CorrectArgs a) {
+    extern __shared__ __align__(16) __nv_bfloat16 csm[];
+    __nv_bfloat16* sHi = csm;                          // [128][kPitch]  (k = channel, n = value)
+    __nv_bfloat16* sLo = sHi + 128 * kPitch;
+    __nv_bfloat16* sW = sLo + 128 * kPitch;            // 2 x [kCorrRows][kPitch]
+    const int H = a.H;
+    const int blocks = a.blocks_per_stretch;
+    const int b = blockIdx.x % blocks;
+    const int jh = blockIdx.x / blocks;
+    const int j = jh / H, h = jh % H;
+    if (a.skip_first && j % a.P == 0) return;          // entering state zero: nothing to add
+    const int64_t bos = a.seg_cu[j], eos = a.seg_cu[j + 1];
+    const int64_t t_begin = bos + (int64_t)b * kCorrTiles * kCorrRows;
+    if (t_begin >= eos) return;
+    const int64_t t_end = eos < t_begin + kCorrTiles * kCorrRows ? eos : t_begin + kCorrTiles * kCorrRows;
+    const int ntiles = (int)((t_end - t_begin + kCorrRows - 1) / kCorrRows);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // W tile loader: 64 rows x 256 B = 1024 16-byte pieces, 4 per thread (rows past the end are
+    // not loaded; their products are never stored)
+    auto load_tile = [&](int tile, int buf) {
+        const int64_t t0 = t_begin + (int64_t)tile * kCorrRows;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int piece = tid + e * kCorrThreads;
+            const int r = piece >> 4, c = piece & 15;
+            if (t0 + r < t_end)
+                cp_async16(smem_addr(sW + (buf * kCorrRows + r) * kPitch + 8 * c),
+                           a.w + ((t0 + r) * H + h) * 128 + 8 * c);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    load_tile(0, 0);
+    // H = Hhi + Hlo, both bf16
+    const float* Hg = a.h_ent + ((size_t)j * H + h) * 128 * 128;
+    for (int e = tid; e < 128 * 32; e += kCorrThreads) {
+        const int r = e >> 5, c4 = e & 31;
+        const float4 v = reinterpret_cast<const float4*>(Hg + r * 128)[c4];
+        const float x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x[u]);
+            sHi[r * kPitch + 4 * c4 + u] = hi;
+            sLo[r * kPitch + 4 * c4 + u] = __float2bfloat16_rn(x[u] - __bfloat162float(hi));
+        }
+    }
+    const int wr = warp & 3, wc = warp >> 2;           // 16-token row block, 64-column half
+    for (int tile = 0; tile < ntiles; ++tile) {
+        const int buf = tile & 1;
+        if (tile + 1 < ntiles) {
+            load_tile(tile + 1, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();                               // tile `tile` (and H) visible to all
+        float acc[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[nt][u] = 0.f;
+        const __nv_bfloat16* wt = sW + buf * kCorrRows * kPitch;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t af[4];
+            ldsm_x4(smem_addr(wt + (16 * wr + (lane & 15)) * kPitch + 16 * ks + 8 * (lane >> 4)),
+                    af[0], af[1], af[2], af[3]);
+            const int krow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {           // pairs of 8-column tiles
+                const int ncol = 64 * wc + 16 * np + 8 * (lane >> 4);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(smem_addr(sHi + krow * kPitch + ncol), b0, b1, b2, b3);
+                mma_bf16_16816(acc[2 * np], af, b0, b1);
+                mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
+                ldsm_x4_t(smem_addr(sLo + krow * kPitch + ncol), b0, b1, b2, b3);
+                mma_bf16_16816(acc[2 * np], af, b0, b1);
+                mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
+            }
+        }
+        // O[t, :] += acc (C fragment: rows lane/4 and lane/4 + 8, columns 2 (lane % 4) + {0, 1});
+        // all 16 reads are issued before the first write, so the tile pays one round trip
+        const int64_t t0 = t_begin + (int64_t)tile * kCorrRows + 16 * wr + (lane >> 2);
+        uint32_t* orow[2];
+        uint32_t ov[2][8];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int64_t t = t0 + 8 * half;
+            orow[half] = t < t_end ? reinterpret_cast<uint32_t*>(a.o + (t * H + h) * 128) : nullptr;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+                ov[half][nt] = orow[half] ? __ldcs(orow[half] + ((64 * wc + 8 * nt + 2 * (lane & 3)) >> 1)) : 0u;
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            if (orow[half] == nullptr) continue;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                __nv_bfloat162 o2 = *reinterpret_cast<__nv_bfloat162*>(&ov[half][nt]);
+                const float2 o0 = __bfloat1622float2(o2);
+                o2 = __floats2bfloat162_rn(o0.x + acc[nt][2 * half], o0.y + acc[nt][2 * half + 1]);
+                __stcs(orow[half] + ((64 * wc + 8 * nt + 2 * (lane & 3)) >> 1),
+                       *reinterpret_cast<uint32_t*>(&o2));
+            }
+        }
+        __syncthreads();                               // buffer `buf` is reloaded next
+    }
+}
+
 template <int DK>
 cudaError_t launch_scan_t(const ScanArgs& a, cudaStream_t stream) {
     const size_t smem = sizeof(float) * ((size_t)DK * (DK + 1) + (size_t)DK * kScanCols);
@@ -110,6 +261,19 @@ cudaError_t launch_split_stretches(const int32_t* cu, int T_pad, int N, int P, i
                                    cudaStream_t stream) {
     if (N == 0) return cudaSuccess;
     split_stretches_kernel<<<(N + 127) / 128, 128, 0, stream>>>(cu, T_pad, N, P, seg_cu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_stretch_correct(const CorrectArgs& a, cudaStream_t stream) {
+    if (a.n_stretch == 0 || a.H == 0 || a.max_len == 0) return cudaSuccess;
+    const size_t smem = sizeof(__nv_bfloat16) * (size_t)kPitch * (2 * 128 + 2 * kCorrRows);
+    cudaError_t e = cudaFuncSetAttribute(stretch_correct_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    CorrectArgs c = a;
+    c.blocks_per_stretch = (int)((a.max_len + kCorrTiles * kCorrRows - 1) / (kCorrTiles * kCorrRows));
+    const int64_t blocks = (int64_t)a.n_stretch * a.H * c.blocks_per_stretch;
+    stretch_correct_kernel<<<(unsigned)blocks, kCorrThreads, smem, stream>>>(c);
     return cudaGetLastError();
 }
 

@@ -24,7 +24,7 @@ EXPORTED = ("kda_status_string", "kda_version", "kda_conv_fwd", "kda_chunk_fwd_w
             "kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_fwd_noalloc", "kda_recurrent_step",
             "kda_conv_recurrent_step", "kda_fused_recurrent_step", "kda_set_wait_limit",
             "kda_last_device_error", "kda_chunk_states", "kda_state_scan",
-            "kda_chunk_fwd_split_workspace_size", "kda_chunk_fwd_split")
+            "kda_chunk_fwd_split_workspace_size", "kda_chunk_fwd_split", "kda_output_correct")
 
 _lock = threading.Lock()
 _lib = None
@@ -85,8 +85,8 @@ def load_library(path: str = LIB_PATH):
         lib.kda_last_device_error.argtypes = [vp]
         lib.kda_last_device_error.restype = ci
         cip = ctypes.POINTER(ctypes.c_int32)
-        lib.kda_chunk_states.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, i32p, cip, ci, ci, ci, ci,
-                                         ci, ci, ci, ci, vp, cs, vp]
+        lib.kda_chunk_states.argtypes = [vp, vp, vp, fp, fp, cf, fp, fp, vp, fp, vp, i32p, cip, ci,
+                                         ci, ci, ci, ci, ci, ci, ci, vp, cs, vp]
         lib.kda_chunk_states.restype = ci
         lib.kda_state_scan.argtypes = [fp, fp, fp, fp, fp, ci, ci, ci, ci, ci, ctypes.c_int64,
                                        ctypes.c_int64, vp]
@@ -97,6 +97,8 @@ def load_library(path: str = LIB_PATH):
         lib.kda_chunk_fwd_split.argtypes = [vp, vp, vp, fp, fp, cf, fp, fp, vp, i32p, cip, ci, ci,
                                             ci, ci, ci, ci, ci, ci, ci, vp, cs, vp]
         lib.kda_chunk_fwd_split.restype = ci
+        lib.kda_output_correct.argtypes = [vp, fp, vp, i32p, cip, ci, ci, ci, ci, ci, ci, ci, vp]
+        lib.kda_output_correct.restype = ci
         if path == LIB_PATH:
             _lib = lib
         return lib
@@ -205,26 +207,31 @@ def _batch(q, cu_seqlens, cu_host):
     return 1, 0, len(cu_host) - 1, T_tot, H, dk
 
 
-def chunk_states(q, k, v, g, beta, h0=None, cu_seqlens=None, cu_host=None, chunk=64,
-                 end_state=True, transition=True, workspace=None, stream=None):
-    """End states (started from h0, or zero) and transitions of every (sequence, head), without
-    the output. Returns (ht [N,H,dk,dv] or None, m [N,H,dk,dk] or None), both fp32."""
+def chunk_states(q, k, v, g, beta, scale=1.0, h0=None, cu_seqlens=None, cu_host=None, chunk=64,
+                 end_state=True, transition=True, output=False, carried_queries=False,
+                 workspace=None, stream=None):
+    """Per (sequence, head): the end state started from h0 (or zero), the transition M, the
+    output (as chunk_fwd), and the queries carried back to the start, scale M_t^T q_t.
+    Returns (ht [N,H,dk,dv], m [N,H,dk,dk], o [T,H,dv], w [T,H,dk]); each None unless asked."""
     lib = load_library()
     B, T, N, T_tot, H, dk = _batch(q, cu_seqlens, cu_host)
     dv = v.shape[-1]
     ht = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device) if end_state else None
     m = torch.empty((N, H, dk, dk), dtype=torch.float32, device=q.device) if transition else None
+    o = torch.empty_like(v) if output else None
+    w = torch.empty_like(q) if carried_queries else None
     io = _io(q)
     if workspace is None:
         need = chunk_fwd_workspace_size(N, T_tot, H, dk, dv, chunk, io)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     keep, cuh = _host_cu(cu_host)
-    st = lib.kda_chunk_states(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(ht),
-                              _ptr(m), _ptr(cu_seqlens), cuh, B, T, N, H, dk, dv, chunk, io,
-                              _ptr(workspace), workspace.numel(), _stream(stream))
+    st = lib.kda_chunk_states(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                              _ptr(h0), _ptr(ht), _ptr(o), _ptr(m), _ptr(w), _ptr(cu_seqlens), cuh,
+                              B, T, N, H, dk, dv, chunk, io, _ptr(workspace), workspace.numel(),
+                              _stream(stream))
     del keep
     _check("kda_chunk_states", st)
-    return ht, m
+    return ht, m, o, w
 
 
 def state_scan(m, s_zero, h0=None, *, N, P, seq_stride, seg_stride, h_start=None, ht=None,
@@ -242,6 +249,18 @@ def state_scan(m, s_zero, h0=None, *, N, P, seq_stride, seg_stride, h_start=None
                                                 _ptr(ht), N, P, H, dk, dv, seq_stride, seg_stride,
                                                 _stream(stream)))
     return h_start, ht
+
+
+def output_correct(w, h, o, cu_seqlens, cu_host, stream=None):
+    """o[t] += h[n]^T w[t] for the tokens t of every sequence n (packed batch, in place)."""
+    lib = load_library()
+    T_tot, H, dk = w.shape
+    keep, cuh = _host_cu(cu_host)
+    st = lib.kda_output_correct(_ptr(w), _ptr(h), _ptr(o), _ptr(cu_seqlens), cuh, 1, 0,
+                                len(cu_host) - 1, H, dk, o.shape[-1], _io(o), _stream(stream))
+    del keep
+    _check("kda_output_correct", st)
+    return o
 
 
 def chunk_fwd_split_plan(q, v, cu_seqlens=None, cu_host=None, n_split=0, chunk=64):

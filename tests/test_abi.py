@@ -247,8 +247,10 @@ def test_split_workspace_query(lib):
         sizes.append(out.value)
     assert sizes[0] == ring.value                       # one stretch: kda_chunk_fwd's rings
     # rings + stretch bounds + (transition, end state, entering state) per stretch and head
+    # + the carried-back queries (bf16, one row per token and head)
     per = 4 * 128 * 128 * 3
-    assert sizes[1] >= ring.value + 2 * 4 * per and sizes[2] >= ring.value + 8 * 4 * per
+    wq = 8192 * 4 * 128 * 2
+    assert sizes[1] >= ring.value + 2 * 4 * per + wq and sizes[2] >= ring.value + 8 * 4 * per + wq
     assert sizes[2] - sizes[1] < 6 * 4 * per + 1024
     keep, cuh = _cu_host([0, 100, 100, 5000])
     assert lib.kda_chunk_fwd_split_workspace_size(cuh, 0, 0, 3, 4, 128, 128, 64, 1, 3,
@@ -270,17 +272,20 @@ def test_split_workspace_query(lib):
 
 
 def _states(lib, **kw):
-    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, h0=None, ht=FAKE, m=FAKE, cu=None,
-             cuh=None, B=1, T=64, N=1, H=2, dk=128, dv=128, chunk=64, io=1, ws=FAKE,
-             wsb=1 << 40, stream=None)
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, scale=1.0, h0=None, ht=FAKE, o=None, m=FAKE,
+             w=None, cu=None, cuh=None, B=1, T=64, N=1, H=2, dk=128, dv=128, chunk=64, io=1,
+             ws=FAKE, wsb=1 << 40, stream=None)
     a.update(kw)
-    return lib.kda_chunk_states(a["q"], a["k"], a["v"], a["g"], a["beta"], a["h0"], a["ht"], a["m"],
-                                a["cu"], a["cuh"], a["B"], a["T"], a["N"], a["H"], a["dk"], a["dv"],
-                                a["chunk"], a["io"], a["ws"], a["wsb"], a["stream"])
+    return lib.kda_chunk_states(a["q"], a["k"], a["v"], a["g"], a["beta"], a["scale"], a["h0"],
+                                a["ht"], a["o"], a["m"], a["w"], a["cu"], a["cuh"], a["B"], a["T"],
+                                a["N"], a["H"], a["dk"], a["dv"], a["chunk"], a["io"], a["ws"],
+                                a["wsb"], a["stream"])
 
 
 def test_chunk_states_checks_arguments(lib):
     assert _states(lib, ht=None, m=None) == kda.KDA_ERR_INVALID_ARG     # nothing to form
+    assert _states(lib, o=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert _states(lib, w=MIS) == kda.KDA_ERR_INVALID_ARG
     assert _states(lib, q=None) == kda.KDA_ERR_INVALID_ARG
     assert _states(lib, m=MIS) == kda.KDA_ERR_INVALID_ARG
     assert _states(lib, beta=None) == kda.KDA_ERR_INVALID_ARG
@@ -319,3 +324,21 @@ def test_chunk_fwd_split_checks_arguments(lib):
     assert split(chunk=32) == kda.KDA_ERR_UNSUPPORTED
     assert split() == kda.KDA_ERR_WORKSPACE                            # 16 bytes is too small
     assert split(ws=None, wsb=1 << 40) == kda.KDA_ERR_WORKSPACE
+
+
+def test_output_correct_checks_arguments(lib):
+    keep, cuh = _cu_host([0, 10, 30])
+
+    def corr(**kw):
+        a = dict(w=FAKE, h=FAKE, o=FAKE, cu=FAKE, cuh=cuh, N=2, H=2, dk=128, dv=128, io=1)
+        a.update(kw)
+        return lib.kda_output_correct(a["w"], a["h"], a["o"], a["cu"], a["cuh"], 0, 0, a["N"],
+                                      a["H"], a["dk"], a["dv"], a["io"], None)
+    assert corr(w=None) == kda.KDA_ERR_INVALID_ARG
+    assert corr(h=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert corr(cuh=None) == kda.KDA_ERR_INVALID_ARG                     # host copy missing
+    assert corr(H=0) == kda.KDA_ERR_INVALID_ARG
+    assert corr(io=0) == kda.KDA_ERR_UNSUPPORTED
+    assert corr(dk=64) == kda.KDA_ERR_UNSUPPORTED
+    assert corr(cu=None, cuh=None) == kda.KDA_ERR_UNSUPPORTED            # padded: not supported
+    del keep

@@ -1,8 +1,10 @@
 """The context-parallel prefill's orchestration (kimi_delta_attention_32_b200.cp) on CPU: ranks
-as gloo processes, each holding one stretch of every sequence, with the four steps run by fp64
-stand-ins written from the oracle (end states and transitions, the join, the stretch's output).
+as gloo processes, each holding one stretch of every sequence, with the steps run by fp64
+stand-ins written from the oracle (the stretch from a zero state with its transition and
+carried-back queries, the join, the output correction).
 The assembled outputs and final states must equal the oracle run over whole sequences: this
-checks which stretch each rank forms, the order of the all-gather and the join's indexing.
+checks which stretch each rank forms, the order of the all-gather, the join's indexing and the
+output correction's entering states.
 The libkda steps themselves are checked against the oracle on the GPU."""
 from __future__ import annotations
 
@@ -53,11 +55,17 @@ def _cuts(world):
 class _OracleOps:
     """fp64 stand-ins for the libkda steps (test infrastructure only)."""
 
-    def chunk_states(self, q, k, v, g, beta, cu_seqlens, cu_host):
+    def chunk_states(self, q, k, v, g, beta, scale, cu_seqlens, cu_host):
         a = [x.numpy() for x in (q, k, v, g, beta)]
-        _, z = oracle.kda_fwd(*a, 1.0, None, cu_host, nthreads=1)
+        o, z = oracle.kda_fwd(*a, scale, None, cu_host, nthreads=1)
         m = oracle.transition(a[1], a[3], a[4], cu_host, nthreads=1)
-        return torch.from_numpy(z), torch.from_numpy(m)
+        # the queries carried back to each stretch's start: the output of the run with v = 0
+        # started from the identity
+        eye = np.broadcast_to(np.eye(DK), (len(cu_host) - 1, H, DK, DK))
+        w, _ = oracle.kda_fwd(a[0], a[1], np.zeros_like(a[0]), a[3], a[4], scale, eye, cu_host,
+                              nthreads=1)
+        return (torch.from_numpy(z), torch.from_numpy(m), torch.from_numpy(o),
+                torch.from_numpy(w))
 
     def state_scan(self, m, z, h0, N, P, seq_stride, seg_stride):
         m, z = m.numpy(), z.numpy()
@@ -72,10 +80,12 @@ class _OracleOps:
             ht[n] = cur
         return torch.from_numpy(hs), torch.from_numpy(ht)
 
-    def chunk_fwd(self, q, k, v, g, beta, scale, h0, cu_seqlens, cu_host):
-        a = [x.numpy() for x in (q, k, v, g, beta)]
-        o, _ = oracle.kda_fwd(*a, scale, h0.numpy(), cu_host, nthreads=1)
-        return torch.from_numpy(o), None
+    def output_correct(self, w, h, o, cu_seqlens, cu_host):
+        w, h, o = w.numpy(), h.numpy(), o.numpy().copy()
+        for n in range(len(cu_host) - 1):
+            sl = slice(cu_host[n], cu_host[n + 1])
+            o[sl] += np.einsum("thi,hic->thc", w[sl], h[n])
+        return torch.from_numpy(o)
 
 
 def _rank_main(rank, world, port, out):

@@ -54,33 +54,45 @@ def _per_unit_worst_o(o, ref, cu, H):
 def test_chunk_states_match_oracle():
     lens = [1, 63, 64, 65, 0, 130, 700]
     d = _inputs(lens, 3, 51)
-    ht, m = kda.chunk_states(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
-                             cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"])
+    ht, m, o, w = kda.chunk_states(d["q"], d["k"], d["v"], d["g"], d["beta"], 0.5, h0=d["h0"],
+                                   cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], output=True,
+                                   carried_queries=True)
     torch.cuda.synchronize()
-    _, ht_ref = oracle.kda_fwd(to64(d["q"]), to64(d["k"]), to64(d["v"]), to64(d["g"]),
-                               to64(d["beta"]), 1.0, to64(d["h0"]), d["cu_host"])
-    m_ref = oracle.transition(to64(d["k"]), to64(d["g"]), to64(d["beta"]), d["cu_host"])
-    ht, m = to64(ht), to64(m)
+    q64, k64, g64, b64 = to64(d["q"]), to64(d["k"]), to64(d["g"]), to64(d["beta"])
+    o_ref, ht_ref = oracle.kda_fwd(q64, k64, to64(d["v"]), g64, b64, 0.5, to64(d["h0"]),
+                                   d["cu_host"])
+    m_ref = oracle.transition(k64, g64, b64, d["cu_host"])
+    # w_t = scale M_t^T q_t: the output of the run with v = 0 started from the identity
+    eye = np.broadcast_to(np.eye(128), (len(lens), 3, 128, 128))
+    w_ref, _ = oracle.kda_fwd(q64, k64, np.zeros_like(q64), g64, b64, 0.5, eye, d["cu_host"])
+    ht, m, o, w = to64(ht), to64(m), to64(o), to64(w)
     eh, em = _per_unit_worst(ht, ht_ref), _per_unit_worst(m, m_ref)
-    record_margin("chunk_states (7 ragged seqs x 3 heads)", "end state, worst unit", eh, TOL_BF16)
-    record_margin("chunk_states (7 ragged seqs x 3 heads)", "transition, worst unit", em, TOL_BF16)
-    assert eh <= TOL_BF16 and em <= TOL_BF16
+    eo = _per_unit_worst_o(o, o_ref, d["cu_host"], 3)
+    ew = _per_unit_worst_o(w, w_ref, d["cu_host"], 3)
+    label = "chunk_states (7 ragged seqs x 3 heads)"
+    record_margin(label, "end state, worst unit", eh, TOL_BF16)
+    record_margin(label, "output, worst unit", eo, TOL_BF16)
+    record_margin(label, "transition, worst unit", em, TOL_BF16)
+    record_margin(label, "carried queries, worst unit", ew, TOL_BF16)
+    assert max(eh, em, eo, ew) <= TOL_BF16
     # an empty sequence: the identity, and the state it was given
     assert np.array_equal(m[4], np.broadcast_to(np.eye(128), (3, 128, 128)))
     assert np.array_equal(ht[4], to64(d["h0"][4]))
 
 
 def test_chunk_states_end_state_only_equals_prefill_state():
-    """Without transitions the launch forms the end states kda_chunk_fwd forms (same
-    arithmetic; only the output store is left out)."""
+    """Without transitions the launch forms the end states and outputs kda_chunk_fwd forms
+    (same arithmetic)."""
     d = _inputs([500, 1, 129], 2, 52)
-    ht, m = kda.chunk_states(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
-                             cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], transition=False)
-    _, ht_ref = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], 1.0, h0=d["h0"],
-                              cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"])
+    ht, m, o, _ = kda.chunk_states(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
+                                   cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"],
+                                   transition=False, output=True)
+    o_ref, ht_ref = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], 1.0, h0=d["h0"],
+                                  cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"])
     torch.cuda.synchronize()
     assert m is None
     assert rel_l2(to64(ht), to64(ht_ref)) <= 1e-6
+    assert rel_l2(to64(o), to64(o_ref)) <= 1e-6
 
 
 @pytest.mark.parametrize("dk,strides", [(128, "seq_major"), (128, "seg_major"), (64, "seq_major")])
@@ -161,3 +173,32 @@ def test_long_256k_tp4_split_full():
                                 cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"])
     torch.cuda.synchronize()
     _check_split(d, o, ht, f"long_256k_tp4 (all 8 heads, {P} stretches)")
+
+
+def test_output_correct_matches_host_product():
+    """o[t] += h[n]^T w[t] per sequence, against an fp64 product of the same bf16 inputs. h is
+    taken as two bf16 halves (16 mantissa bits: each product within 2^-16 of exact), and the
+    sum is rounded once to bf16, so every element lies within
+    2^-8 |ref| + 2^-14 sum_i |w_i h_ij| of the exact value (each term with a 2x-4x margin)."""
+    lens = [1, 700, 0, 64, 1500]
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    H = 3
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(56)
+    w = torch.randn((cu[-1], H, 128), generator=gen, device=DEV).bfloat16()
+    o = torch.randn((cu[-1], H, 128), generator=gen, device=DEV).bfloat16()
+    h = torch.randn((len(lens), H, 128, 128), generator=gen, device=DEV) * 0.1
+    ref = to64(o).copy()
+    mag = np.zeros_like(ref)
+    w64, h64 = to64(w), to64(h)
+    for n in range(len(lens)):
+        ref[cu[n]:cu[n + 1]] += np.einsum("thi,hic->thc", w64[cu[n]:cu[n + 1]], h64[n])
+        mag[cu[n]:cu[n + 1]] = np.einsum("thi,hic->thc", np.abs(w64[cu[n]:cu[n + 1]]), np.abs(h64[n]))
+    cu_t = torch.tensor(cu, dtype=torch.int32, device=DEV)
+    kda.output_correct(w, h, o, cu_t, cu)
+    torch.cuda.synchronize()
+    excess = np.abs(to64(o) - ref) / (2.0 ** -8 * np.abs(ref) + 2.0 ** -14 * mag)
+    assert np.max(excess) <= 1.0, f"error {np.max(excess):.2f}x its bound"
+    assert rel_l2(to64(o), ref) <= 2e-3
