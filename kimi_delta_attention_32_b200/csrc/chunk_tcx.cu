@@ -148,10 +148,10 @@ constexpr uint32_t M_WCV = 2816;      // kConv: this head's conv weights, halved
                                       //   channel groups read 16 consecutive float4)
 constexpr uint32_t kMiscP = M_WCV + 3 * 128 * 16;
 // consumer barriers ([X ; O] and delta per half; A, B parts per slot; V per half and slot;
-// kNorm: the halves' sums of squares per chunk parity, each half's output complete, each half's
-// output gate tile)
+// kNorm: the halves' sums of squares per chunk parity, each half's output gate tile; 224..239
+// spare)
 constexpr uint32_t M_XO = 0, M_DS = 16, M_AFULL = 32, M_BFULL = 48, M_AFREE = 64, M_BFREE = 80,
-                   M_VFULL = 96, M_VFREE = 128, M_GFULL = 160, M_NRM = 208, M_OD = 224, M_ZFULL = 240;
+                   M_VFULL = 96, M_VFREE = 128, M_GFULL = 160, M_NRM = 208, M_ZFULL = 240;
 constexpr int kBarsC = 32;
 constexpr uint32_t M_WN = 512;        // kNorm: the norm weight [128]
 constexpr uint32_t M_SS = 1024;       // kNorm: sums of squares [chunk % 3][half][column part][64]
@@ -229,6 +229,18 @@ __device__ __forceinline__ float softplus_fast(float x) {
 // sigmoid with the fast divide (two ulp, far below the bf16 rounding of what it scales; the
 // correctly rounded divide's software sequence cost the normed prefill half its time)
 __device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 with one SFU operation (tanh.approx: absolute error below
+// 2.5e-4 in the sigmoid; the output gate it feeds is stored as bf16, relative error 2^-9)
+__device__ __forceinline__ float sigmoid_tanh(float x) {
+    float th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(0.5f * x));
+    return fmaf(0.5f, th, 0.5f);
+}
+// Prefetch of a 3-D tiled box into L2 (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(tmap), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
 // silu(z) from h = z / 2: h + h tanh(h) (the conv prologue sums with halved weights).
 __device__ __forceinline__ float silu_half(float hz) {
     float th;
@@ -1095,6 +1107,42 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
     // the swizzled staging and one TMA store, or straight to global for a ragged last chunk
     // (rows past the sequence belong to the next one). The named barriers run whether or not
     // `ok` holds, so the four warps always meet.
+    // kNorm, by the output warps once O(nn) is complete in tensor memory (the wait for the
+    // [X ; O] products of chunk nn + 1 covers it), while the other warps form U: the per-token
+    // sums of squares over this half's 64 columns, published for both halves' epilogues, and
+    // the gate tile of chunk nn (landed in the staging buffer) turned into sigmoid(z) w_norm in
+    // place. Returns false if a wait gave up; the named barrier runs either way.
+    auto norm_prep = [&](int nn, bool ok) -> bool {
+        const int t = 32 * (q - 2) + lane;
+        float ss = 0.f;
+        if (ok) {
+#pragma unroll
+            for (int hx = 0; hx < 2; ++hx) {
+                float ov[16];
+                tmem_ld16(t_xo + 64 * (nn & 1) + lane_sel + 32 * cp + 16 * hx, ov);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) ss = fmaf(ov[u], ov[u], ss);
+            }
+        }
+        float* s_ss = reinterpret_cast<float*>(misc + M_SS) + (nn % 3) * 256;
+        s_ss[(2 * half + cp) * 64 + t] = ss * p.scale * p.scale;
+        bar_sync(bar_out, 128);
+        if (ok && lw == 2 && lane == 0) mbar_arrive(bar_at(misc, M_NRM + 8 * (nn & 1)));
+        ok = ok && wait_warp(bar_at(misc, M_ZFULL + 8 * half), (uint32_t)nn & 1u, p);
+        if (ok) {
+            const float* wn = reinterpret_cast<const float*>(misc + M_WN) + jg0;
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+                const uint32_t off = ost_h + sw128(t, 4 * cp + k8, 0, 0);
+                float zv[8];
+                unpack8(ld16(sm, off), zv);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) zv[u] = sigmoid_tanh(zv[u]) * wn[8 * k8 + u];
+                st16(sm, off, pack8(zv));
+            }
+        }
+        return ok;
+    };
     auto epilogue_o = [&](int nn, bool ok) {
         const int64_t c0 = bos + (int64_t)nn * kC;
         const int L = (int)(eos - c0 < kC ? eos - c0 : kC);
@@ -1103,13 +1151,12 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         float inv = 0.f;                            // kNorm: 1 / rms of token t over 128 columns
         uint4 zr[4];
         if constexpr (kN) {
-            // the gate of this thread's 32 outputs: TMA-loaded into the staging tile beforehand
-            // (each thread overwrites exactly the 16-byte chunks it reads)
-            ok = ok && wait_warp(bar_at(misc, M_ZFULL + 8 * half), (uint32_t)nn & 1u, p);
+            // sigmoid(z) w_norm for this thread's 32 outputs, formed in the staging tile by
+            // norm_prep (the same thread, the same 16-byte chunks, which it overwrites below)
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8)
                 zr[k8] = ok ? ld16(sm, ost_h + sw128(t, 4 * cp + k8, 0, 0)) : make_uint4(0, 0, 0, 0);
-            // both halves' sums of squares of chunk nn, published a step earlier (see (3))
+            // both halves' sums of squares of chunk nn, published by norm_prep
             const float* s_ss = reinterpret_cast<const float*>(misc + M_SS) + (nn % 3) * 256;
             ok = ok && wait_warp(bar_at(misc, M_NRM + 8 * (nn & 1)), (uint32_t)(nn >> 1) & 1u, p);
             if (ok) {
@@ -1122,12 +1169,11 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
 #pragma unroll
             for (int u = 0; u < 16; ++u) ov[u] *= p.scale;
             if constexpr (kN) {
-                const float* wn = reinterpret_cast<const float*>(misc + M_WN) + jg0 + 16 * hx;
                 float zv[16];
                 unpack8(zr[2 * hx], zv);
                 unpack8(zr[2 * hx + 1], zv + 8);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) ov[u] = ov[u] * inv * wn[u] * sigmoid_f(zv[u]);
+                for (int u = 0; u < 16; ++u) ov[u] = ov[u] * inv * zv[u];
             }
         };
         if (L == kC) {
@@ -1174,6 +1220,10 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
     // of chunk n, well after chunk n - 1's output has been read from it; the epilogue of chunk n
     // reads it a step later
     int z_issued = 0;
+    if (kN && lw == 2 && lane == 0 && !stop) {       // the first two gate tiles into L2
+        for (int nn = 0; nn < 2 && nn < nchunks; ++nn)
+            tma_prefetch_l2_3d(&p.tz, 64 * half, h, (int)(bos + (int64_t)nn * kC));
+    }
     // prologue: Sm(0), then [X ; O](0)
     if (!stop && nchunks > 0) {
         const bool ok = wait_warp(bar_at(misc, M_AFULL), 0, p);
@@ -1192,6 +1242,9 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         if (issuer && ok) ++xo_waited;
         tc_fence_after();
         if (ok && n > 0 && tid_h == 0) mbar_arrive(bar_at(misc, M_BFREE + 8 * ((n - 1) & 1)));
+        if constexpr (kN) {
+            if (q >= 2 && n > 0) ok = norm_prep(n - 1, ok);
+        }
         if (q < 2) {
             if (ok) ok = wait_warp(bar_at(misc, M_VFULL + 8 * (2 * half + b)), (uint32_t)(n >> 1) & 1u, p);
             if (ok) {
@@ -1240,7 +1293,6 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                     for (int s = 0; s < 4; ++s)
                         mma_bf16(t_xo + 64 * b, make_desc(bp + 8192 + s * 32, 16, 1024),
                                  make_desc(sb + u_h + s * 2048, 8192, 1024), id, 1);
-                    if (kN) mma_commit(bar_at(misc, M_OD + 8 * half));   // O(n) is complete
                 }
                 __syncwarp();
                 ++ds_issued;
@@ -1263,29 +1315,6 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
                 for (int u = 0; u < 16; ++u) S[16 * hx + u] = fmaf(eC, S[16 * hx + u], dv[u]);
             }
         }
-        if (kN && q >= 2) {
-            // the output's per-token sums of squares over this half's 64 columns, published for
-            // both halves' epilogues of chunk n (one step later). Three buffers: a half can run
-            // at most two chunks ahead of the other (they share the A buffers).
-            bool oko = ok && wait_warp(bar_at(misc, M_OD + 8 * half), (uint32_t)b, p);
-            trace_mark(0, n, 8 * half + 7, 256 * half + 64);
-            tc_fence_after();
-            float ss = 0.f;
-            if (oko) {
-#pragma unroll
-                for (int hx = 0; hx < 2; ++hx) {
-                    float ov[16];
-                    tmem_ld16(t_xo + 64 * b + lane_sel + 32 * cp + 16 * hx, ov);
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) ss = fmaf(ov[u], ov[u], ss);
-                }
-            }
-            float* s_ss = reinterpret_cast<float*>(misc + M_SS) + (n % 3) * 256;
-            s_ss[(2 * half + cp) * 64 + 32 * (q - 2) + lane] = ss * p.scale * p.scale;
-            bar_sync(bar_out, 128);
-            if (oko && lw == 2 && lane == 0) mbar_arrive(bar_at(misc, M_NRM + 8 * (n & 1)));
-            ok = oko;
-        }
         if (ok) {
             if (n + 1 < nchunks) {
                 ok = wait_warp(bar_at(misc, M_AFULL + 8 * ((n + 1) & 1)), (uint32_t)((n + 1) >> 1) & 1u, p);
@@ -1304,6 +1333,8 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
             mbar_arrive_expect_tx(zf, 8192u);
             tma_load_3d(sb + ost_h, &p.tz, 64 * half, h, (int)(bos + (int64_t)n * kC), zf);
             z_issued = n + 1;
+            // the gate tile two chunks on, into L2, so that its load then hits L2
+            if (n + 2 < nchunks) tma_prefetch_l2_3d(&p.tz, 64 * half, h, (int)(bos + (int64_t)(n + 2) * kC));
         }
         // (4) the next chunk's [X ; O], or a commit that covers O(n) after the last chunk
         if (issuer) {
@@ -1321,7 +1352,11 @@ __device__ void consumer(const Params& p, uint8_t* sm, uint32_t sb, int n_seq, i
         const bool ok = wait_warp(bar_xo, (uint32_t)(nchunks & 1), p);
         if (issuer && ok) ++xo_waited;
         tc_fence_after();
-        if (has_out && q >= 2) epilogue_o(nchunks - 1, ok);
+        bool oke = ok;
+        if constexpr (kN) {
+            if (q >= 2) oke = norm_prep(nchunks - 1, oke);
+        }
+        if (has_out && q >= 2) epilogue_o(nchunks - 1, oke);
         stop = bar_sync_or(bar_half, 256, !ok) != 0;
     }
     float* const hdst = trans ? p.mt : p.ht;
@@ -1369,8 +1404,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tcx_kernel(const __grid_con
         if (is_consumer) {
             for (int b = 0; b < kBarsC; ++b) {
                 const uint32_t off = 8u * b;
-                const bool two = (off >= M_AFREE && off < M_VFULL) || (off >= M_NRM && off < M_OD);
-                // (M_OD: one commit per chunk and half)
+                const bool two = (off >= M_AFREE && off < M_VFULL) || (off >= M_NRM && off < M_NRM + 16);
                 mbar_init(bar_at(misc, off), two ? 2 : 1);
             }
             const uint32_t id = smid();
