@@ -333,21 +333,24 @@ def run_ours(args):
                                                 io=kda.KDA_IO_F32 if wl.io == "f32" else kda.KDA_IO_BF16)
         ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev) if ws_bytes else None
 
-        def step():
-            kda.chunk_fwd(q, k, v, d["g"], d["beta"], 1.0, h0=d["h0"], ht=ht, o=o,
+        def prefill(qq, kk, vv, gg, bb):
+            kda.chunk_fwd(qq, kk, vv, gg, bb, 1.0, h0=d["h0"], ht=ht, o=o,
                           cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], workspace=ws,
                           stream=stream)
         if args.workload == "long_256k_tp4":
             # too few (sequence, head) pairs to fill the GPU: the split prefill (stretch bounds,
-            # stretch states and transitions, the join, the stretches' outputs)
+            # stretches from a zero state with their transitions, the join, the correction)
             P, need = kda.chunk_fwd_split_plan(q, v, d["cu_seqlens"], d["cu_host"], 0)
             ws = torch.empty(need, dtype=torch.uint8, device=dev)
             launches_per_step = 4 if P > 1 else 1
 
-            def step():
-                kda.chunk_fwd_split(q, k, v, d["g"], d["beta"], 1.0, h0=d["h0"], ht=ht, o=o,
+            def prefill(qq, kk, vv, gg, bb):
+                kda.chunk_fwd_split(qq, kk, vv, gg, bb, 1.0, h0=d["h0"], ht=ht, o=o,
                                     cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"], n_split=P,
                                     workspace=ws, stream=stream)
+
+        def step():
+            prefill(q, k, v, d["g"], d["beta"])
         units = T_tot
         algo_bytes = prefill_bytes(T_tot, H, dk, dv, N, h0=d["h0"] is not None)
         wl_desc = dict(WL_DESC, varlen_prologue=f"varlen_prologue: 64 packed sequences "
@@ -403,9 +406,7 @@ def run_ours(args):
         def e2e_step():
             for nm in names:
                 dbuf[nm].copy_(host[nm], non_blocking=True)
-            kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], 1.0,
-                          h0=d["h0"], ht=ht, o=o, cu_seqlens=d["cu_seqlens"],
-                          cu_host=d["cu_host"], workspace=ws, stream=stream)
+            prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"])
             o_host.copy_(o, non_blocking=True)
             ht_host.copy_(ht, non_blocking=True)
         et = _events_time(torch, e2e_step, max(2, args.steps // 2), 2, stream=stream)
