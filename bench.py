@@ -38,7 +38,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # It is reported only while that kernel's sources hash to what was profiled.
 MEASURED_TRAFFIC = {
     "prefill_8k": (("chunk_tcx.cu", "tc.cuh", "common.cuh", "tma_host.h"),
-                   "0716dc2e7752154918079bf0d08a5f9add4073aca64e868a6b4dd04c972ee6fe", 392807168),
+                   "fb083c4b23146025607119dc4bd5b0292d087831482b6dbf0e1565890c8cc62b", 392144640),
     "conv_8k": (("conv.cu", "common.cuh"),
                 "28908a4c60fb3f184b90005e406d903129202d5acbbcbca4cb52243982fcf542", 365856512),
     "decode_256x32": (("recurrent_step.cu", "common.cuh"),
