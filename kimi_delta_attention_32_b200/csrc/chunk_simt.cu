@@ -25,6 +25,7 @@ constexpr int kC = 64;          // chunk length
 constexpr int kDVB = 32;        // value columns per CTA
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr float kLog2eS = 1.4426950408889634f;   // log2(e): gamma is kept in log2 units
 
 template <int DK>
 struct SimtSmem {
@@ -79,43 +80,41 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         }
         for (int r = tid; r < kC; r += kThreads) sm.beta[r] = r < L ? beta[(c0 + r) * H + h] : 0.f;
         __syncthreads();
-        // ---- gamma = in-chunk cumulative sum of g, per channel ----
+        // ---- gamma = in-chunk cumulative sum of g, per channel, in log2 units ----
         for (int c = tid; c < DK; c += kThreads) {
             float acc = 0.f;
-            for (int r = 0; r < kC; ++r) { acc += sm.gam[r][c]; sm.gam[r][c] = acc; }
+            for (int r = 0; r < kC; ++r) { acc += sm.gam[r][c]; sm.gam[r][c] = acc * kLog2eS; }
         }
         __syncthreads();
-        // ---- A and P: one warp per (r, i) pair, lanes over channels ----
-        for (int pidx = warp; pidx < kC * (kC + 1) / 2; pidx += kWarps) {
+        // ---- A and P: one thread per (r, i) pair (i <= r), channels visited from a per-lane
+        //      offset so that the row-strided reads of a warp fall in different banks ----
+        for (int pidx = tid; pidx < kC * (kC + 1) / 2; pidx += kThreads) {
             int r = (int)((sqrtf(8.f * pidx + 1.f) - 1.f) * 0.5f);
             while ((r + 1) * (r + 2) / 2 <= pidx) ++r;
             while (r * (r + 1) / 2 > pidx) --r;
             const int i = pidx - r * (r + 1) / 2;
             float a = 0.f, pp = 0.f;
-            for (int c = lane; c < DK; c += 32) {
-                const float e = expf(sm.gam[r][c] - sm.gam[i][c]);
-                const float ki = sm.k[i][c] * e;
+#pragma unroll 8
+            for (int cc = 0; cc < DK; ++cc) {
+                const int c = (cc + lane) & (DK - 1);
+                const float ki = sm.k[i][c] * exp2f(sm.gam[r][c] - sm.gam[i][c]);
                 a = fmaf(sm.k[r][c], ki, a);
                 pp = fmaf(sm.q[r][c], ki, pp);
             }
-            a = warp_sum(a);
-            pp = warp_sum(pp);
-            if (lane == 0) {
-                sm.A[r][i] = (i < r) ? a : 0.f;
-                sm.P[r][i] = pp;
-                if (i < r) sm.P[i][r] = 0.f;
-                sm.A[i][r] = 0.f;
-            }
+            sm.A[r][i] = (i < r) ? a : 0.f;
+            sm.P[r][i] = pp;
+            if (i < r) sm.P[i][r] = 0.f;
+            sm.A[i][r] = 0.f;
         }
         __syncthreads();
         // ---- W rhs = beta_r k_r exp(gamma_r); q <- q exp(gamma); k <- k exp(gamma_last - gamma) ----
         for (int e = tid; e < kC * DK; e += kThreads) {
             const int r = e / DK, c = e % DK;
             const float gr = sm.gam[r][c];
-            const float er = expf(gr);
+            const float er = exp2f(gr);
             sm.W[r][c] = sm.beta[r] * sm.k[r][c] * er;
             sm.q[r][c] *= er;
-            sm.k[r][c] *= expf(sm.gam[kC - 1][c] - gr);
+            sm.k[r][c] *= exp2f(sm.gam[kC - 1][c] - gr);
         }
         __syncthreads();
         // ---- forward substitution: X_r -= beta_r sum_{i<r} A[r,i] X_i ----
@@ -160,7 +159,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             const int j = lane;
             for (int c = warp; c < DK; c += kWarps) {
                 const float gl = sm.gam[kC - 1][c];
-                float acc = expf(gl) * sm.S[c][j];
+                float acc = exp2f(gl) * sm.S[c][j];
                 for (int r = 0; r < L; ++r) acc = fmaf(sm.k[r][c], sm.U[r][j], acc);
                 sm.S[c][j] = acc;
             }
