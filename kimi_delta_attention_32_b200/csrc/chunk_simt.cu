@@ -117,22 +117,31 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             sm.k[r][c] *= exp2f(sm.gam[kC - 1][c] - gr);
         }
         __syncthreads();
-        // ---- forward substitution: X_r -= beta_r sum_{i<r} A[r,i] X_i ----
-        for (int r = 1; r < L; ++r) {
-            const float br = sm.beta[r];
-            for (int col = tid; col < DK + kDVB; col += kThreads) {
-                float acc = 0.f;
-                if (col < DK) {
-                    for (int i = 0; i < r; ++i) acc = fmaf(sm.A[r][i], sm.W[i][col], acc);
-                    sm.W[r][col] -= br * acc;
-                } else {
-                    const int j = col - DK;
-                    for (int i = 0; i < r; ++i) acc = fmaf(sm.A[r][i], sm.U[i][j], acc);
-                    sm.U[r][j] -= br * acc;
+        // ---- forward substitution X_r -= beta_r sum_{i<r} A[r,i] X_i: columns of [W | U] are
+        //      independent, so one thread solves one column in registers, with no barrier
+        //      between rows (rows past L have beta = 0 and stay zero) ----
+        for (int col = tid; col < DK + kDVB; col += kThreads) {
+            const bool wcol = col < DK;
+            float* const xs = wcol ? &sm.W[0][col] : &sm.U[0][col - DK];
+            const int ld = wcol ? DK : kDVB;
+            float x[kC];
+#pragma unroll
+            for (int r = 0; r < kC; ++r) x[r] = xs[r * ld];
+#pragma unroll
+            for (int r = 1; r < kC; ++r) {
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int i = 0; i + 1 < r; i += 2) {
+                    a0 = fmaf(sm.A[r][i], x[i], a0);
+                    a1 = fmaf(sm.A[r][i + 1], x[i + 1], a1);
                 }
+                if (r & 1) a0 = fmaf(sm.A[r][r - 1], x[r - 1], a0);
+                x[r] -= sm.beta[r] * (a0 + a1);
             }
-            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < kC; ++r) xs[r * ld] = x[r];
         }
+        __syncthreads();
         // ---- Ut = U - W S  (thread: column j = lane, rows warp + 8m) ----
         {
             const int j = lane;
