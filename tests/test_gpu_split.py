@@ -202,3 +202,59 @@ def test_output_correct_matches_host_product():
     excess = np.abs(to64(o) - ref) / (2.0 ** -8 * np.abs(ref) + 2.0 ** -14 * mag)
     assert np.max(excess) <= 1.0, f"error {np.max(excess):.2f}x its bound"
     assert rel_l2(to64(o), ref) <= 2e-3
+
+
+def test_cross_rank_steps_through_the_abi():
+    """The cross-rank context-parallel steps on one GPU: two ranks' stretches (cut anywhere,
+    not at chunk bounds, one of them empty for a sequence) run through kda_chunk_states,
+    are stacked in the all-gather's order, joined by kda_state_scan with the rank-major index,
+    and corrected by kda_output_correct; the assembled outputs and final states must match the
+    whole-sequence oracle."""
+    lens = [700, 130, 95]
+    cuts = [300, 130, 1]                    # rank 0 takes the first cut tokens of each sequence
+    d = _inputs(lens, 2, 57)
+    cu = d["cu_host"]
+    parts = []
+    for r in range(2):
+        idx = torch.cat([torch.arange(cu[n] + (0 if r == 0 else cuts[n]),
+                                      cu[n] + (cuts[n] if r == 0 else lens[n]))
+                         for n in range(len(lens))]).to(DEV)
+        cu_r = [0]
+        for n in range(len(lens)):
+            cu_r.append(cu_r[-1] + (cuts[n] if r == 0 else lens[n] - cuts[n]))
+        sl = {x: d[x].index_select(0, idx).contiguous() for x in ("q", "k", "v", "g", "beta")}
+        cu_t = torch.tensor(cu_r, dtype=torch.int32, device=DEV)
+        z, m, o, w = kda.chunk_states(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], 1.0,
+                                      cu_seqlens=cu_t, cu_host=cu_r, output=True,
+                                      carried_queries=True)
+        parts.append((idx, cu_t, cu_r, z, m, o, w))
+    N = len(lens)
+    h_start, ht = kda.state_scan(torch.cat([p[4] for p in parts]), torch.cat([p[3] for p in parts]),
+                                 d["h0"], N=N, P=2, seq_stride=1, seg_stride=N)
+    o_full = torch.empty_like(d["v"])
+    for r, (idx, cu_t, cu_r, z, m, o, w) in enumerate(parts):
+        kda.output_correct(w, h_start[r * N:(r + 1) * N].contiguous(), o, cu_t, cu_r)
+        o_full.index_copy_(0, idx, o)
+    torch.cuda.synchronize()
+    _check_split(d, o_full, ht, "cross-rank steps, 2 ranks x 3 seqs x 2 heads")
+
+
+def test_chunk_fwd_cp_one_rank():
+    """cp.chunk_fwd_cp through its libkda steps and an NCCL group of one rank."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from kimi_delta_attention_32_b200 import cp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        d = _inputs([500, 64, 3], 2, 58)
+        o, ht = cp.chunk_fwd_cp(d["q"], d["k"], d["v"], d["g"], d["beta"], 1.0, h0=d["h0"],
+                                cu_seqlens=d["cu_seqlens"], cu_host=d["cu_host"])
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    _check_split(d, o, ht, "cp.chunk_fwd_cp, 1 rank x 3 seqs x 2 heads")
