@@ -415,8 +415,9 @@ def run_ours(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ems / len(et)}
 
-    # ---------------- other rows of the path, same run ----------------
-    if not args.no_rows and args.workload == "prefill_8k":
+    # ---------------- other rows of the path, same run (one GPU: they characterise the
+    # kernels, and under torchrun they would hold every GPU for minutes between collectives) ----
+    if not args.no_rows and args.workload == "prefill_8k" and world == 1:
         rows = measure_rows(torch, kda, dev, flush, hbm_peak, stream)
 
     cpu = None
