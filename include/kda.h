@@ -209,12 +209,14 @@ kda_status kda_output_correct(const void* w, const float* h, void* o, const int3
 
 /*
  * kda_chunk_fwd_split_workspace_size -- stretches per sequence and workspace bytes of
- * kda_chunk_fwd_split for this batch (host-only, apart from reading the device's SM count when
- * n_split == 0).
+ * kda_chunk_fwd_split for this batch. Host-only, except that n_split == 0 asks the current
+ * device, once per device, how many of the prefill's 4-SM clusters it holds at once
+ * (cudaOccupancyMaxActiveClusters; KDA_ERR_CUDA if that query fails).
  *  cu_seqlens_host, B, T, N: the batch as for kda_chunk_fwd (host data only).
  *  n_split: stretches per sequence, or 0 to choose: the split is taken when the (sequence,
- *  head) pairs leave most of the GPU's 4-SM clusters idle and the cost model (serial chunks
- *  per stretch, waves of clusters) gains more than 10%; 1 otherwise.
+ *  head) pairs leave most of those clusters idle and the cost model (serial chunks per
+ *  stretch, waves of clusters, the join and the output correction) gains more than 10%; 1
+ *  otherwise.
  *  n_split_out: host, receives the stretch count; bytes: host, receives the size.
  */
 kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_host, int B, int T,
