@@ -225,6 +225,17 @@ kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_host, in
                                               size_t* bytes);
 
 /*
+ * kda_chunk_fwd_split_plan -- kda_chunk_fwd_split_workspace_size for a device that holds
+ * resident_clusters of the prefill's 4-SM clusters at once (33 on a B200), with no device
+ * query: host-only, so a batch can be planned away from the GPU that runs it.
+ *  resident_clusters: > 0 when n_split == 0 (KDA_ERR_INVALID_ARG otherwise); unused when
+ *  n_split > 0. Other arguments and results as for kda_chunk_fwd_split_workspace_size.
+ */
+kda_status kda_chunk_fwd_split_plan(const int32_t* cu_seqlens_host, int B, int T, int N, int H,
+                                    int dk, int dv, int chunk, kda_io_dtype io, int n_split,
+                                    int resident_clusters, int* n_split_out, size_t* bytes);
+
+/*
  * kda_chunk_fwd_split -- kda_chunk_fwd with every sequence split into stretches of whole
  * chunks that run side by side (context parallelism inside one GPU; same sources as
  * kda_chunk_states). Four launches on the stream: the stretch bounds; every stretch from a

@@ -79,26 +79,31 @@ SplitLayout split_layout(int N, int64_t T_tot, int P, int H, int dk, int dv) {
 // and one cluster of 4 SMs carries one (stretch, head) at a time; `clusters` of them fit on the
 // GPU at once (33 on a B200: clusters are placed within GPCs). The split runs 2 U P units
 // (outputs and end states from zero, and the transitions) over stretches P times shorter; it
-// pays when U = N H units leave most clusters idle. Cost in chunk steps (~2 us each): one per
-// stretch for the join, and the output correction, an HBM-bound pass of 768 bytes per token and
-// head (~1/16384 of a step). The split is taken only for a gain above 10%.
+// pays when U = N H units leave most clusters idle. Cost in chunk steps (~2 us each):
+//  - per wave of clusters, the longest stretch plus the pipeline's fill and drain (measured:
+//    a 128-chunk prefill spans 141 steps of its steady period, so 12 per wave);
+//  - one step per stretch for the join;
+//  - the output correction, an HBM-bound pass of 768 bytes per token and head (~1/16384 step).
+// The cheapest count is taken if it gains more than 10% over one stretch.
 int auto_split(int64_t longest, int64_t T_tot, int H, int64_t units, int clusters) {
+    constexpr int64_t kFill = 12;
     if (units <= 0 || longest <= 0 || clusters <= 0) return 1;
     const int64_t chunks = (longest + 63) / 64;
     auto waves = [&](int64_t u) { return (u + clusters - 1) / clusters; };
     const int64_t correct = T_tot * H / 16384 + 1;
+    const int64_t unsplit = waves(units) * (chunks + kFill);
     int best_p = 1;
-    int64_t best = waves(units) * chunks;
+    int64_t best = unsplit;
     for (int P = 2; P <= 64; ++P) {
         const int64_t per = (chunks + P - 1) / P;
         if (per < 2) break;
-        const int64_t cost = waves(2 * units * P) * per + P + correct;
-        if (10 * cost < 9 * best) {
+        const int64_t cost = waves(2 * units * P) * (per + kFill) + P + correct;
+        if (cost < best) {
             best = cost;
             best_p = P;
         }
     }
-    return best_p;
+    return 10 * best < 9 * unsplit ? best_p : 1;
 }
 
 }  // namespace
@@ -273,12 +278,12 @@ KDA_API kda_status kda_output_correct(const void* w, const float* h, void* o,
     return from_cuda(kda::launch_stretch_correct(c, static_cast<cudaStream_t>(stream)));
 }
 
-KDA_API kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_host, int B, int T,
-                                                      int N, int H, int dk, int dv, int chunk,
-                                                      kda_io_dtype io, int n_split, int* n_split_out,
-                                                      size_t* bytes) {
+KDA_API kda_status kda_chunk_fwd_split_plan(const int32_t* cu_seqlens_host, int B, int T, int N,
+                                            int H, int dk, int dv, int chunk, kda_io_dtype io,
+                                            int n_split, int resident_clusters, int* n_split_out,
+                                            size_t* bytes) {
     if (bytes == nullptr || n_split_out == nullptr || n_split < 0 || H <= 0 || dk <= 0 || dv <= 0 ||
-        chunk <= 0)
+        chunk <= 0 || (n_split == 0 && resident_clusters <= 0))
         return KDA_ERR_INVALID_ARG;
     if (io != KDA_IO_F32 && io != KDA_IO_BF16) return KDA_ERR_INVALID_ARG;
     if (cu_seqlens_host == nullptr ? (B < 0 || T < 0) : N < 0) return KDA_ERR_INVALID_ARG;
@@ -294,15 +299,24 @@ KDA_API kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_
             if (len > longest) longest = len;
         }
     }
-    int P = n_split;
-    if (P == 0) {
-        const int slots = kda::chunk_tcx_cluster_slots();
-        if (slots == 0) return KDA_ERR_CUDA;
-        P = auto_split(longest, T_tot, H, (int64_t)Nn * H, slots);
-    }
+    const int P = n_split > 0 ? n_split : auto_split(longest, T_tot, H, (int64_t)Nn * H, resident_clusters);
     *n_split_out = P;
     *bytes = P == 1 ? kda::chunk_tcx_workspace_bytes() : split_layout(Nn, T_tot, P, H, dk, dv).total;
     return KDA_OK;
+}
+
+KDA_API kda_status kda_chunk_fwd_split_workspace_size(const int32_t* cu_seqlens_host, int B, int T,
+                                                      int N, int H, int dk, int dv, int chunk,
+                                                      kda_io_dtype io, int n_split, int* n_split_out,
+                                                      size_t* bytes) {
+    // the resident cluster count matters only for n_split == 0 on the cluster path
+    int slots = 1;
+    if (n_split == 0 && H > 0 && cluster_prefill_path(io, dk, dv, chunk)) {
+        slots = kda::chunk_tcx_cluster_slots();
+        if (slots == 0) return KDA_ERR_CUDA;
+    }
+    return kda_chunk_fwd_split_plan(cu_seqlens_host, B, T, N, H, dk, dv, chunk, io, n_split, slots,
+                                    n_split_out, bytes);
 }
 
 KDA_API kda_status kda_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,

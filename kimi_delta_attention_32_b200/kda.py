@@ -24,7 +24,8 @@ EXPORTED = ("kda_status_string", "kda_version", "kda_conv_fwd", "kda_chunk_fwd_w
             "kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_fwd_noalloc", "kda_recurrent_step",
             "kda_conv_recurrent_step", "kda_fused_recurrent_step", "kda_set_wait_limit",
             "kda_last_device_error", "kda_chunk_states", "kda_state_scan",
-            "kda_chunk_fwd_split_workspace_size", "kda_chunk_fwd_split", "kda_output_correct")
+            "kda_chunk_fwd_split_workspace_size", "kda_chunk_fwd_split", "kda_output_correct",
+            "kda_chunk_fwd_split_plan")
 
 _lock = threading.Lock()
 _lib = None
@@ -99,6 +100,9 @@ def load_library(path: str = LIB_PATH):
         lib.kda_chunk_fwd_split.restype = ci
         lib.kda_output_correct.argtypes = [vp, fp, vp, i32p, cip, ci, ci, ci, ci, ci, ci, ci, vp]
         lib.kda_output_correct.restype = ci
+        lib.kda_chunk_fwd_split_plan.argtypes = [cip, ci, ci, ci, ci, ci, ci, ci, ci, ci, ci,
+                                                 ctypes.POINTER(ci), ctypes.POINTER(cs)]
+        lib.kda_chunk_fwd_split_plan.restype = ci
         if path == LIB_PATH:
             _lib = lib
         return lib

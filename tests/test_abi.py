@@ -342,3 +342,36 @@ def test_output_correct_checks_arguments(lib):
     assert corr(dk=64) == kda.KDA_ERR_UNSUPPORTED
     assert corr(cu=None, cuh=None) == kda.KDA_ERR_UNSUPPORTED            # padded: not supported
     del keep
+
+
+def _plan(lib, cuh=None, B=1, T=8192, N=0, H=32, n_split=0, clusters=33):
+    P, out = ctypes.c_int(0), ctypes.c_size_t(0)
+    st = lib.kda_chunk_fwd_split_plan(cuh, B, T, N, H, 128, 128, 64, 1, n_split, clusters,
+                                      ctypes.byref(P), ctypes.byref(out))
+    return st, P.value, out.value
+
+
+def test_split_plan_choices(lib):
+    """The split's cost model on a B200 (33 resident 4-SM clusters), host-only: the benchmark's
+    workloads with 32 heads keep one stretch; the 8 heads of one of four tensor-parallel GPUs
+    over 262144 tokens split in two (measured 4.7 ms against 8.4 ms unsplit); 4 heads split in
+    four; a GPU that 8 heads already fill does not split."""
+    assert _plan(lib, T=8192, H=32)[:2] == (kda.KDA_OK, 1)              # prefill_8k
+    assert _plan(lib, T=262144, H=32)[:2] == (kda.KDA_OK, 1)            # long_256k
+    assert _plan(lib, T=262144, H=8)[:2] == (kda.KDA_OK, 2)             # long_256k_tp4
+    assert _plan(lib, T=262144, H=4)[:2] == (kda.KDA_OK, 4)
+    assert _plan(lib, T=262144, H=8, clusters=8)[:2] == (kda.KDA_OK, 1)
+    assert _plan(lib, T=256, H=2)[:2] == (kda.KDA_OK, 1)                # too short to pay
+    lens = [128 + (97 * i) % 16257 for i in range(64)]                   # a varlen batch
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    keep, cuh = _cu_host(cu)
+    assert _plan(lib, cuh=cuh, B=0, T=0, N=64, H=32)[:2] == (kda.KDA_OK, 1)
+    del keep
+    # the same sizes as the device query reports for a given count
+    st, P, nbytes = _plan(lib, T=262144, H=8)
+    st2, P2, nbytes2 = _plan(lib, T=262144, H=8, n_split=2, clusters=0)   # count unused
+    assert (st2, P2, nbytes2) == (st, P, nbytes)
+    assert _plan(lib, clusters=0)[0] == kda.KDA_ERR_INVALID_ARG          # n_split 0 needs a count
+    assert _plan(lib, clusters=-3)[0] == kda.KDA_ERR_INVALID_ARG
