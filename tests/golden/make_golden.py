@@ -1,4 +1,5 @@
-"""Writes tests/golden/kda_tiny.json: a tiny fixed KDA case and the oracle's outputs.
+"""Writes tests/golden/kda_tiny.json: a tiny fixed KDA case and the oracle's outputs (o, the
+final state, and the transition of the whole sequence).
 
 The pages about the model print no worked numeric example for KDA, so this fixture is
 a regression pin only: its inputs are small exact decimals chosen here, and its
@@ -35,8 +36,9 @@ def case():
 if __name__ == "__main__":
     c = case()
     o, ht = oracle.kda_fwd(c["q"], c["k"], c["v"], c["g"], c["beta"], c["scale"], c["h0"])
+    m = oracle.transition(c["k"], c["g"], c["beta"])
     out = {k: np.asarray(v).tolist() for k, v in c.items() if k != "scale"}
-    out.update(scale=c["scale"], o=o.tolist(), ht=ht.tolist())
+    out.update(scale=c["scale"], o=o.tolist(), ht=ht.tolist(), m=m.tolist())
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "kda_tiny.json")
     with open(path, "w") as f:
         json.dump(out, f, indent=1)

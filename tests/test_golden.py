@@ -17,3 +17,5 @@ def test_oracle_reproduces_golden_tiny(oracle_lib):
                            arr["h0"], lib=oracle_lib)
     np.testing.assert_allclose(o, arr["o"], rtol=0, atol=1e-15)
     np.testing.assert_allclose(ht, arr["ht"], rtol=0, atol=1e-15)
+    m = oracle.transition(arr["k"], arr["g"], arr["beta"], lib=oracle_lib)
+    np.testing.assert_allclose(m, arr["m"], rtol=0, atol=1e-15)
